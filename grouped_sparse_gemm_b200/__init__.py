@@ -1,0 +1,323 @@
+"""grouped_sparse_gemm_b200 -- grouped paired-4:8 NVFP4 expert GEMM for routed MoE on B200.
+
+Thin Python binding over the C ABI of ``libgsg.so`` (declared in ``include/gsg.h``).  The
+functions keep the ABI's names without the ``gsg_`` prefix and only marshal arguments: torch
+provides device memory and the current stream, every step runs in the library's CUDA kernels.
+There is no CPU fallback: if the library is missing or no GPU is present the calls raise.
+
+The path (after "Hardware-Native Joint Sparse-Quantization for Trillion-Scale Mixture-of-Experts",
+paperlayer.ai summary, §3.4 and §D.1): pack_sparse_nvfp4 (offline weights) ->
+moe_route_permute -> quantize_act_nvfp4 -> grouped_sparse_gemm -> unpermute_scale.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+from . import _build
+
+__all__ = [
+    "GsgError", "lib", "load_library", "library_path",
+    "PackedSparseWeights", "PackedDenseWeights", "Routing", "QuantizedActivations",
+    "pack_sparse_nvfp4", "pack_dense_nvfp4", "moe_route_permute", "quantize_act_nvfp4",
+    "grouped_sparse_gemm", "grouped_dense_gemm", "unpermute_scale", "get_device_status",
+    "act_scales_bytes", "workspace_size", "OP_PACK_SPARSE", "OP_PACK_DENSE", "OP_ROUTE",
+    "OP_QUANTIZE", "OP_GEMM", "EXPORTED_SYMBOLS",
+]
+
+OP_PACK_SPARSE, OP_PACK_DENSE, OP_ROUTE, OP_QUANTIZE, OP_GEMM = 1, 2, 3, 4, 5
+OUT_BF16, OUT_F32 = 0, 1
+ACT_SCALE_PAD_ROWS = 256
+
+EXPORTED_SYMBOLS = [
+    "gsg_sparse_values_bytes", "gsg_sparse_meta_bytes", "gsg_weight_scales_bytes",
+    "gsg_dense_codes_bytes", "gsg_act_codes_bytes", "gsg_act_scales_bytes", "gsg_workspace_size",
+    "gsg_pack_sparse_nvfp4", "gsg_pack_dense_nvfp4", "gsg_moe_route_permute",
+    "gsg_quantize_act_nvfp4", "gsg_grouped_sparse_gemm", "gsg_grouped_dense_gemm",
+    "gsg_unpermute_scale", "gsg_get_device_status", "gsg_status_string", "gsg_version",
+]
+
+_STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported shape", -3: "CUDA error",
+           -4: "bad routing", -5: "non-finite input", -6: "device timeout", -7: "workspace"}
+
+
+class GsgError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {_STATUS.get(status, status)} ({status})")
+        self.status = status
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def load_library(build_if_missing: bool = False) -> ctypes.CDLL:
+    """Load libgsg.so (optionally compiling it first).  Raises when it is not there."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = library_path()
+    if not os.path.exists(path):
+        if not build_if_missing:
+            raise RuntimeError(f"libgsg.so is not built ({path}); run grouped_sparse_gemm_b200._build.build()")
+        _build.build()
+    L = ctypes.CDLL(path)
+    vp, i, sz, fp = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
+    sig = {
+        "gsg_sparse_values_bytes": (sz, [i, i, i]),
+        "gsg_sparse_meta_bytes": (sz, [i, i, i]),
+        "gsg_weight_scales_bytes": (sz, [i, i, i, i]),
+        "gsg_dense_codes_bytes": (sz, [i, i, i]),
+        "gsg_act_codes_bytes": (sz, [i, i]),
+        "gsg_act_scales_bytes": (sz, [i, i, i]),
+        "gsg_workspace_size": (sz, [i, i, i, i, i, i]),
+        "gsg_pack_sparse_nvfp4": (i, [vp, i, i, i, vp, vp, vp, fp, vp, sz, vp]),
+        "gsg_pack_dense_nvfp4": (i, [vp, i, i, i, vp, vp, fp, vp, sz, vp]),
+        "gsg_moe_route_permute": (i, [vp, i, i, i, vp, vp, vp, vp, sz, vp]),
+        "gsg_quantize_act_nvfp4": (i, [vp, i, i, i, vp, i, vp, vp, vp, vp, vp, sz, vp]),
+        "gsg_grouped_sparse_gemm": (i, [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, i, vp]),
+        "gsg_grouped_dense_gemm": (i, [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, i, vp]),
+        "gsg_unpermute_scale": (i, [vp, vp, vp, i, i, i, vp, vp]),
+        "gsg_get_device_status": (i, [vp]),
+        "gsg_status_string": (ctypes.c_char_p, [i]),
+        "gsg_version": (i, []),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = L
+    return L
+
+
+def lib() -> ctypes.CDLL:
+    return load_library()
+
+
+# ------------------------------------------------------------------ helpers
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream: Optional[torch.cuda.Stream] = None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn: str, st: int):
+    if st != 0:
+        raise GsgError(fn, st)
+
+
+def _need_cuda(*ts: Optional[torch.Tensor]):
+    for t in ts:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("grouped_sparse_gemm_b200 works on CUDA tensors only (no CPU fallback)")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def workspace_size(op: int, E: int = 0, N: int = 0, K: int = 0, T: int = 0, k: int = 1) -> int:
+    return int(lib().gsg_workspace_size(op, E, N, K, T, k))
+
+
+def act_scales_bytes(R: int, K: int, sf_block: int) -> int:
+    return int(lib().gsg_act_scales_bytes(R, K, sf_block))
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+
+
+# ------------------------------------------------------------------ packed containers
+@dataclass
+class PackedSparseWeights:
+    values: torch.Tensor   # uint8 [E*N*K/4]
+    meta: torch.Tensor     # uint8 [E*N*K/16]
+    scales: torch.Tensor   # uint8 [E*N*K/32]
+    w_scale: torch.Tensor  # fp32 [E]
+    E: int
+    N: int
+    K: int
+
+    def nbytes(self) -> int:
+        return self.values.numel() + self.meta.numel() + self.scales.numel()
+
+
+@dataclass
+class PackedDenseWeights:
+    codes: torch.Tensor    # uint8 [E*N*K/2]
+    scales: torch.Tensor   # uint8 [E*N*K/16]
+    w_scale: torch.Tensor  # fp32 [E]
+    E: int
+    N: int
+    K: int
+
+    def nbytes(self) -> int:
+        return self.codes.numel() + self.scales.numel()
+
+
+@dataclass
+class Routing:
+    offsets: torch.Tensor   # int32 [E+1]
+    perm_src: torch.Tensor  # int32 [R]
+    inv_perm: torch.Tensor  # int32 [R]
+    T: int
+    k: int
+    E: int
+
+
+@dataclass
+class QuantizedActivations:
+    codes: torch.Tensor     # uint8 [R, K/2]
+    scales: torch.Tensor    # uint8, quad layout
+    x_scale: torch.Tensor   # fp32 [1]
+    R: int
+    K: int
+    sf_block: int
+
+
+# ------------------------------------------------------------------ entry points
+def pack_sparse_nvfp4(W: torch.Tensor, out: Optional[PackedSparseWeights] = None,
+                      workspace: Optional[torch.Tensor] = None, stream=None) -> PackedSparseWeights:
+    """W fp32 [E, N, K] -> paired 4:8 NVFP4 packed weights (gsg_pack_sparse_nvfp4)."""
+    _need_cuda(W)
+    assert W.dtype == torch.float32 and W.dim() == 3
+    E, N, K = W.shape
+    L = lib()
+    dev = W.device
+    if out is None:
+        out = PackedSparseWeights(
+            values=torch.empty(L.gsg_sparse_values_bytes(E, N, K), dtype=torch.uint8, device=dev),
+            meta=torch.empty(L.gsg_sparse_meta_bytes(E, N, K), dtype=torch.uint8, device=dev),
+            scales=torch.empty(L.gsg_weight_scales_bytes(E, N, K, 32), dtype=torch.uint8, device=dev),
+            w_scale=torch.empty(E, dtype=torch.float32, device=dev), E=E, N=N, K=K)
+    need = workspace_size(OP_PACK_SPARSE, E, N, K)
+    ws = workspace if workspace is not None else _workspace(need, dev)
+    _check("gsg_pack_sparse_nvfp4", L.gsg_pack_sparse_nvfp4(
+        _ptr(W), E, N, K, _ptr(out.values), _ptr(out.meta), _ptr(out.scales), _ptr(out.w_scale),
+        _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def pack_dense_nvfp4(W: torch.Tensor, out: Optional[PackedDenseWeights] = None,
+                     workspace: Optional[torch.Tensor] = None, stream=None) -> PackedDenseWeights:
+    """W fp32 [E, N, K] -> dense NVFP4 (16-element blocks) for the control GEMM."""
+    _need_cuda(W)
+    assert W.dtype == torch.float32 and W.dim() == 3
+    E, N, K = W.shape
+    L = lib()
+    dev = W.device
+    if out is None:
+        out = PackedDenseWeights(
+            codes=torch.empty(L.gsg_dense_codes_bytes(E, N, K), dtype=torch.uint8, device=dev),
+            scales=torch.empty(L.gsg_weight_scales_bytes(E, N, K, 16), dtype=torch.uint8, device=dev),
+            w_scale=torch.empty(E, dtype=torch.float32, device=dev), E=E, N=N, K=K)
+    need = workspace_size(OP_PACK_DENSE, E, N, K)
+    ws = workspace if workspace is not None else _workspace(need, dev)
+    _check("gsg_pack_dense_nvfp4", L.gsg_pack_dense_nvfp4(
+        _ptr(W), E, N, K, _ptr(out.codes), _ptr(out.scales), _ptr(out.w_scale),
+        _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def moe_route_permute(topk_ids: torch.Tensor, E: int, out: Optional[Routing] = None,
+                      workspace: Optional[torch.Tensor] = None, stream=None) -> Routing:
+    """topk ids int32 [T, k] -> expert offsets, perm_src, inv_perm (gsg_moe_route_permute)."""
+    _need_cuda(topk_ids)
+    assert topk_ids.dtype == torch.int32 and topk_ids.dim() == 2
+    T, k = topk_ids.shape
+    dev = topk_ids.device
+    if out is None:
+        out = Routing(offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+                      perm_src=torch.empty(max(T * k, 1), dtype=torch.int32, device=dev),
+                      inv_perm=torch.empty(max(T * k, 1), dtype=torch.int32, device=dev), T=T, k=k, E=E)
+    need = workspace_size(OP_ROUTE, E, 0, 0, T, k)
+    ws = workspace if workspace is not None else (_workspace(need, dev) if need else None)
+    _check("gsg_moe_route_permute", lib().gsg_moe_route_permute(
+        _ptr(topk_ids), T, k, E, _ptr(out.offsets), _ptr(out.perm_src), _ptr(out.inv_perm),
+        _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+    return out
+
+
+def quantize_act_nvfp4(X: torch.Tensor, sf_block: int = 32, inv_perm: Optional[torch.Tensor] = None,
+                       top_k: int = 1, x_scale_in: Optional[torch.Tensor] = None,
+                       out: Optional[QuantizedActivations] = None,
+                       workspace: Optional[torch.Tensor] = None, stream=None) -> QuantizedActivations:
+    """X bf16 [T, K] -> NVFP4 codes/scales in routed row order (gsg_quantize_act_nvfp4)."""
+    _need_cuda(X, inv_perm, x_scale_in)
+    assert X.dtype == torch.bfloat16 and X.dim() == 2
+    T, K = X.shape
+    R = T * top_k
+    dev = X.device
+    if out is None:
+        out = QuantizedActivations(
+            codes=torch.empty(max(R, 1), K // 2, dtype=torch.uint8, device=dev),
+            scales=torch.empty(act_scales_bytes(R, K, sf_block), dtype=torch.uint8, device=dev),
+            x_scale=torch.empty(1, dtype=torch.float32, device=dev), R=R, K=K, sf_block=sf_block)
+    need = workspace_size(OP_QUANTIZE, 0, 0, K, T, top_k)
+    ws = workspace if workspace is not None else _workspace(need, dev)
+    _check("gsg_quantize_act_nvfp4", lib().gsg_quantize_act_nvfp4(
+        _ptr(X), T, K, sf_block, _ptr(inv_perm), top_k, _ptr(x_scale_in), _ptr(out.codes),
+        _ptr(out.scales), _ptr(out.x_scale), _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def grouped_sparse_gemm(act: QuantizedActivations, w: PackedSparseWeights, offsets: torch.Tensor,
+                        max_rows_per_expert: int = -1, out: Optional[torch.Tensor] = None,
+                        out_dtype: torch.dtype = torch.bfloat16, stream=None) -> torch.Tensor:
+    """Y [R, N] = per-expert X_e . W_e^T on paired 4:8 NVFP4 weights (gsg_grouped_sparse_gemm)."""
+    assert act.sf_block == 32 and act.K == w.K
+    _need_cuda(act.codes, act.scales, offsets)
+    if out is None:
+        out = torch.empty(max(act.R, 1), w.N, dtype=out_dtype, device=act.codes.device)
+    ydt = OUT_F32 if out.dtype == torch.float32 else OUT_BF16
+    _check("gsg_grouped_sparse_gemm", lib().gsg_grouped_sparse_gemm(
+        _ptr(act.codes), _ptr(act.scales), _ptr(act.x_scale), _ptr(w.values), _ptr(w.meta),
+        _ptr(w.scales), _ptr(w.w_scale), _ptr(offsets), w.E, w.N, w.K, act.R, max_rows_per_expert,
+        _ptr(out), ydt, _stream(stream)))
+    return out
+
+
+def grouped_dense_gemm(act: QuantizedActivations, w: PackedDenseWeights, offsets: torch.Tensor,
+                       max_rows_per_expert: int = -1, out: Optional[torch.Tensor] = None,
+                       out_dtype: torch.dtype = torch.bfloat16, stream=None) -> torch.Tensor:
+    """Dense-NVFP4 control on the same skeleton (gsg_grouped_dense_gemm)."""
+    assert act.sf_block == 16 and act.K == w.K
+    _need_cuda(act.codes, act.scales, offsets)
+    if out is None:
+        out = torch.empty(max(act.R, 1), w.N, dtype=out_dtype, device=act.codes.device)
+    ydt = OUT_F32 if out.dtype == torch.float32 else OUT_BF16
+    _check("gsg_grouped_dense_gemm", lib().gsg_grouped_dense_gemm(
+        _ptr(act.codes), _ptr(act.scales), _ptr(act.x_scale), _ptr(w.codes), _ptr(w.scales),
+        _ptr(w.w_scale), _ptr(offsets), w.E, w.N, w.K, act.R, max_rows_per_expert,
+        _ptr(out), ydt, _stream(stream)))
+    return out
+
+
+def unpermute_scale(Y: torch.Tensor, inv_perm: torch.Tensor, gates: torch.Tensor, top_k: int,
+                    out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """out[t] = bf16(sum_j gates[t, j] * Y[inv_perm[t*k + j]]) (gsg_unpermute_scale)."""
+    _need_cuda(Y, inv_perm, gates)
+    assert Y.dtype == torch.bfloat16 and gates.dtype == torch.float32
+    T = gates.shape[0]
+    N = Y.shape[1]
+    if out is None:
+        out = torch.empty(T, N, dtype=torch.bfloat16, device=Y.device)
+    _check("gsg_unpermute_scale", lib().gsg_unpermute_scale(
+        _ptr(Y), _ptr(inv_perm), _ptr(gates), T, top_k, N, _ptr(out), _stream(stream)))
+    return out
+
+
+def get_device_status(stream=None) -> int:
+    """Synchronise the stream; return and clear the device status word (0 = ok)."""
+    return int(lib().gsg_get_device_status(_stream(stream)))

@@ -1,0 +1,236 @@
+// gsg_api.cu -- the exported C ABI (include/gsg.h): argument checks, per-device state,
+// device status word, launches.  Every entry point returns before launching anything when
+// an argument is invalid.
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "gsg_internal.cuh"
+#include "gsg_launch.h"
+
+namespace {
+
+__device__ int g_device_status;  // sticky first device-side error of this device
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  bool ready = false;
+  int* status = nullptr;
+  int num_sms = 0;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+
+// Per-device set-up on first use (needs that device current): status word address, SM count,
+// shared-memory limits of the kernels that need more than 48 KB.
+gsg_status_t device_state(DeviceState** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GSG_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceState& d = g_dev[dev];
+  if (!d.ready) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return GSG_ERR_CUDA;
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return GSG_ERR_CUDA;
+    if (gsg::route_set_smem_attrs() != cudaSuccess) return GSG_ERR_CUDA;
+    if (gsg::gemm_set_smem_attrs() != cudaSuccess) return GSG_ERR_CUDA;
+    d.status = static_cast<int*>(p);
+    d.num_sms = sms;
+    d.ready = true;
+  }
+  *out = &d;
+  return GSG_OK;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+inline gsg_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? GSG_OK : GSG_ERR_CUDA; }
+
+bool weight_shape_ok(int E, int N, int K) {
+  return E >= 1 && N >= 128 && K >= 256 && N % 128 == 0 && K % 256 == 0;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t gsg_sparse_values_bytes(int E, int N, int K) { return (size_t)E * N * K / 4; }
+size_t gsg_sparse_meta_bytes(int E, int N, int K) { return (size_t)E * N * K / 16; }
+size_t gsg_weight_scales_bytes(int E, int N, int K, int sf_block) {
+  return sf_block > 0 ? (size_t)E * N * K / sf_block : 0;
+}
+size_t gsg_dense_codes_bytes(int E, int N, int K) { return (size_t)E * N * K / 2; }
+size_t gsg_act_codes_bytes(int R, int K) { return (size_t)R * K / 2; }
+size_t gsg_act_scales_bytes(int R, int K, int sf_block) {
+  if (sf_block <= 0) return 0;
+  return (size_t)(K / (4 * sf_block)) * (size_t)(R + gsg::kActScalePadRows) * 16;
+}
+
+size_t gsg_workspace_size(int op, int E, int N, int K, int T, int k) {
+  switch (op) {
+    case GSG_OP_PACK_SPARSE:
+    case GSG_OP_PACK_DENSE:
+      if (E < 1 || N < 1 || K < 8) return 0;
+      return (size_t)E * gsg::pack_partials_per_expert(N, K) * sizeof(float);
+    case GSG_OP_ROUTE:
+      if (E < 1 || T < 0 || k < 1) return 0;
+      return gsg::route_workspace_bytes(T * k, E);
+    case GSG_OP_QUANTIZE:
+      if (T < 0 || K < 1) return 0;
+      return (size_t)gsg::quant_partials((long long)T * K) * sizeof(float);
+    default:
+      return 0;
+  }
+}
+
+static gsg_status_t pack_common(bool sparse, const float* W, int E, int N, int K, uint8_t* values, uint8_t* meta,
+                                uint8_t* scales, float* w_tensor_scale, void* ws, size_t ws_bytes, void* stream) {
+  if (!W || !values || !scales || !w_tensor_scale || (sparse && !meta)) return GSG_ERR_INVALID_ARG;
+  if (!weight_shape_ok(E, N, K)) return GSG_ERR_UNSUPPORTED_SHAPE;
+  if (E > 65535) return GSG_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(W) || !aligned16(values) || (sparse && !aligned16(meta))) return GSG_ERR_INVALID_ARG;
+  const size_t need = gsg_workspace_size(sparse ? GSG_OP_PACK_SPARSE : GSG_OP_PACK_DENSE, E, N, K, 0, 1);
+  if (ws == nullptr || ws_bytes < need) return GSG_ERR_WORKSPACE;
+  DeviceState* d = nullptr;
+  gsg_status_t st = device_state(&d);
+  if (st != GSG_OK) return st;
+  return from_cuda(gsg::launch_pack(sparse, W, E, N, K, values, meta, scales, w_tensor_scale,
+                                    static_cast<float*>(ws), d->status, as_stream(stream)));
+}
+
+gsg_status_t gsg_pack_sparse_nvfp4(const float* W, int E, int N, int K, uint8_t* values, uint8_t* meta,
+                                   uint8_t* scales, float* w_tensor_scale, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+  return pack_common(true, W, E, N, K, values, meta, scales, w_tensor_scale, workspace, workspace_bytes, stream);
+}
+
+gsg_status_t gsg_pack_dense_nvfp4(const float* W, int E, int N, int K, uint8_t* codes, uint8_t* scales,
+                                  float* w_tensor_scale, void* workspace, size_t workspace_bytes, void* stream) {
+  return pack_common(false, W, E, N, K, codes, nullptr, scales, w_tensor_scale, workspace, workspace_bytes, stream);
+}
+
+gsg_status_t gsg_moe_route_permute(const int32_t* topk_ids, int T, int k, int E, int32_t* expert_offsets,
+                                   int32_t* perm_src, int32_t* inv_perm, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+  if (T < 0 || k < 1) return GSG_ERR_INVALID_ARG;
+  if (!gsg::route_supported(E)) return GSG_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)T * k > (1ll << 30)) return GSG_ERR_UNSUPPORTED_SHAPE;
+  if (!expert_offsets) return GSG_ERR_INVALID_ARG;
+  if (T > 0 && (!topk_ids || !perm_src || !inv_perm)) return GSG_ERR_INVALID_ARG;
+  const size_t need = gsg::route_workspace_bytes(T * k, E);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return GSG_ERR_WORKSPACE;
+  DeviceState* d = nullptr;
+  gsg_status_t st = device_state(&d);
+  if (st != GSG_OK) return st;
+  return from_cuda(gsg::launch_route(topk_ids, T * k, E, expert_offsets, perm_src, inv_perm, workspace, d->status,
+                                     as_stream(stream)));
+}
+
+gsg_status_t gsg_quantize_act_nvfp4(const uint16_t* X, int T, int K, int sf_block, const int32_t* inv_perm, int k,
+                                    const float* x_tensor_scale_in, uint8_t* codes, uint8_t* scales,
+                                    float* x_tensor_scale_out, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+  if (T < 0 || k < 1 || (sf_block != 16 && sf_block != 32)) return GSG_ERR_INVALID_ARG;
+  if (K < 256 || K % 256 != 0) return GSG_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)T * k > (1ll << 30)) return GSG_ERR_UNSUPPORTED_SHAPE;
+  if (inv_perm == nullptr && k != 1) return GSG_ERR_INVALID_ARG;
+  if (!scales || !x_tensor_scale_out) return GSG_ERR_INVALID_ARG;
+  if (T > 0 && (!X || !codes)) return GSG_ERR_INVALID_ARG;
+  if ((X && !aligned16(X)) || (codes && !aligned16(codes)) || !aligned16(scales)) return GSG_ERR_INVALID_ARG;
+  if (x_tensor_scale_in == nullptr) {
+    const size_t need = gsg_workspace_size(GSG_OP_QUANTIZE, 0, 0, K, T, k);
+    if (workspace == nullptr || workspace_bytes < need) return GSG_ERR_WORKSPACE;
+  }
+  DeviceState* d = nullptr;
+  gsg_status_t st = device_state(&d);
+  if (st != GSG_OK) return st;
+  return from_cuda(gsg::launch_quant(X, T, K, sf_block, inv_perm, k, x_tensor_scale_in, codes, scales,
+                                     x_tensor_scale_out, static_cast<float*>(workspace), d->status, d->num_sms,
+                                     as_stream(stream)));
+}
+
+static gsg_status_t gemm_common(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, const float* x_scale,
+                                const uint8_t* w_vals, const uint8_t* w_meta, const uint8_t* w_scales,
+                                const float* w_scale, const int32_t* off, int E, int N, int K, int R, int max_rows,
+                                void* Y, int y_dtype, void* stream) {
+  if (R < 0 || (y_dtype != GSG_OUT_BF16 && y_dtype != GSG_OUT_F32)) return GSG_ERR_INVALID_ARG;
+  if (!weight_shape_ok(E, N, K) || !gsg::gemm_supported(E)) return GSG_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)R > (1ll << 30)) return GSG_ERR_UNSUPPORTED_SHAPE;
+  if (!off || !w_vals || !w_scales || !w_scale || !x_scale || (sparse && !w_meta)) return GSG_ERR_INVALID_ARG;
+  if (R == 0) return GSG_OK;  // nothing routed: nothing to compute or write
+  if (!a_codes || !a_scales || !Y) return GSG_ERR_INVALID_ARG;
+  if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(w_vals) || !aligned16(w_scales) ||
+      (sparse && !aligned16(w_meta)))
+    return GSG_ERR_INVALID_ARG;
+  DeviceState* d = nullptr;
+  gsg_status_t st = device_state(&d);
+  if (st != GSG_OK) return st;
+  const int rc = gsg::launch_gemm(sparse, a_codes, a_scales, x_scale, w_vals, w_meta, w_scales, w_scale, off, E, N,
+                                  K, R, max_rows, Y, y_dtype == GSG_OUT_F32 ? 1 : 0, d->status, d->num_sms,
+                                  as_stream(stream));
+  return rc == 0 ? GSG_OK : GSG_ERR_CUDA;
+}
+
+gsg_status_t gsg_grouped_sparse_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* x_tensor_scale,
+                                     const uint8_t* w_values, const uint8_t* w_meta, const uint8_t* w_scales,
+                                     const float* w_tensor_scale, const int32_t* expert_offsets, int E, int N, int K,
+                                     int R, int max_rows_per_expert, void* Y, int y_dtype, void* stream) {
+  return gemm_common(true, a_codes, a_scales, x_tensor_scale, w_values, w_meta, w_scales, w_tensor_scale,
+                     expert_offsets, E, N, K, R, max_rows_per_expert, Y, y_dtype, stream);
+}
+
+gsg_status_t gsg_grouped_dense_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* x_tensor_scale,
+                                    const uint8_t* w_codes, const uint8_t* w_scales, const float* w_tensor_scale,
+                                    const int32_t* expert_offsets, int E, int N, int K, int R,
+                                    int max_rows_per_expert, void* Y, int y_dtype, void* stream) {
+  return gemm_common(false, a_codes, a_scales, x_tensor_scale, w_codes, nullptr, w_scales, w_tensor_scale,
+                     expert_offsets, E, N, K, R, max_rows_per_expert, Y, y_dtype, stream);
+}
+
+gsg_status_t gsg_unpermute_scale(const uint16_t* Y, const int32_t* inv_perm, const float* gates, int T, int k, int N,
+                                 uint16_t* out, void* stream) {
+  if (T < 0 || k < 1 || N < 8 || N % 8 != 0) return GSG_ERR_INVALID_ARG;
+  if ((long long)T * k > (1ll << 30)) return GSG_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return GSG_OK;
+  if (!Y || !inv_perm || !gates || !out) return GSG_ERR_INVALID_ARG;
+  if (!aligned16(Y) || !aligned16(out)) return GSG_ERR_INVALID_ARG;
+  DeviceState* d = nullptr;
+  gsg_status_t st = device_state(&d);
+  if (st != GSG_OK) return st;
+  return from_cuda(gsg::launch_unpermute(Y, inv_perm, gates, T, k, N, out, d->status, d->num_sms, as_stream(stream)));
+}
+
+gsg_status_t gsg_get_device_status(void* stream) {
+  DeviceState* d = nullptr;
+  gsg_status_t st = device_state(&d);
+  if (st != GSG_OK) return st;
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return GSG_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, d->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return GSG_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(d->status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return GSG_ERR_CUDA;
+  }
+  return static_cast<gsg_status_t>(v);
+}
+
+const char* gsg_status_string(gsg_status_t s) {
+  switch (s) {
+    case GSG_OK: return "ok";
+    case GSG_ERR_INVALID_ARG: return "invalid argument";
+    case GSG_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case GSG_ERR_CUDA: return "CUDA error";
+    case GSG_ERR_BAD_ROUTING: return "expert id or expert offsets out of range";
+    case GSG_ERR_NONFINITE: return "non-finite value in a quantized tensor";
+    case GSG_ERR_DEVICE_TIMEOUT: return "a bounded wait inside a kernel timed out";
+    case GSG_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+int gsg_version(void) { return 1; }
+
+}  // extern "C"

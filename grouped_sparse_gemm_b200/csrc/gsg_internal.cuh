@@ -1,0 +1,111 @@
+// gsg_internal.cuh -- shared device helpers of libgsg (sm_100a only).
+//
+// Number formats (App. A of "Hardware-Native Joint Sparse-Quantization for Trillion-Scale
+// Mixture-of-Experts", p.14): E2M1 values and UE4M3 block scales.  Encoders round to nearest,
+// ties to even, and saturate; every fp32 step uses the _rn intrinsics so that no
+// multiply-add is contracted and the results are reproducible bit for bit.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include "../../include/gsg.h"
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "libgsg is written for sm_100a (Blackwell B200) only"
+#endif
+
+namespace gsg {
+
+constexpr int kTileN = 128;            // weight rows per tile (MMA M)
+constexpr int kChunkK = 256;           // logical K per pipeline stage / metadata chunk
+constexpr int kActScalePadRows = 256;  // extra zero rows of the quad activation-scale layout
+constexpr float kTensorScaleDen = 2688.0f;  // 6 * 448
+
+// ------------------------------------------------------------------ status word
+__device__ __forceinline__ void set_status(int* status, int code) {
+  if (status != nullptr) atomicCAS(status, 0, code);
+}
+
+// ------------------------------------------------------------------ codecs
+// UE4M3 (E4M3 without sign): bias 7, subnormal q * 2^-9, max 448 = code 0x7E.
+__device__ __forceinline__ float ue4m3_decode(uint32_t code) {
+  uint32_t e = (code >> 3) & 0xF, m = code & 7;
+  if (e == 0) return __uint2float_rn(m) * (1.0f / 512.0f);
+  // (8 + m) * 2^(e - 10): exact in fp32.
+  return __uint_as_float(((e + 120u) << 23) | (m << 20));
+}
+
+// x >= 0 and finite.  Round to nearest, ties to even code, saturate at 448.
+__device__ __forceinline__ uint32_t ue4m3_encode(float x) {
+  if (!(x > 0.0f)) return 0u;
+  if (x >= 448.0f) return 0x7Eu;
+  uint32_t u = __float_as_uint(x);
+  int e = int(u >> 23) - 127;
+  if (e < -6) {                                  // UE4M3 subnormal range: q * 2^-9, q in 0..8
+    return __float2uint_rn(__fmul_rn(x, 512.0f));  // exact scaling, round half to even
+  }
+  uint32_t m = u & 0x7FFFFFu;
+  uint32_t q = m >> 20;
+  uint32_t rem = m & 0xFFFFFu;
+  if (rem > 0x80000u || (rem == 0x80000u && (q & 1u))) q += 1u;
+  uint32_t eb = uint32_t(e + 7);
+  if (q == 8u) { q = 0u; eb += 1u; }
+  uint32_t code = (eb << 3) | q;
+  return code > 0x7Eu ? 0x7Eu : code;
+}
+
+// E2M1: magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6}; sign bit 3 copied from the input (-0 -> 0x8).
+__device__ __forceinline__ uint32_t e2m1_encode(float v) {
+  float a = fabsf(v);
+  uint32_t c;
+  if (a <= 0.25f) c = 0u;
+  else if (a < 0.75f) c = 1u;
+  else if (a <= 1.25f) c = 2u;
+  else if (a < 1.75f) c = 3u;
+  else if (a <= 2.5f) c = 4u;
+  else if (a < 3.5f) c = 5u;
+  else if (a <= 5.0f) c = 6u;
+  else c = 7u;
+  return c | ((__float_as_uint(v) >> 28) & 8u);
+}
+
+// Block rule shared by weights and activations (s = tensor scale, b = block amax):
+//   sc = UE4M3(b / (6 s)),  d = dec(sc) * s,  inv = d == 0 ? 0 : 1/d,  code = E2M1(v * inv)
+struct BlockScale {
+  uint32_t sc;
+  float inv;
+};
+__device__ __forceinline__ BlockScale block_scale(float blk_amax, float six_s, float s) {
+  BlockScale r;
+  r.sc = ue4m3_encode(__fdiv_rn(blk_amax, six_s));
+  float d = __fmul_rn(ue4m3_decode(r.sc), s);
+  r.inv = (d == 0.0f) ? 0.0f : __frcp_rn(d);
+  return r;
+}
+
+__device__ __forceinline__ float tensor_scale_from_amax(float amax) {
+  return amax == 0.0f ? 1.0f : __fdiv_rn(amax, kTensorScaleDen);
+}
+
+// ------------------------------------------------------------------ small utilities
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__host__ __device__ inline int ceil_div_i(int a, int b) { return (a + b - 1) / b; }
+
+}  // namespace gsg

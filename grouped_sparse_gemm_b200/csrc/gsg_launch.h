@@ -1,0 +1,42 @@
+// gsg_launch.h -- host-side launchers of the individual kernels (internal to libgsg).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace gsg {
+
+// gsg_pack.cu
+int pack_partials_per_expert(int N, int K);
+cudaError_t launch_pack(bool sparse, const float* W, int E, int N, int K, uint8_t* values, uint8_t* meta,
+                        uint8_t* scales, float* w_tensor_scale, float* partial, int* status, cudaStream_t stream);
+
+// gsg_quant.cu
+int quant_partials(long long n_elems);
+cudaError_t launch_quant(const uint16_t* X, int T, int K, int sf, const int32_t* inv_perm, int k, const float* s_in,
+                         uint8_t* codes, uint8_t* scales, float* s_out, float* partial, int* status, int num_sms,
+                         cudaStream_t stream);
+
+// gsg_route.cu
+int route_chunks(int R);
+size_t route_workspace_bytes(int R, int E);
+bool route_supported(int E);
+cudaError_t route_set_smem_attrs();
+cudaError_t launch_route(const int32_t* ids, int R, int E, int32_t* off, int32_t* perm_src, int32_t* inv_perm,
+                         void* ws, int* status, cudaStream_t stream);
+
+// gsg_unpermute.cu
+cudaError_t launch_unpermute(const uint16_t* Y, const int32_t* inv_perm, const float* gates, int T, int k, int N,
+                             uint16_t* out, int* status, int num_sms, cudaStream_t stream);
+
+// gsg_gemm.cu
+bool gemm_supported(int E);
+int gemm_pick_bn(int max_rows);
+cudaError_t gemm_set_smem_attrs();
+int launch_gemm(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, const float* x_scale,
+                const uint8_t* w_vals, const uint8_t* w_meta, const uint8_t* w_scales, const float* w_scale,
+                const int32_t* off, int E, int N, int K, int R, int max_rows, void* Y, int y_f32, int* status,
+                int num_sms, cudaStream_t stream);
+
+}  // namespace gsg

@@ -1,0 +1,202 @@
+// gsg_quant.cu -- NVFP4 activation quantizer fused with MoE dispatch.
+//
+// "Hardware-Native Joint Sparse-Quantization for Trillion-Scale Mixture-of-Experts"
+// (paperlayer.ai summary), §D.1 (p.19): activation quantization forms 32-element scale blocks
+// and is fused with dispatch for the first expert GEMM; §3.4 (pp.5-6): weights and quantized
+// activations are packed in corresponding scale blocks.
+//
+// Launch 1 (skipped when the caller supplies s_x): partial max|X| per block, 128-bit loads,
+// warp-shuffle reductions.  Launch 2: every block folds the partials into s_x = amax/2688,
+// then each thread quantizes 16 consecutive elements of one token row (two 128-bit loads),
+// pairs of lanes combine their maxima into the 32-element block amax, eight lanes assemble
+// the four scales of one MMA k-block into a 32-bit word, and the token's codes and scale
+// words are written to each of its k routed rows (the dispatch).  The same launch zero-fills
+// the padding entries of the quad scale layout.
+#include "gsg_internal.cuh"
+
+namespace gsg {
+
+constexpr int kQuantThreads = 256;
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
+
+__global__ void __launch_bounds__(kQuantThreads)
+act_amax_kernel(const uint16_t* __restrict__ X, long long n8, float* __restrict__ partial, int* status) {
+  __shared__ float red[kQuantThreads / 32];
+  float mx = 0.0f;
+  bool finite = true;
+  const uint4* X4 = reinterpret_cast<const uint4*>(X);
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
+       i += (long long)gridDim.x * blockDim.x) {
+    uint4 v = __ldg(X4 + i);
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t lo = w[j] & 0xFFFFu, hi = w[j] >> 16;
+      finite &= ((lo & 0x7F80u) != 0x7F80u) && ((hi & 0x7F80u) != 0x7F80u);
+      mx = fmaxf(mx, fmaxf(fabsf(bf16_bits_to_f32(lo)), fabsf(bf16_bits_to_f32(hi))));
+    }
+  }
+  if (!finite) set_status(status, GSG_ERR_NONFINITE);
+  mx = warp_max(mx);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < kQuantThreads / 32 ? red[threadIdx.x] : 0.0f;
+    v = warp_max(v);
+    if (threadIdx.x == 0) partial[blockIdx.x] = v;
+  }
+}
+
+struct QuantParams {
+  const uint16_t* X;
+  const int32_t* inv_perm;
+  const float* s_in;
+  const float* partial;
+  int nparts;
+  int T, K, sf, k, R, rcap;
+  uint8_t* codes;
+  uint8_t* scales;
+  float* s_out;
+  int* status;
+};
+
+__global__ void __launch_bounds__(kQuantThreads)
+act_quant_kernel(QuantParams p) {
+  __shared__ float red[kQuantThreads / 32];
+  __shared__ float s_sh;
+  // ---- tensor scale
+  if (p.s_in != nullptr) {
+    if (threadIdx.x == 0) s_sh = __ldg(p.s_in);
+  } else {
+    float v = 0.0f;
+    for (int i = threadIdx.x; i < p.nparts; i += blockDim.x) v = fmaxf(v, p.partial[i]);
+    v = warp_max(v);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      float w = threadIdx.x < kQuantThreads / 32 ? red[threadIdx.x] : 0.0f;
+      w = warp_max(w);
+      if (threadIdx.x == 0) s_sh = tensor_scale_from_amax(w);
+    }
+  }
+  __syncthreads();
+  const float s = s_sh;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *p.s_out = s;
+  const float six_s = __fmul_rn(6.0f, s);
+
+  const int lane = threadIdx.x & 31;
+  const int units_per_row = p.K / 16;
+  const long long U = (long long)p.T * units_per_row;
+  const int KBa = p.K / (4 * p.sf);
+  const int gwarp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  // ---- main: warp-uniform loop so that the lane shuffles below always see the full warp
+  for (long long base = (long long)gwarp * 32; base < U; base += (long long)nwarps * 32) {
+    const long long unit = base + lane;
+    const bool valid = unit < U;
+    const int t = valid ? int(unit / units_per_row) : 0;
+    const int c16 = valid ? int(unit % units_per_row) : 0;
+    float x[16];
+    float amax = 0.0f;
+    if (valid) {
+      const uint4* src = reinterpret_cast<const uint4*>(p.X + (size_t)t * p.K + (size_t)c16 * 16);
+      uint4 a = __ldg(src), b = __ldg(src + 1);
+      uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        x[2 * j] = bf16_bits_to_f32(w[j] & 0xFFFFu);
+        x[2 * j + 1] = bf16_bits_to_f32(w[j] >> 16);
+      }
+#pragma unroll
+      for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(x[j]));
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) x[j] = 0.0f;
+    }
+    if (p.sf == 32) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    const BlockScale bs = block_scale(amax, six_s, s);
+    uint64_t codes = 0;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) codes |= uint64_t(e2m1_encode(__fmul_rn(x[j], bs.inv))) << (4 * j);
+    // four scales of one MMA k-block -> one 32-bit word (sf 32: lanes g, g+2, g+4, g+6; sf 16: g..g+3)
+    uint32_t word;
+    int kb;
+    bool writer;
+    if (p.sf == 32) {
+      const int g = lane & ~7;
+      word = __shfl_sync(0xffffffffu, bs.sc, g) | (__shfl_sync(0xffffffffu, bs.sc, g + 2) << 8) |
+             (__shfl_sync(0xffffffffu, bs.sc, g + 4) << 16) | (__shfl_sync(0xffffffffu, bs.sc, g + 6) << 24);
+      kb = c16 >> 3;
+      writer = (lane & 7) == 0;
+    } else {
+      const int g = lane & ~3;
+      word = __shfl_sync(0xffffffffu, bs.sc, g) | (__shfl_sync(0xffffffffu, bs.sc, g + 1) << 8) |
+             (__shfl_sync(0xffffffffu, bs.sc, g + 2) << 16) | (__shfl_sync(0xffffffffu, bs.sc, g + 3) << 24);
+      kb = c16 >> 2;
+      writer = (lane & 3) == 0;
+    }
+    if (!valid) continue;
+    for (int j = 0; j < p.k; ++j) {
+      int row = t;
+      if (p.inv_perm != nullptr) {
+        row = __ldg(p.inv_perm + (size_t)t * p.k + j);
+        if (row < 0 || row >= p.R) { set_status(p.status, GSG_ERR_BAD_ROUTING); continue; }
+      }
+      *reinterpret_cast<uint64_t*>(p.codes + (size_t)row * (p.K / 2) + (size_t)c16 * 8) = codes;
+      if (writer) {
+        uint32_t* sw = reinterpret_cast<uint32_t*>(p.scales);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int rr = row - 32 * c;
+          if (rr >= 0) sw[((size_t)kb * p.rcap + rr) * 4 + c] = word;
+        }
+      }
+    }
+  }
+  // ---- zero the quad entries that refer to rows >= R
+  const int r_lo = p.R > 96 ? p.R - 96 : 0;
+  const long long npad = (long long)KBa * (p.rcap - r_lo) * 4;
+  uint32_t* sw = reinterpret_cast<uint32_t*>(p.scales);
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < npad;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int c = int(i & 3);
+    const long long rest = i >> 2;
+    const int rr = r_lo + int(rest % (p.rcap - r_lo));
+    const int kb = int(rest / (p.rcap - r_lo));
+    if (rr + 32 * c >= p.R) sw[((size_t)kb * p.rcap + rr) * 4 + c] = 0u;
+  }
+}
+
+int quant_partials(long long n_elems) {
+  long long n8 = n_elems / 8;
+  long long b = (n8 + kQuantThreads * 4 - 1) / (kQuantThreads * 4);
+  if (b < 1) b = 1;
+  if (b > 512) b = 512;
+  return int(b);
+}
+
+cudaError_t launch_quant(const uint16_t* X, int T, int K, int sf, const int32_t* inv_perm, int k,
+                         const float* s_in, uint8_t* codes, uint8_t* scales, float* s_out,
+                         float* partial, int* status, int num_sms, cudaStream_t stream) {
+  const long long n = (long long)T * K;
+  int P = quant_partials(n);
+  if (s_in == nullptr && n > 0) {
+    act_amax_kernel<<<P, kQuantThreads, 0, stream>>>(X, n / 8, partial, status);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+  }
+  if (n == 0) P = 0;  // no data: the quant kernel folds zero partials -> amax 0 -> s_x = 1
+  QuantParams p;
+  p.X = X; p.inv_perm = inv_perm; p.s_in = s_in; p.partial = partial; p.nparts = P;
+  p.T = T; p.K = K; p.sf = sf; p.k = k; p.R = T * k; p.rcap = T * k + kActScalePadRows;
+  p.codes = codes; p.scales = scales; p.s_out = s_out; p.status = status;
+  const long long units = (long long)T * (K / 16);
+  long long blocks = (units + kQuantThreads - 1) / kQuantThreads;
+  if (blocks < 1) blocks = 1;
+  if (blocks > (long long)num_sms * 8) blocks = (long long)num_sms * 8;
+  act_quant_kernel<<<(unsigned)blocks, kQuantThreads, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace gsg

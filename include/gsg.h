@@ -1,0 +1,188 @@
+/*
+ * gsg.h -- C ABI of the grouped sparse-NVFP4 expert GEMM library (libgsg.so).
+ *
+ * The operation is the routed Mixture-of-Experts expert projection described in
+ * "Hardware-Native Joint Sparse-Quantization for Trillion-Scale Mixture-of-Experts"
+ * (paperlayer.ai summary page): for every expert e, Y_e = X_e . W_e^T over the rows
+ * routed to e, with W_e stored as paired 4:8 NVFP4 (App. A "Blackwell paired 4:8 NVFP4",
+ * p.14; "Storage layout", p.15), activations quantized to NVFP4 with 32-element scale
+ * blocks and fused with dispatch (§D.1, p.19), all experts executed in one grouped launch
+ * with the sparse weight as MMA operand A (§3.4, pp.5-6).
+ *
+ * Conventions for every call
+ *   - Pointers are DEVICE pointers owned by the caller unless stated otherwise.  The library
+ *     allocates nothing; calls that need scratch take a caller workspace (size from
+ *     gsg_workspace_size).  `stream` is a cudaStream_t (NULL = legacy default stream).
+ *   - Calls are asynchronous on `stream`.  Errors the host can detect (bad sizes, NULL
+ *     pointers, small workspace) return at once without launching anything.  Errors found
+ *     on the device (expert id out of range, non-finite input, a bounded wait that timed
+ *     out) set a sticky per-device status word (first error wins); read and clear it with
+ *     gsg_get_device_status.  Outputs of a call that raised a device error are unspecified.
+ *   - Shapes: K % 256 == 0, N % 128 == 0, E >= 1.  bf16 tensors are passed as uint16_t bit
+ *     patterns.  Multi-dimensional buffers are dense, last index fastest.
+ *   - Re-entrant across streams; the only global state is the device status word.
+ *
+ * Packed weight layouts (tile-major, the order the GEMM streams them; n-tile = 128 output
+ * rows, NT = N/128; k-block = one MMA step = 64 stored 4-bit values per row):
+ *   sparse values  [E][NT][K/128][4096 B]  row r (0..127), stored value v (0..63) of the k-block
+ *                  -> byte c = v/2 (low nibble = even v) at (r/8)*256 + (c/16)*128 + (r%8)*16 + c%16.
+ *                  Stored values are the four retained E2M1 codes of each 8-group in K order.
+ *   sparse meta    [E][NT][K/256][2048 B] row r, 8-group g of the 256-wide chunk (0..31)
+ *                  -> byte r*16 + g/2, low nibble = even g; nibble = i0 | i1 << 2 (kept pairs i0<i1).
+ *   weight scales  [E][NT][K/(4*sf)][512 B] row r, block j (0..3) of the k-block
+ *                  -> byte 16*(r%32) + 4*(r/32) + j.  UE4M3 codes; sf = 32 sparse, 16 dense.
+ *   dense codes    [E][NT][K/64][4096 B]  same index function as sparse values, v = K index.
+ * Activation layouts (R routed rows; KBa = K/(4*sf)):
+ *   codes  [R][K/2]  row-major E2M1, low nibble = even k.
+ *   scales [KBa][R + 256][4][4 B]: entry (kb, r, c, j) = UE4M3 scale of block 4*kb + j of
+ *          row r + 32*c (0 when r + 32*c >= R).  Each scale is stored four times so that the
+ *          GEMM fetches the scale tile of ANY starting row with one contiguous copy.
+ */
+#ifndef GSG_H
+#define GSG_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GSG_OK = 0,
+  GSG_ERR_INVALID_ARG = -1,       /* NULL pointer, negative size, bad enum value            */
+  GSG_ERR_UNSUPPORTED_SHAPE = -2, /* K % 256, N % 128, sizes beyond the library's limits      */
+  GSG_ERR_CUDA = -3,              /* a CUDA runtime call or a launch failed                   */
+  GSG_ERR_BAD_ROUTING = -4,       /* device: expert id outside [0, E), or inconsistent offsets */
+  GSG_ERR_NONFINITE = -5,         /* device: NaN/Inf in a tensor that is being quantized      */
+  GSG_ERR_DEVICE_TIMEOUT = -6,    /* device: a bounded wait inside a kernel gave up           */
+  GSG_ERR_WORKSPACE = -7          /* workspace NULL or smaller than gsg_workspace_size()      */
+} gsg_status_t;
+
+/* Operation ids for gsg_workspace_size. */
+enum {
+  GSG_OP_PACK_SPARSE = 1,
+  GSG_OP_PACK_DENSE = 2,
+  GSG_OP_ROUTE = 3,
+  GSG_OP_QUANTIZE = 4,
+  GSG_OP_GEMM = 5
+};
+
+/* Output element types of the grouped GEMMs. */
+enum { GSG_OUT_BF16 = 0, GSG_OUT_F32 = 1 };
+
+/* ----------------------------------------------------------------------------------------
+ * Buffer sizes in bytes (host-only arithmetic, no GPU access).
+ */
+size_t gsg_sparse_values_bytes(int E, int N, int K);          /* E*N*K/4                    */
+size_t gsg_sparse_meta_bytes(int E, int N, int K);            /* E*N*K/16                   */
+size_t gsg_weight_scales_bytes(int E, int N, int K, int sf_block); /* E*N*K/sf_block      */
+size_t gsg_dense_codes_bytes(int E, int N, int K);            /* E*N*K/2                    */
+size_t gsg_act_codes_bytes(int R, int K);                     /* R*K/2                      */
+size_t gsg_act_scales_bytes(int R, int K, int sf_block);      /* K/(4 sf) * (R+256) * 16    */
+/* Workspace needed by `op` (0 when none).  T = tokens, k = experts per token. */
+size_t gsg_workspace_size(int op, int E, int N, int K, int T, int k);
+
+/* ----------------------------------------------------------------------------------------
+ * gsg_pack_sparse_nvfp4 -- weight packer (offline).
+ * Paper: App. A "Blackwell paired 4:8 NVFP4" (p.14) and "Storage layout" (p.15); §3.4 (p.5).
+ * W fp32 [E][N][K] (K contiguous).  Per 8-group of K the two adjacent pairs with the largest
+ * energy w0*w0 + w1*w1 (fp32, ties -> lower pair) are kept; s_w[e] = amax(kept W_e)/2688
+ * (1 if 0); per 32-block b: sc = UE4M3(b / (6 s_w)), codes = E2M1(w / (dec(sc) s_w)),
+ * round-to-nearest-even with saturation.  Writes values/meta/scales in the layouts above and
+ * w_tensor_scale fp32 [E].  Non-finite W sets GSG_ERR_NONFINITE on the device.
+ */
+gsg_status_t gsg_pack_sparse_nvfp4(const float* W, int E, int N, int K,
+                                   uint8_t* values, uint8_t* meta, uint8_t* scales,
+                                   float* w_tensor_scale,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* gsg_pack_dense_nvfp4 -- dense NVFP4 packer for the in-repo control GEMM (16-element
+ * blocks, the block size the dense block-scaled MMA takes; §D.2, p.19: the control differs
+ * from the sparse kernel only in sparsity).  codes [E][NT][K/64][4096], scales [E][NT][K/64][512]. */
+gsg_status_t gsg_pack_dense_nvfp4(const float* W, int E, int N, int K,
+                                  uint8_t* codes, uint8_t* scales, float* w_tensor_scale,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* ----------------------------------------------------------------------------------------
+ * gsg_moe_route_permute -- group routed rows by expert.
+ * Paper: §2 "Execution gap" (p.3): routing-dependent expert products with different token
+ * counts run together; §D.1 (p.19): dispatch.  topk_ids int32 [T][k] in [0, E).
+ * Routed pair (t, j) has flat index f = t*k + j.  Rows of expert e are [off[e], off[e+1]),
+ * in ascending f.  Outputs: expert_offsets int32 [E+1], perm_src int32 [R] (row -> f),
+ * inv_perm int32 [R] (f -> row).  Out-of-range ids set GSG_ERR_BAD_ROUTING (outputs then
+ * unspecified).  Deterministic.
+ */
+gsg_status_t gsg_moe_route_permute(const int32_t* topk_ids, int T, int k, int E,
+                                   int32_t* expert_offsets, int32_t* perm_src, int32_t* inv_perm,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* ----------------------------------------------------------------------------------------
+ * gsg_quantize_act_nvfp4 -- NVFP4 activation quantizer fused with dispatch.
+ * Paper: §D.1 (p.19): activation quantization forms 32-element scale blocks and is fused
+ * with dispatch; §3.4 (pp.5-6): corresponding scale blocks for weights and activations.
+ * X bf16 [T][K].  s_x = max|X|/2688 (1 if 0), or *x_tensor_scale_in when that is non-NULL.
+ * Each token row is quantized once (per sf_block block: UE4M3 scale + E2M1 codes, same rule
+ * as the weights) and written to each of its k routed rows inv_perm[t*k + j]
+ * (inv_perm NULL: row t, and k must be 1).  sf_block: 32 (sparse GEMM) or 16 (dense control).
+ * Outputs: codes [R][K/2], scales in the quad layout above (R = T*k), x_tensor_scale_out fp32[1].
+ */
+gsg_status_t gsg_quantize_act_nvfp4(const uint16_t* X, int T, int K, int sf_block,
+                                    const int32_t* inv_perm, int k,
+                                    const float* x_tensor_scale_in,
+                                    uint8_t* codes, uint8_t* scales, float* x_tensor_scale_out,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* ----------------------------------------------------------------------------------------
+ * gsg_grouped_sparse_gemm -- the grouped paired-4:8 NVFP4 expert GEMM.
+ * Paper: §3.4 (pp.5-6): Blackwell sparse MMA with grouped scheduling, one launch, the sparse
+ * weight as operand A; §2 (p.3): the sparse NVFP4 path peaks at 2x dense NVFP4.
+ * For each expert e and routed row r in [off[e], off[e+1]):
+ *     Y[r][n] = s_x * s_w[e] * sum_k a[r][k] * w[e][n][k]      (fp32 accumulation)
+ * a_codes/a_scales from gsg_quantize_act_nvfp4 (sf_block 32); w_* from gsg_pack_sparse_nvfp4.
+ * expert_offsets int32 [E+1], monotone, off[0] = 0, off[E] <= R.  max_rows_per_expert is a
+ * host-side hint that picks the token tile (<= 0: unknown).  Y [R][N] bf16 (y_dtype
+ * GSG_OUT_BF16) or fp32 (GSG_OUT_F32); rows >= off[E] are not written.  No workspace.
+ * Persistent kernel, one CTA per SM: TMA/bulk copies into a shared-memory ring, tcgen05
+ * block-scaled sparse MMA into TMEM, epilogue applies s_x*s_w[e].
+ */
+gsg_status_t gsg_grouped_sparse_gemm(const uint8_t* a_codes, const uint8_t* a_scales,
+                                     const float* x_tensor_scale,
+                                     const uint8_t* w_values, const uint8_t* w_meta,
+                                     const uint8_t* w_scales, const float* w_tensor_scale,
+                                     const int32_t* expert_offsets, int E, int N, int K, int R,
+                                     int max_rows_per_expert, void* Y, int y_dtype, void* stream);
+
+/* gsg_grouped_dense_gemm -- the dense-NVFP4 control on the same skeleton (non-sparse MMA,
+ * 16-element blocks).  a_* from gsg_quantize_act_nvfp4 with sf_block 16; w_* from
+ * gsg_pack_dense_nvfp4.  Same semantics as gsg_grouped_sparse_gemm. */
+gsg_status_t gsg_grouped_dense_gemm(const uint8_t* a_codes, const uint8_t* a_scales,
+                                    const float* x_tensor_scale,
+                                    const uint8_t* w_codes, const uint8_t* w_scales,
+                                    const float* w_tensor_scale,
+                                    const int32_t* expert_offsets, int E, int N, int K, int R,
+                                    int max_rows_per_expert, void* Y, int y_dtype, void* stream);
+
+/* ----------------------------------------------------------------------------------------
+ * gsg_unpermute_scale -- gate-weighted scatter back to tokens.
+ * Paper: §D.1 (p.19): scatter after the expert GEMM.
+ *     out[t][n] = bf16_rne( sum_{j<k} fp32(gates[t][j] * Y[inv_perm[t*k+j]][n]) )
+ * fp32 products and running sum (starting at 0), j ascending.  Y bf16 [R][N],
+ * gates fp32 [T][k], out bf16 [T][N].  N % 8 == 0.
+ */
+gsg_status_t gsg_unpermute_scale(const uint16_t* Y, const int32_t* inv_perm, const float* gates,
+                                 int T, int k, int N, uint16_t* out, void* stream);
+
+/* ----------------------------------------------------------------------------------------
+ * Status.  gsg_get_device_status synchronizes `stream`, returns the device status word of the
+ * current device and clears it.  gsg_status_string never returns NULL.
+ */
+gsg_status_t gsg_get_device_status(void* stream);
+const char* gsg_status_string(gsg_status_t status);
+int gsg_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GSG_H */

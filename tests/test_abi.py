@@ -1,0 +1,82 @@
+"""The C ABI library loads, exports every declared symbol and rejects bad arguments on the host
+(no GPU needed: every check here returns before any CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import grouped_sparse_gemm_b200 as gsg
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from grouped_sparse_gemm_b200 import _build
+    _build.build()
+    return gsg.load_library()
+
+
+def declared_symbols():
+    with open(os.path.join(ROOT, "include", "gsg.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gsg_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    decl = declared_symbols()
+    assert len(decl) >= 15
+    for name in decl:
+        assert hasattr(L, name), name
+    assert sorted(decl) == sorted(gsg.EXPORTED_SYMBOLS)
+
+
+def test_sizes(L):
+    E, N, K = 3, 256, 512
+    total = L.gsg_sparse_values_bytes(E, N, K) + L.gsg_sparse_meta_bytes(E, N, K) + \
+        L.gsg_weight_scales_bytes(E, N, K, 32)
+    assert total * 8 == 2.75 * E * N * K                       # 2.75 bit per weight
+    assert L.gsg_dense_codes_bytes(E, N, K) + L.gsg_weight_scales_bytes(E, N, K, 16) == 4.5 * E * N * K / 8
+    assert L.gsg_act_codes_bytes(10, 256) == 1280
+    assert L.gsg_act_scales_bytes(10, 256, 32) == 2 * (10 + 256) * 16
+    assert L.gsg_workspace_size(gsg.OP_ROUTE, 384, 0, 0, 64, 8) == 0          # single-launch routing
+    assert L.gsg_workspace_size(gsg.OP_ROUTE, 384, 0, 0, 8192, 8) == 2 * 8 * 384 * 4
+    assert L.gsg_workspace_size(gsg.OP_GEMM, 384, 4096, 7168, 8192, 8) == 0
+
+
+def test_status_strings(L):
+    for s in (0, -1, -2, -3, -4, -5, -6, -7, 42):
+        assert L.gsg_status_string(s)
+
+
+P = ctypes.c_void_p(16)   # a non-NULL, 16-byte aligned placeholder never dereferenced by the checks below
+
+
+def test_host_argument_checks(L):
+    # bad shapes (K % 256, N % 128) -> unsupported shape, no launch
+    assert L.gsg_pack_sparse_nvfp4(P, 1, 128, 100, P, P, P, P, P, 1 << 20, None) == -2
+    assert L.gsg_pack_sparse_nvfp4(P, 1, 100, 256, P, P, P, P, P, 1 << 20, None) == -2
+    assert L.gsg_pack_sparse_nvfp4(None, 1, 128, 256, P, P, P, P, P, 1 << 20, None) == -1
+    assert L.gsg_pack_sparse_nvfp4(P, 1, 128, 256, P, P, P, P, None, 0, None) == -7
+    assert L.gsg_grouped_sparse_gemm(P, P, P, P, P, P, P, P, 4, 128, 300, 8, -1, P, 0, None) == -2
+    assert L.gsg_grouped_sparse_gemm(P, P, P, P, P, P, P, P, 4, 128, 256, 8, -1, P, 7, None) == -1
+    assert L.gsg_grouped_sparse_gemm(P, P, P, P, P, P, P, P, 2000, 128, 256, 8, -1, P, 0, None) == -2
+    assert L.gsg_grouped_sparse_gemm(P, P, P, P, None, P, P, P, 4, 128, 256, 8, -1, P, 0, None) == -1
+    assert L.gsg_grouped_sparse_gemm(P, P, P, P, P, P, P, P, 4, 128, 256, 0, -1, P, 0, None) == 0  # R = 0
+    assert L.gsg_moe_route_permute(P, 4, 2, 0, P, P, P, None, 0, None) == -2
+    assert L.gsg_moe_route_permute(P, 4, 2, 5000, P, P, P, None, 0, None) == -2
+    assert L.gsg_moe_route_permute(P, 8192, 8, 16, P, P, P, None, 0, None) == -7
+    assert L.gsg_quantize_act_nvfp4(P, 4, 256, 24, P, 2, None, P, P, P, P, 1 << 20, None) == -1
+    assert L.gsg_quantize_act_nvfp4(P, 4, 256, 32, None, 2, None, P, P, P, P, 1 << 20, None) == -1
+    assert L.gsg_quantize_act_nvfp4(P, 4, 200, 32, P, 2, None, P, P, P, P, 1 << 20, None) == -2
+    assert L.gsg_quantize_act_nvfp4(P, 4, 256, 32, P, 2, None, P, P, P, None, 0, None) == -7
+    assert L.gsg_unpermute_scale(P, P, P, 4, 2, 12, P, None) == -1
+    assert L.gsg_unpermute_scale(P, P, P, 0, 2, 128, P, None) == 0
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        gsg.quantize_act_nvfp4(torch.zeros(4, 256, dtype=torch.bfloat16))

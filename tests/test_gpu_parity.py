@@ -1,0 +1,330 @@
+"""GPU parity: every kernel of the path against the oracle, through the C ABI.
+
+Packed weights, activation codes/scales, routing and the scatter must match bit for bit;
+GEMM outputs must satisfy |y - y_ref| <= 2^-10 * sum|a*w| + 1e-6 (fp32 output; a bf16 output
+adds its own half-ulp of rounding).
+"""
+import numpy as np
+import pytest
+import torch
+
+from grouped_sparse_gemm_b200 import inputs
+from oracle import layout as olayout
+from oracle import pack as opack
+from oracle import unpermute as ounperm
+from tests import gsg_testlib as tl
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module")
+def gsg():
+    import grouped_sparse_gemm_b200 as g
+    g.load_library()
+    assert g.lib().gsg_version() == 1
+    return g
+
+
+def _status_ok(gsg):
+    assert gsg.get_device_status() == 0
+
+
+# ---------------------------------------------------------------- packing
+@pytest.mark.parametrize("E,N,K", [(1, 128, 256), (3, 256, 768), (2, 384, 2048)])
+def test_pack_sparse_bit_exact(gsg, E, N, K):
+    cfg = inputs.custom_config("p", E=E, K=K, N=N, T=1, top_k=1)
+    W = inputs.all_weights(cfg)
+    W[0, :3] = 0.0                     # a zero row: all-zero blocks
+    W[0, 5, :8] = 0.25                 # a group of equal pair energies (ties)
+    if E > 1:
+        W[1].mul_(1e-3)                # a small-magnitude expert
+    pw = gsg.pack_sparse_nvfp4(W.to(DEV))
+    vals, meta, scs, sws, _ = tl.oracle_pack_sparse(W.numpy())
+    np.testing.assert_array_equal(pw.values.cpu().numpy(), vals)
+    np.testing.assert_array_equal(pw.meta.cpu().numpy(), meta)
+    np.testing.assert_array_equal(pw.scales.cpu().numpy(), scs)
+    np.testing.assert_array_equal(pw.w_scale.cpu().numpy(), sws)
+    _status_ok(gsg)
+
+
+@pytest.mark.parametrize("E,N,K", [(1, 128, 256), (2, 256, 768)])
+def test_pack_dense_bit_exact(gsg, E, N, K):
+    cfg = inputs.custom_config("p", E=E, K=K, N=N, T=1, top_k=1)
+    W = inputs.all_weights(cfg)
+    W[0, 1] = 0.0
+    pw = gsg.pack_dense_nvfp4(W.to(DEV))
+    vals, scs, sws, _ = tl.oracle_pack_dense(W.numpy(), 16)
+    np.testing.assert_array_equal(pw.codes.cpu().numpy(), vals)
+    np.testing.assert_array_equal(pw.scales.cpu().numpy(), scs)
+    np.testing.assert_array_equal(pw.w_scale.cpu().numpy(), sws)
+
+
+def test_pack_flags_nonfinite(gsg):
+    W = torch.zeros(1, 128, 256)
+    W[0, 7, 9] = float("nan")
+    gsg.pack_sparse_nvfp4(W.to(DEV))
+    assert gsg.get_device_status() == -5
+    _status_ok(gsg)
+
+
+# ---------------------------------------------------------------- routing
+@pytest.mark.parametrize("T,k,E,mode", [(32, 2, 4, "uniform"), (512, 8, 128, "zipf"), (64, 8, 128, "uniform"),
+                                        (1025, 4, 7, "zipf"), (8192, 8, 384, "zipf"), (3, 1, 1, "uniform"),
+                                        (256, 8, 384, "uniform")])
+def test_route_matches_oracle(gsg, T, k, E, mode):
+    cfg = inputs.custom_config("r", E=E, K=256, N=128, T=T, top_k=k, routing=mode, zipf_s=1.1)
+    ids = inputs.routing(cfg) if k <= E else torch.zeros(T, k, dtype=torch.int32)
+    r = gsg.moe_route_permute(ids.to(DEV), E)
+    off, ps, ip = tl.route_np(ids, E)
+    np.testing.assert_array_equal(r.offsets.cpu().numpy(), off)
+    np.testing.assert_array_equal(r.perm_src.cpu().numpy()[:T * k], ps)
+    np.testing.assert_array_equal(r.inv_perm.cpu().numpy()[:T * k], ip)
+    _status_ok(gsg)
+
+
+def test_route_duplicates_and_empty(gsg):
+    ids = torch.tensor([[2, 2], [0, 2], [2, 0]], dtype=torch.int32)
+    r = gsg.moe_route_permute(ids.to(DEV), 4)
+    off, ps, ip = tl.route_np(ids, 4)
+    np.testing.assert_array_equal(r.offsets.cpu().numpy(), off)
+    np.testing.assert_array_equal(r.perm_src.cpu().numpy(), ps)
+    r0 = gsg.moe_route_permute(torch.zeros(0, 8, dtype=torch.int32, device=DEV), 5)
+    assert r0.offsets.cpu().tolist() == [0] * 6
+
+
+def test_route_flags_bad_ids(gsg):
+    ids = torch.tensor([[0, 9]], dtype=torch.int32, device=DEV)
+    gsg.moe_route_permute(ids, 4)
+    assert gsg.get_device_status() == -4
+    _status_ok(gsg)
+
+
+# ---------------------------------------------------------------- activation quantizer
+@pytest.mark.parametrize("name,sf", [("tiny", 32), ("30b_down_decode", 32), ("30b_up_prefill", 32), ("tiny", 16),
+                                     ("1t_down_decode_b1", 32)])
+def test_quantize_matches_oracle(gsg, name, sf):
+    cfg = inputs.CONFIGS[name]
+    X = inputs.activations(cfg)
+    ids = inputs.routing(cfg)
+    off, ps, ip = tl.route_np(ids, cfg.E)
+    qa = gsg.quantize_act_nvfp4(X.to(DEV), sf_block=sf, inv_perm=torch.from_numpy(ip).to(DEV), top_k=cfg.top_k)
+    codes, quad, s, _, _ = tl.oracle_act(X.float().numpy(), sf, ps, cfg.top_k)
+    assert qa.x_scale.item() == s
+    np.testing.assert_array_equal(qa.codes.cpu().numpy(), codes)
+    np.testing.assert_array_equal(qa.scales.cpu().numpy(), quad)
+    _status_ok(gsg)
+
+
+def test_quantize_identity_and_given_scale(gsg):
+    cfg = inputs.custom_config("q", E=1, K=512, N=128, T=37, top_k=1, outlier_frac=0.01, outlier_scale=50.0)
+    X = inputs.activations(cfg)
+    s_in = torch.tensor([0.0123], dtype=torch.float32)
+    qa = gsg.quantize_act_nvfp4(X.to(DEV), sf_block=32, x_scale_in=s_in.to(DEV))
+    codes, quad, s, _, _ = tl.oracle_act(X.float().numpy(), 32, None, 1, np.float32(0.0123))
+    assert qa.x_scale.item() == np.float32(0.0123)
+    np.testing.assert_array_equal(qa.codes.cpu().numpy(), codes)
+    np.testing.assert_array_equal(qa.scales.cpu().numpy(), quad)
+    Z = torch.zeros(5, 256, dtype=torch.bfloat16)
+    qz = gsg.quantize_act_nvfp4(Z.to(DEV), sf_block=32)
+    assert qz.x_scale.item() == 1.0 and not qz.codes.any().item()
+
+
+# ---------------------------------------------------------------- scatter
+@pytest.mark.parametrize("T,k,N", [(32, 2, 128), (64, 8, 2048), (7, 3, 136)])
+def test_unpermute_bit_exact(gsg, T, k, N):
+    Y = inputs.random_bf16((T * k, N), seed=21)
+    g = inputs.gates(inputs.custom_config("u", E=8, K=256, N=N, T=T, top_k=k))
+    ip = torch.randperm(T * k, generator=torch.Generator().manual_seed(5)).to(torch.int32)
+    out = gsg.unpermute_scale(Y.to(DEV), ip.to(DEV), g.to(DEV), k)
+    ref = ounperm.unpermute_scale(Y.view(torch.uint16).numpy(), ip.numpy(), g.numpy(), k)
+    np.testing.assert_array_equal(out.cpu().view(torch.uint16).numpy(), ref)
+
+
+# ---------------------------------------------------------------- grouped GEMM on oracle-packed inputs
+def _gemm_case(counts, N, K, seed=0, sparse=True):
+    E = len(counts)
+    cfg = inputs.custom_config("g", E=E, K=K, N=N, T=int(sum(counts)), top_k=1, w_sigma=0.02)
+    W = inputs.all_weights(cfg).numpy()
+    X = inputs.activations(cfg).float().numpy()
+    off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    sf = 32 if sparse else 16
+    a_codes, a_quad, s_x, q, sc = tl.oracle_act(X, sf, None, 1)
+    if sparse:
+        vals, meta, scs, sws, canon = tl.oracle_pack_sparse(W)
+        w = dict(values=vals, meta=meta, scales=scs, w_scale=sws)
+    else:
+        vals, scs, sws, canon = tl.oracle_pack_dense(W, 16)
+        w = dict(codes=vals, scales=scs, w_scale=sws)
+    return dict(E=E, N=N, K=K, R=int(off[-1]), off=off, a_codes=a_codes, a_quad=a_quad, s_x=s_x, q=q, sc=sc,
+                w=w, canon=canon, sws=sws, sf=sf)
+
+
+def _run_gemm(gsg, c, sparse, hint, out_dtype):
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+    act = gsg.QuantizedActivations(codes=t(c["a_codes"]), scales=t(c["a_quad"]),
+                                   x_scale=torch.tensor([c["s_x"]], dtype=torch.float32, device=DEV),
+                                   R=c["R"], K=c["K"], sf_block=c["sf"])
+    off = t(c["off"])
+    if sparse:
+        w = gsg.PackedSparseWeights(values=t(c["w"]["values"]), meta=t(c["w"]["meta"]), scales=t(c["w"]["scales"]),
+                                    w_scale=t(c["w"]["w_scale"]), E=c["E"], N=c["N"], K=c["K"])
+        return gsg.grouped_sparse_gemm(act, w, off, max_rows_per_expert=hint, out_dtype=out_dtype)
+    w = gsg.PackedDenseWeights(codes=t(c["w"]["codes"]), scales=t(c["w"]["scales"]), w_scale=t(c["w"]["w_scale"]),
+                               E=c["E"], N=c["N"], K=c["K"])
+    return gsg.grouped_dense_gemm(act, w, off, max_rows_per_expert=hint, out_dtype=out_dtype)
+
+
+GEMM_CASES = [
+    ([16], 128, 256),                              # one tile
+    ([5, 0, 33], 256, 512),                        # ragged, an empty expert, two n-tiles
+    ([0, 1, 7, 8, 9, 127, 128, 129], 128, 768),    # the ragged-tail ladder
+    ([300, 2, 64], 384, 1024),
+]
+
+
+@pytest.mark.parametrize("counts,N,K", GEMM_CASES)
+@pytest.mark.parametrize("hint", [-1, 16, 64])
+def test_sparse_gemm_oracle_inputs(gsg, counts, N, K, hint):
+    c = _gemm_case(counts, N, K, sparse=True)
+    y = _run_gemm(gsg, c, True, hint, torch.float32)
+    torch.cuda.synchronize()
+    _status_ok(gsg)
+    y_ref, bound = tl.reference_rows(np.arange(c["R"]), c["off"], c["q"], c["sc"], 32, c["canon"], c["s_x"], c["sws"])
+    tl.assert_gemm_close(y[:c["R"]], y_ref, bound, f"sparse {counts} hint {hint}")
+
+
+@pytest.mark.parametrize("counts,N,K", GEMM_CASES[:3])
+def test_sparse_gemm_bf16_output(gsg, counts, N, K):
+    c = _gemm_case(counts, N, K, sparse=True)
+    y = _run_gemm(gsg, c, True, -1, torch.bfloat16)
+    y_ref, bound = tl.reference_rows(np.arange(c["R"]), c["off"], c["q"], c["sc"], 32, c["canon"], c["s_x"], c["sws"])
+    tl.assert_gemm_close(y[:c["R"]], y_ref, bound, "sparse bf16")
+
+
+@pytest.mark.parametrize("counts,N,K", GEMM_CASES)
+def test_dense_gemm_oracle_inputs(gsg, counts, N, K):
+    c = _gemm_case(counts, N, K, sparse=False)
+    y = _run_gemm(gsg, c, False, -1, torch.float32)
+    y_ref, bound = tl.reference_rows(np.arange(c["R"]), c["off"], c["q"], c["sc"], 16, c["canon"], c["s_x"],
+                                     c["sws"], sparse=False, w_sf=16)
+    tl.assert_gemm_close(y[:c["R"]], y_ref, bound, f"dense {counts}")
+
+
+def test_gemm_deterministic(gsg):
+    c = _gemm_case([40, 3, 77], 256, 512, sparse=True)
+    y1 = _run_gemm(gsg, c, True, 32, torch.float32)
+    y2 = _run_gemm(gsg, c, True, 32, torch.float32)
+    assert torch.equal(y1, y2)
+
+
+def test_dense_and_sparse_agree_on_48_weights(gsg):
+    """The control differs from the sparse kernel only in sparsity: a W that is already paired
+    4:8 gives results within tolerance of one reference on both (32-blocks copied into 16-blocks)."""
+    counts, N, K = [20, 9], 128, 512
+    c = _gemm_case(counts, N, K, sparse=True)
+    # dense weights: scatter the retained codes with +0 at pruned slots; duplicate each 32-block scale
+    dv, ds = [], []
+    for (codes, pats, scales) in c["canon"]:
+        full = np.zeros((N, K // 8, 4, 2), dtype=np.uint8)
+        np.put_along_axis(full, opack.pattern_pairs(pats)[..., None].repeat(2, axis=-1),
+                          codes.reshape(N, K // 8, 2, 2), axis=-2)
+        dv.append(olayout.tile_values_fast(full.reshape(N, K)).reshape(-1))
+        ds.append(olayout.tile_scales(np.repeat(scales, 2, axis=1)).reshape(-1))
+    # activations with 16-blocks carrying the same scale as their 32-block
+    q, sc = c["q"], c["sc"]
+    d = dict(c)
+    d["w"] = dict(codes=np.concatenate(dv), scales=np.concatenate(ds), w_scale=c["sws"])
+    d["a_quad"] = olayout.quad_act_scales(np.repeat(sc, 2, axis=1)).reshape(-1)
+    d["sf"] = 16
+    y_sparse = _run_gemm(gsg, c, True, -1, torch.float32)
+    y_dense = _run_gemm(gsg, d, False, -1, torch.float32)
+    y_ref, bound = tl.reference_rows(np.arange(c["R"]), c["off"], q, sc, 32, c["canon"], c["s_x"], c["sws"])
+    tl.assert_gemm_close(y_sparse[:c["R"]], y_ref, bound, "sparse")
+    tl.assert_gemm_close(y_dense[:c["R"]], y_ref, bound, "dense control")
+
+
+# ---------------------------------------------------------------- the whole path
+@pytest.mark.parametrize("name", ["tiny", "30b_down_decode", "1t_down_decode_b1"])
+def test_pipeline_matches_oracle(gsg, name):
+    cfg = inputs.CONFIGS[name]
+    E, N, K = cfg.E, cfg.N, cfg.K
+    W = torch.stack([inputs.expert_weight(cfg, e, DEV) for e in range(E)])
+    X = inputs.activations(cfg)
+    ids = inputs.routing(cfg)
+    gates = inputs.gates(cfg)
+    pw = gsg.pack_sparse_nvfp4(W)
+    r = gsg.moe_route_permute(ids.to(DEV), E)
+    qa = gsg.quantize_act_nvfp4(X.to(DEV), 32, r.inv_perm, cfg.top_k)
+    counts = torch.bincount(ids.reshape(-1).long(), minlength=E)
+    Y = gsg.grouped_sparse_gemm(qa, pw, r.offsets, int(counts.max()), out_dtype=torch.float32)
+    out = gsg.unpermute_scale(Y.to(torch.bfloat16), r.inv_perm, gates.to(DEV), cfg.top_k)
+    torch.cuda.synchronize()
+    _status_ok(gsg)
+    # oracle, from the same inputs only
+    off, ps, ip = tl.route_np(ids, E)
+    _, _, s_x, q, sc = tl.oracle_act(X.float().numpy(), 32, ps, cfg.top_k)
+    touched = np.unique(ids.numpy())
+    rows = np.arange(cfg.R)
+    canon = {}
+    sws = np.zeros(E, dtype=np.float32)
+    for e in touched:
+        codes, pats, scales, s_w = opack.pack_sparse_expert(W[int(e)].cpu().numpy())
+        canon[int(e)] = (codes, pats, scales)
+        sws[e] = s_w
+    y_ref, bound = tl.reference_rows(rows, off, q, sc, 32, canon, s_x, sws)
+    tl.assert_gemm_close(Y[:cfg.R], y_ref, bound, f"pipeline GEMM {name}")
+    # scatter: tolerance form against y_ref (sum_j |g_j| (tol_j) + bf16 rounding of the sum)
+    g = gates.numpy().astype(np.float64)
+    yr = y_ref[ip.reshape(cfg.T, cfg.top_k)]
+    br = bound[ip.reshape(cfg.T, cfg.top_k)]
+    ref = np.einsum("tj,tjn->tn", g, yr)
+    tol = np.einsum("tj,tjn->tn", np.abs(g), 2.0 ** -10 * br + 1e-6 + tl.ogemm.bf16_half_ulp(np.abs(yr) + 1e-6))
+    tol = tol + 2.0 ** -8 * np.abs(ref) + 1e-6
+    err = np.abs(out.float().cpu().numpy() - ref)
+    assert np.all(err <= tol), float(np.max(err / tol))
+
+
+def test_gemm_full_size_sampled_30b_up(gsg):
+    """The bench workload (30B-A3B-shaped up-projection prefill) at full size; sampled rows."""
+    cfg = inputs.CONFIGS["30b_up_prefill"]
+    E, N, K = cfg.E, cfg.N, cfg.K
+    pw = gsg.PackedSparseWeights(
+        values=torch.empty(E * N * K // 4, dtype=torch.uint8, device=DEV),
+        meta=torch.empty(E * N * K // 16, dtype=torch.uint8, device=DEV),
+        scales=torch.empty(E * N * K // 32, dtype=torch.uint8, device=DEV),
+        w_scale=torch.empty(E, dtype=torch.float32, device=DEV), E=E, N=N, K=K)
+    ids = inputs.routing(cfg)
+    off, ps, ip = tl.route_np(ids, E)
+    counts = np.diff(off)
+    sample_e = sorted({int(np.argmax(counts)), int(np.argmin(counts)), 0, E - 1, 17, 64})
+    canon, sws = {}, np.zeros(E, dtype=np.float32)
+    for e in range(E):
+        We = inputs.expert_weight(cfg, e, DEV)
+        sub = gsg.PackedSparseWeights(values=pw.values[e * N * K // 4:(e + 1) * N * K // 4],
+                                      meta=pw.meta[e * N * K // 16:(e + 1) * N * K // 16],
+                                      scales=pw.scales[e * N * K // 32:(e + 1) * N * K // 32],
+                                      w_scale=pw.w_scale[e:e + 1], E=1, N=N, K=K)
+        gsg.pack_sparse_nvfp4(We[None], out=sub)
+        if e in sample_e:
+            codes, pats, scales, s_w = opack.pack_sparse_expert(We.cpu().numpy())
+            canon[e] = (codes, pats, scales)
+            sws[e] = s_w
+            np.testing.assert_array_equal(sub.values.cpu().numpy(), olayout.tile_values_fast(codes).reshape(-1))
+            np.testing.assert_array_equal(sub.meta.cpu().numpy(), olayout.tile_meta(pats).reshape(-1))
+            np.testing.assert_array_equal(sub.scales.cpu().numpy(), olayout.tile_scales(scales).reshape(-1))
+            assert sub.w_scale.item() == s_w
+    X = inputs.activations(cfg)
+    r = gsg.moe_route_permute(ids.to(DEV), E)
+    qa = gsg.quantize_act_nvfp4(X.to(DEV), 32, r.inv_perm, cfg.top_k)
+    Y = gsg.grouped_sparse_gemm(qa, pw, r.offsets, int(counts.max()), out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    _status_ok(gsg)
+    _, _, s_x, q, sc = tl.oracle_act(X.float().numpy(), 32, ps, cfg.top_k)
+    rows = []
+    for e in sample_e:
+        lo, hi = int(off[e]), int(off[e + 1])
+        if hi > lo:
+            rows += sorted({lo, hi - 1, (lo + hi) // 2, min(lo + 128, hi - 1), min(lo + 129, hi - 1)})
+    y_ref, bound = tl.reference_rows(np.array(rows), off, q, sc, 32, canon, s_x, sws)
+    tl.assert_gemm_close(Y[torch.tensor(rows, device=DEV)], y_ref, bound, "30b_up_prefill sampled")
