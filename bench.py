@@ -1,0 +1,510 @@
+#!/usr/bin/env python3
+"""Benchmark of the grouped sparse-NVFP4 expert GEMM path on B200.
+
+One step = one pass of the hot path over one batch of routed tokens, inputs resident in HBM:
+moe_route_permute -> quantize_act_nvfp4 (fused dispatch) -> grouped_sparse_gemm ->
+unpermute_scale, replayed as one CUDA graph (the weights are packed once, offline, as in
+serving).  The L2 cache is flushed (a 256 MB write) before every timed step; each step is timed
+with CUDA events on the launching stream and the flush is left outside the events.
+
+Reported (rank 0, one JSON line):
+  value     dense-equivalent TFLOP/s of the whole step (2*R*N*K per step, the unit the sparse
+            NVFP4 tensor peak is quoted in), summed over ranks / max time over ranks
+  e2e       the same metric through the Python API with host (pinned) inputs and outputs,
+            host<->device copies inside the timed region
+  roofline  the grouped GEMM kernel alone: algorithmic bytes per launch / its event time
+            against the measured HBM copy bandwidth
+  cpu_baseline  the CPU oracle timed on a bounded sample of the same workload (N=1, rank 0)
+  control   the dense-NVFP4 grouped GEMM on the same routed activations
+
+--impl reference runs the CPU oracle as the reference arm (the pages ship no implementation).
+Multi-GPU (torchrun): every rank runs an independent replica (weak scaling); the path has no
+data exchange on one GPU's workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import grouped_sparse_gemm_b200 as gsg  # noqa: E402
+from grouped_sparse_gemm_b200 import inputs  # noqa: E402
+
+DEFAULT_CONFIG = "30b_up_prefill"
+METRIC = "grouped sparse-NVFP4 GEMM TFLOP/s + weight GB/s, as % of B200 roofline"
+SPARSE_NVFP4_PEAK_TFLOPS_NOMINAL = 18000.0     # the pages' sparse NVFP4 figure (dense-equivalent)
+HBM_NOMINAL_GBS = 8000.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ------------------------------------------------------------------ distributed plumbing
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device(f"cuda:{local}"))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int, dev) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ peaks and clocks
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                       "-i", str(gpu_index), "-lms", "50"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except Exception:
+            self.p.kill()
+        self.f.flush()
+        self.f.seek(0)
+        rows = [r.split(",") for r in self.f.read().strip().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        sm, reasons, smax = [], set(), None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                smax = float(r[2])
+                for n, v in zip(names, r[5:9]):
+                    if v.strip().lower() == "active":
+                        reasons.add(n)
+            except (ValueError, IndexError):
+                continue
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": 0}
+        busy = [s for s in sm if s > 0.5 * max(sm)]
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ workload
+class Workload:
+    """Packed weights, routed inputs and every output buffer of one step, resident on the GPU."""
+
+    def __init__(self, cfg: inputs.MoEConfig, dev: torch.device, with_dense: bool = True):
+        self.cfg, self.dev = cfg, dev
+        E, N, K, T, k = cfg.E, cfg.N, cfg.K, cfg.T, cfg.top_k
+        u8 = dict(dtype=torch.uint8, device=dev)
+        self.pw = gsg.PackedSparseWeights(values=torch.empty(E * N * K // 4, **u8),
+                                          meta=torch.empty(E * N * K // 16, **u8),
+                                          scales=torch.empty(E * N * K // 32, **u8),
+                                          w_scale=torch.empty(E, dtype=torch.float32, device=dev), E=E, N=N, K=K)
+        self.pd = None
+        if with_dense:
+            self.pd = gsg.PackedDenseWeights(codes=torch.empty(E * N * K // 2, **u8),
+                                             scales=torch.empty(E * N * K // 16, **u8),
+                                             w_scale=torch.empty(E, dtype=torch.float32, device=dev), E=E, N=N, K=K)
+        ws_pack = torch.empty(max(gsg.workspace_size(gsg.OP_PACK_SPARSE, 1, N, K), 16), **u8)
+        for e in range(E):          # generate and pack one expert at a time (offline step)
+            We = inputs.expert_weight(cfg, e, str(dev))[None]
+            vs, ms, ss = N * K // 4, N * K // 16, N * K // 32
+            sub = gsg.PackedSparseWeights(values=self.pw.values[e * vs:(e + 1) * vs], meta=self.pw.meta[e * ms:(e + 1) * ms],
+                                          scales=self.pw.scales[e * ss:(e + 1) * ss], w_scale=self.pw.w_scale[e:e + 1],
+                                          E=1, N=N, K=K)
+            gsg.pack_sparse_nvfp4(We, out=sub, workspace=ws_pack)
+            if with_dense:
+                cs, ds = N * K // 2, N * K // 16
+                subd = gsg.PackedDenseWeights(codes=self.pd.codes[e * cs:(e + 1) * cs],
+                                              scales=self.pd.scales[e * ds:(e + 1) * ds],
+                                              w_scale=self.pd.w_scale[e:e + 1], E=1, N=N, K=K)
+                gsg.pack_dense_nvfp4(We, out=subd, workspace=ws_pack)
+            del We
+        torch.cuda.synchronize()
+        self.X_h = inputs.activations(cfg)
+        self.ids_h = inputs.routing(cfg)
+        self.gates_h = inputs.gates(cfg)
+        self.X = self.X_h.to(dev)
+        self.ids = self.ids_h.to(dev)
+        self.gates = self.gates_h.to(dev)
+        counts = torch.bincount(self.ids_h.reshape(-1).long(), minlength=E)
+        self.counts = counts
+        self.max_rows = int(counts.max())
+        self.touched = int((counts > 0).sum())
+        R = cfg.R
+        self.route = gsg.Routing(offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+                                 perm_src=torch.empty(R, dtype=torch.int32, device=dev),
+                                 inv_perm=torch.empty(R, dtype=torch.int32, device=dev), T=T, k=k, E=E)
+        self.ws_route = torch.empty(max(gsg.workspace_size(gsg.OP_ROUTE, E, 0, 0, T, k), 16), **u8)
+        self.ws_quant = torch.empty(max(gsg.workspace_size(gsg.OP_QUANTIZE, 0, 0, K, T, k), 16), **u8)
+        self.qa = gsg.QuantizedActivations(codes=torch.empty(R, K // 2, **u8),
+                                           scales=torch.empty(gsg.act_scales_bytes(R, K, 32), **u8),
+                                           x_scale=torch.empty(1, dtype=torch.float32, device=dev), R=R, K=K,
+                                           sf_block=32)
+        self.Y = torch.empty(R, N, dtype=torch.bfloat16, device=dev)
+        self.out = torch.empty(T, N, dtype=torch.bfloat16, device=dev)
+        self.qa16 = None
+        self.Yd = None
+        if with_dense:
+            self.Yd = torch.empty(R, N, dtype=torch.bfloat16, device=dev)
+
+    # one step of the hot path
+    def step(self):
+        c = self.cfg
+        gsg.moe_route_permute(self.ids, c.E, out=self.route, workspace=self.ws_route)
+        gsg.quantize_act_nvfp4(self.X, 32, self.route.inv_perm, c.top_k, out=self.qa, workspace=self.ws_quant)
+        gsg.grouped_sparse_gemm(self.qa, self.pw, self.route.offsets, self.max_rows, out=self.Y)
+        gsg.unpermute_scale(self.Y, self.route.inv_perm, self.gates, c.top_k, out=self.out)
+
+    def launches_per_step(self) -> int:
+        route = 1 if self.cfg.R <= 8192 else 3
+        return route + 2 + 1 + 1        # route, amax + quantize, GEMM, scatter
+
+    def gemm(self):
+        gsg.grouped_sparse_gemm(self.qa, self.pw, self.route.offsets, self.max_rows, out=self.Y)
+
+    def prepare_dense(self):
+        self.qa16 = gsg.quantize_act_nvfp4(self.X, 16, self.route.inv_perm, self.cfg.top_k)
+
+    def dense_gemm(self):
+        gsg.grouped_dense_gemm(self.qa16, self.pd, self.route.offsets, self.max_rows, out=self.Yd)
+
+    # algorithmic bytes of one grouped GEMM launch
+    def gemm_bytes(self):
+        c = self.cfg
+        w = self.touched * c.N * c.K * 11 // 32          # 2.75 bit per weight of every touched expert
+        a = c.R * c.K // 2 + c.R * c.K // 32            # activation codes + one scale per 32
+        y = c.R * c.N * 2
+        return w, a, y
+
+    def dense_gemm_bytes(self):
+        c = self.cfg
+        return self.touched * c.N * c.K * 9 // 16 + c.R * c.K // 2 + c.R * c.K // 16 + c.R * c.N * 2
+
+
+def capture(fn, warm=2):
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for _ in range(warm):
+            fn()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def timed_ms(fn, steps: int, flush_buf: torch.Tensor, world: int):
+    """Mean device time of fn over `steps` runs, L2 flushed before each (outside the events)."""
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush_buf.fill_(i & 0xFF)
+        starts[i].record()
+        fn()
+        ends[i].record()
+    torch.cuda.synchronize()
+    barrier(world)
+    ts = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    return sum(ts) / steps, ts
+
+
+# ------------------------------------------------------------------ CPU oracle (baseline / reference arm)
+class OracleSample:
+    """The CPU oracle on a bounded sample of the workload.
+
+    Prerequisites (untimed): oracle routing and activation quantization of the whole batch, and
+    oracle packing of the sampled experts' weights (packing is the offline step).  Timed unit:
+    the oracle's grouped GEMM for one (expert, 128-row weight tile) -- decode of the packed
+    weights and of the expert's activation rows, fp64 matmul, tensor scales.
+    """
+
+    def __init__(self, cfg, X_h, ids_h, n_experts: int, seed: int = 0):
+        from oracle import pack as opack
+        from oracle import quant as oquant
+        from oracle import route as oroute
+        self.cfg = cfg
+        ids = ids_h.numpy()
+        counts = np.bincount(ids.reshape(-1), minlength=cfg.E)
+        order = [int(e) for e in np.argsort(-counts, kind="stable") if counts[e] > 0]
+        big = order[: max(1, n_experts // 2)]
+        rng = np.random.default_rng(seed)
+        rest = [int(e) for e in rng.permutation(order[len(big):])][: max(0, n_experts - len(big))]
+        self.experts = big + rest
+        self.off, perm_src, _ = oroute.route(ids, cfg.E)
+        self.q, self.sc, self.s_x = oquant.quantize_routed(X_h.float().numpy(), 32, perm_src, cfg.top_k)
+        self.packed = {e: opack.pack_sparse_expert(inputs.expert_weight(cfg, e).numpy()) for e in self.experts}
+        self.units = [(e, nt) for e in self.experts for nt in range(cfg.N // 128)]
+
+    def run(self, units):
+        from oracle import gemm as ogemm
+        from oracle import pack as opack
+        from oracle import quant as oquant
+        rows = 0
+        t0 = time.perf_counter()
+        for e, nt in units:
+            lo, hi = int(self.off[e]), int(self.off[e + 1])
+            codes, pats, scales, s_w = self.packed[e]
+            sl = slice(nt * 128, (nt + 1) * 128)
+            wd = opack.decode_sparse_expert(codes[sl], pats[sl], scales[sl])
+            ad = oquant.decode_rows(self.q[lo:hi], self.sc[lo:hi], 32)
+            ogemm.gemm_rows(ad, wd, float(self.s_x) * float(s_w))
+            rows += hi - lo
+        dt = time.perf_counter() - t0
+        return dt, 2.0 * rows * 128 * self.cfg.K
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def workload_config(cfg, l2="flushed before every timed step (256 MB write, outside the events)"):
+    return {"workload": f"{cfg.name}: E={cfg.E} K={cfg.K} N={cfg.N}, {cfg.T} tokens top-{cfg.top_k} "
+                        f"(R={cfg.R}), routing {cfg.routing}"
+                        + (f" s={cfg.zipf_s}" if cfg.routing == "zipf" else ""),
+            "E": cfg.E, "K": cfg.K, "N": cfg.N, "tokens": cfg.T, "top_k": cfg.top_k, "routed_rows": cfg.R,
+            "weights": "paired 4:8 NVFP4 (2.75 bit/weight)", "l2": l2}
+
+
+def run_reference(args, world, rank):
+    """Reference arm: the CPU oracle, a bounded sample per step (about 90 s in all), rank 0 only."""
+    if rank != 0:
+        return
+    cfg = inputs.CONFIGS[args.config]
+    smp = OracleSample(cfg, inputs.activations(cfg), inputs.routing(cfg), n_experts=2)
+    t_unit, _ = smp.run(smp.units[:2])
+    t_unit /= 2
+    per_step = int(max(1, min(len(smp.units), 90.0 / max(1, args.steps + args.warmup) / max(t_unit, 1e-6))))
+    units = smp.units[:per_step]
+    for _ in range(args.warmup):
+        smp.run(units)
+    ts, fl = [], 0.0
+    for _ in range(args.steps):
+        dt, fl = smp.run(units)
+        ts.append(dt)
+    mean = sum(ts) / len(ts)
+    value = fl / mean / 1e12
+    sample = (f"per step: the oracle grouped GEMM (packed-weight and activation decode + fp64 matmul) of "
+              f"{per_step} (expert, 128-row weight tile) units of experts {smp.experts}; routing, activation "
+              f"quantization and weight packing done once beforehand")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(cfg, l2="n/a (CPU)"),
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def traffic_from_profiles(config_name: str):
+    """DRAM bytes per GEMM launch from the committed ncu summary, if the kernel is unchanged."""
+    p = os.path.join(ROOT, "profiles", "gemm_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    src = os.path.join(ROOT, "grouped_sparse_gemm_b200", "csrc", "gsg_gemm.cu")
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    ent = d.get(config_name)
+    if not ent or ent.get("gemm_src_sha") != sha:
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+def run_ours(args, world, rank, local):
+    dev = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(dev)
+    gsg.load_library()
+    cfg = inputs.CONFIGS[args.config]
+    wl = Workload(cfg, dev, with_dense=not args.quick)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    wl.step()
+    torch.cuda.synchronize()
+    st = gsg.get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after the first step")
+    g_step = capture(wl.step)
+    g_gemm = capture(wl.gemm)
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        g_step.replay()
+    torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    step_ms, _ = timed_ms(g_step.replay, args.steps, flush, world)
+    gemm_ms, _ = timed_ms(g_gemm.replay, args.steps, flush, world)
+    clk = clocks.stop()
+    step_ms = max_over_ranks(step_ms, world, dev)
+    gemm_ms_max = max_over_ranks(gemm_ms, world, dev)
+    st = gsg.get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after timing")
+
+    flops = 2.0 * cfg.R * cfg.N * cfg.K
+    w_b, a_b, y_b = wl.gemm_bytes()
+    value = world * flops / (step_ms * 1e-3) / 1e12
+    peaks, peak_kind = measured_peaks()
+    hbm_peak = float(peaks["hbm_gbs"])
+    tensor_peak = float(peaks["bf16_tflops"]) * 8.0     # sparse NVFP4 / dense bf16 nominal ratio 18 / 2.25
+    gemm_bytes = w_b + a_b + y_b
+    achieved_gbs = gemm_bytes / (gemm_ms * 1e-3) / 1e9
+    gemm_tflops = flops / (gemm_ms * 1e-3) / 1e12
+
+    # end to end through the Python API: pinned host inputs -> device, step, result -> pinned host
+    e2e = None
+    if not args.quick:
+        X_p, ids_p, g_p = wl.X_h.pin_memory(), wl.ids_h.pin_memory(), wl.gates_h.pin_memory()
+        out_p = torch.empty(cfg.T, cfg.N, dtype=torch.bfloat16).pin_memory()
+
+        def e2e_step():
+            wl.X.copy_(X_p, non_blocking=True)
+            wl.ids.copy_(ids_p, non_blocking=True)
+            wl.gates.copy_(g_p, non_blocking=True)
+            wl.step()
+            out_p.copy_(wl.out, non_blocking=True)
+        for _ in range(3):
+            e2e_step()
+        e2e_ms, _ = timed_ms(e2e_step, max(10, args.steps // 10), flush, world)
+        e2e_ms = max_over_ranks(e2e_ms, world, dev)
+        h2d = X_p.numel() * 2 + ids_p.numel() * 4 + g_p.numel() * 4
+        e2e = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(out_p.numel() * 2),
+               "path": "pinned host -> device copies, 4 library calls via the Python binding, result -> pinned host"}
+
+    control = None
+    if not args.quick:
+        wl.prepare_dense()
+        g_dense = capture(wl.dense_gemm)
+        dense_ms, _ = timed_ms(g_dense.replay, max(10, args.steps // 2), flush, world)
+        control = {"kernel": "dense-NVFP4 grouped GEMM (16-element UE4M3 blocks, 4.5 bit/weight), same skeleton",
+                   "gemm_ms": dense_ms, "tflops": flops / (dense_ms * 1e-3) / 1e12,
+                   "hbm_gbs": wl.dense_gemm_bytes() / (dense_ms * 1e-3) / 1e9,
+                   "sparse_speedup": dense_ms / gemm_ms}
+
+    cpu = None
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        smp = OracleSample(cfg, wl.X_h, wl.ids_h, args.cpu_experts)
+        dt, fl = smp.run(smp.units)
+        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": (f"the oracle grouped GEMM (packed-weight and activation decode + fp64 matmul) of all "
+                          f"{cfg.N // 128} weight tiles of {len(smp.experts)} experts (the largest half and seeded "
+                          f"random others, {int(sum(smp.off[e + 1] - smp.off[e] for e in smp.experts))} of "
+                          f"{cfg.R} routed rows), {dt:.1f} s; routing, quantization and packing untimed")}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic (seeded; random weights, no checkpoint)",
+            "config": workload_config(cfg),
+            "weight_gbs": world * w_b / (step_ms * 1e-3) / 1e9,
+            "roofline_pct": {
+                "tensor_sparse_nvfp4_nominal_18pf": 100.0 * value / world / SPARSE_NVFP4_PEAK_TFLOPS_NOMINAL,
+                "hbm_nominal_8tbs": 100.0 * (gemm_bytes / (step_ms * 1e-3) / 1e9) / HBM_NOMINAL_GBS},
+            "gemm": {"ms": gemm_ms_max, "tflops": gemm_tflops, "weight_gbs": w_b / (gemm_ms * 1e-3) / 1e9,
+                     "total_gbs": achieved_gbs, "token_tile": gsg_token_tile(wl.max_rows),
+                     "touched_experts": wl.touched, "max_rows_per_expert": wl.max_rows,
+                     "tensor_frac_of_measured": gemm_tflops / tensor_peak},
+            "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": achieved_gbs / hbm_peak, "traffic": traffic_from_profiles(cfg.name),
+                         "kernel": "grouped_gemm_kernel<sparse>",
+                         "algorithmic_bytes_per_launch": int(gemm_bytes),
+                         "peak_source": f"{peak_kind} hbm_gbs (burst copy)"},
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "control": control,
+            "gpu_launches": wl.launches_per_step() * args.steps,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def gsg_token_tile(max_rows: int) -> int:
+    for bn in (16, 32, 64):
+        if 0 < max_rows <= bn:
+            return bn
+    return 128
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(inputs.CONFIGS))
+    ap.add_argument("--quick", action="store_true", help="skip e2e, dense control and CPU baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-experts", type=int, default=24)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -50,7 +50,8 @@ def reference_rows(rows, off, a_codes, a_scales, sf_block, w_canon, s_x, s_w, sp
     """y_ref and bound for the given routed rows (all N columns), fp64."""
     rows = np.asarray(rows, dtype=np.int64)
     experts = ogemm.expert_of_rows(off, rows)
-    N = (w_canon[0][0].shape[0])
+    first = next(iter(w_canon.values())) if isinstance(w_canon, dict) else w_canon[0]
+    N = first[0].shape[0]
     y = np.zeros((rows.size, N))
     b = np.zeros((rows.size, N))
     for e in np.unique(experts):
