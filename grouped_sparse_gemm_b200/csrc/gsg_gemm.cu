@@ -6,15 +6,18 @@
 // §2 "Hardware opportunity" (p.3) -- paired 4:8 NVFP4 runs at twice the dense NVFP4 rate;
 // §D.2 (p.19) -- a dense control that differs from the sparse kernel only in sparsity.
 //
-// One CTA per SM, 192 threads, warp-specialised:
-//   warp 0      producer: per 256-wide K chunk, bulk copies of the pre-tiled weight values,
-//               metadata and scales, one tensor-map TMA box of activation codes (128B swizzle)
-//               and bulk copies of the activation scale atoms, into a ring of smem stages.
-//   warp 1      TMEM owner and MMA issuer: tcgen05.cp metadata/scales into TMEM, then
-//               tcgen05.mma(.sp) kind::mxf4nvf4 block_scale (M = 128 weight rows, N = token
-//               tile, K = 128 logical sparse / 64 dense), accumulating in one of two TMEM
-//               accumulators; tcgen05.commit releases smem stages and hands tiles to the epilogue.
-//   warps 2..5  epilogue: tcgen05.ld accumulator lanes, multiply by s_x * s_w[e], store rows of Y.
+// One CTA per SM, 352 threads (11 warps), warp-specialised around one shared-memory ring whose
+// stages hold 256 or 512 logical K of one tile (weights, activation codes and both scales):
+//   warp 0      weight producer: three bulk copies per stage (pre-tiled values, metadata, scales).
+//   warp 2      activation producer: tensor-map TMA boxes (128B swizzle) of only the token rows the
+//               tile holds, and one 3-D TMA box of the activation scale atoms.
+//   warps 7..10 scale/metadata loaders, one per TMEM lane quadrant: read the stage's metadata and
+//               scale atoms from shared memory and tcgen05.st them into one of three TMEM sets.
+//   warp 1      TMEM owner and MMA issuer: per stage only tcgen05.mma(.sp) kind::mxf4nvf4
+//               block_scale (M = 128 weight rows, N = the tile's token count rounded to 16, K = 128
+//               logical sparse / 64 dense) and one tcgen05.commit; up to eight TMEM accumulators.
+//   warps 3..6  epilogue: tcgen05.ld accumulator lanes, multiply by s_x * s_w[e], store rows of Y.
+// Every TMA and tcgen05 instruction is issued by an elected lane of a converged warp.
 // Tiles are (expert e, 128 weight rows nt, token tile mt) in e -> nt -> mt order; CTAs take
 // tiles round-robin.  Experts with no rows produce no tiles.  Every mbarrier wait is bounded:
 // on expiry the kernel records GSG_ERR_DEVICE_TIMEOUT, drains its own copies and MMAs, frees
@@ -25,14 +28,14 @@
 
 namespace gsg {
 
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 352;
 constexpr int kMaxE = 1024;
+constexpr int kMaxAcc = 8;
+constexpr int kNSets = 3;                  // TMEM sets of metadata + scales
+constexpr uint32_t kSetCols = 64;
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;   // 2 s
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColAcc1 = 128;
-constexpr uint32_t kColMeta = 256;
-constexpr uint32_t kColSFA = 272;
-constexpr uint32_t kColSFB = 304;
+constexpr uint32_t kColAcc = kNSets * kSetCols;       // first accumulator (192)
 
 struct GemmParams {
   const uint8_t* a_scales;
@@ -44,8 +47,8 @@ struct GemmParams {
   const int32_t* off;
   void* Y;
   int* status;
-  int E, N, K, R, BN, y_f32, rcap;
-  int stages, stage_bytes;
+  int E, N, K, R, y_f32, rcap;
+  int stages, nacc;
 };
 
 // ------------------------------------------------------------------ PTX wrappers
@@ -66,48 +69,96 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
+// The issue wrappers below are executed by a whole converged warp: elect.sync picks one lane
+// and predicates the instruction on it, so the warp never diverges around a TMA or tcgen05
+// instruction (issuing them from a lone lane of a diverged warp costs several times more).
+#define GSG_ELECT "elect.sync _|P, 0xffffffff;\n\t"
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+  asm volatile("{\n\t.reg .pred P;\n\t" GSG_ELECT "@P mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n\t}" ::"r"(bar),
+               "r"(bytes)
+               : "memory");
 }
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "{\n\t.reg .pred P;\n\t" GSG_ELECT
+      "@P cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n\t}" ::"r"(dst),
       "l"(src), "r"(bytes), "r"(bar)
       : "memory");
 }
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+      "{\n\t.reg .pred P;\n\t" GSG_ELECT
+      "@P cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n\t}" ::
           "r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
       : "memory");
 }
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z, uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t" GSG_ELECT
+      "@P cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];\n\t}" ::
+          "r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void lds128(uint32_t saddr, uint32_t& a, uint32_t& b, uint32_t& c, uint32_t& d) {
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(a), "=r"(b), "=r"(c), "=r"(d) : "r"(saddr) : "memory");
+}
+// tcgen05.st of N consecutive 32-bit columns for the 32 lanes of this warp's quadrant.
+__device__ __forceinline__ void tc_st_x4(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(r[0]), "r"(r[1]),
+               "r"(r[2]), "r"(r[3])
+               : "memory");
+}
+__device__ __forceinline__ void tc_st_x8(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+__device__ __forceinline__ void tc_st_x16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// Writes `kCols` (a multiple of 4) columns from registers, largest pieces first.
+template <int kCols>
+__device__ __forceinline__ void tc_st_cols(uint32_t taddr, const uint32_t* r) {
+  int c = 0;
+#pragma unroll
+  for (; c + 16 <= kCols; c += 16) tc_st_x16(taddr + c, r + c);
+  if constexpr (kCols % 16 >= 8) {
+    tc_st_x8(taddr + (kCols / 16) * 16, r + (kCols / 16) * 16);
+  }
+  if constexpr (kCols % 8 >= 4) {
+    tc_st_x4(taddr + (kCols / 8) * 8, r + (kCols / 8) * 8);
+  }
+}
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void tc_cp_128x128b(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
-__device__ __forceinline__ void tc_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+  asm volatile("{\n\t.reg .pred P;\n\t" GSG_ELECT
+               "@P tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
+               : "memory");
 }
 __device__ __forceinline__ void tc_mma_sparse(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                               uint32_t accumulate, uint32_t sfa, uint32_t sfb, uint32_t meta) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.sp.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, [%7], %3, [%5], [%6], p;\n\t}" ::"r"(d),
+      "{\n\t.reg .pred p, P;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t" GSG_ELECT
+      "@P tcgen05.mma.sp.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, [%7], %3, [%5], [%6], p;\n\t}" ::"r"(d),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb), "r"(meta)
       : "memory");
 }
 __device__ __forceinline__ void tc_mma_dense(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                              uint32_t accumulate, uint32_t sfa, uint32_t sfb) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+      "{\n\t.reg .pred p, P;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t" GSG_ELECT
+      "@P tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
       : "memory");
 }
@@ -159,68 +210,92 @@ __device__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_
   }
 }
 
+// Warp-uniform bounded wait: every lane polls, and the warp agrees on the outcome so that the
+// .sync instructions that follow (elect.sync, tcgen05.ld/st) always see a converged warp.
+__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* status) {
+  const bool ok = wait_bounded(bar, parity, abort_flag, status);
+  return __all_sync(0xffffffffu, ok);
+}
+
 struct TileCoord {
   int e, nt, mt;
 };
 
-// Largest e with pref[e] <= t (pref[0] = 0, pref[E] = total tiles).
-__device__ __forceinline__ TileCoord decode_tile(int t, const int* pref, const int* offs, int E, int NT, int BN) {
-  int lo = 0, hi = E;
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (pref[mid] <= t) lo = mid; else hi = mid;
+// Tiles are visited in increasing order, so the owning expert only moves forward: a linear
+// scan from the previous expert replaces a search.  pref[E] = total tiles > t ends the scan.
+struct TileCursor {
+  int e = 0;
+  __device__ __forceinline__ TileCoord next(int t, const int* pref, const int* offs, int BN) {
+    while (pref[e + 1] <= t) ++e;
+    TileCoord c;
+    c.e = e;
+    const int local = t - pref[e];
+    const int mte = (offs[e + 1] - offs[e] + BN - 1) / BN;
+    c.nt = local / mte;
+    c.mt = local % mte;
+    return c;
   }
-  TileCoord c;
-  c.e = lo;
-  const int local = t - pref[lo];
-  const int mte = (offs[lo + 1] - offs[lo] + BN - 1) / BN;
-  c.nt = local / mte;
-  c.mt = local % mte;
-  (void)NT;
-  return c;
-}
+};
 
-template <bool kSparse>
+// Compile-time stage geometry of one (sparse/dense, token tile) instantiation.
+template <bool kSparse, int kBN>
+struct Geo {
+  static constexpr int kKbLogical = kSparse ? 128 : 64;            // logical K per MMA
+  static constexpr int kKbPerChunk = kChunkK / kKbLogical;         // 2 sparse, 4 dense
+  static constexpr int kCPS = (kSparse ? kBN <= 64 : kBN <= 32) ? 2 : 1;   // 256-wide chunks per stage
+  static constexpr int kKbps = kCPS * kKbPerChunk;                 // MMAs per stage
+  static constexpr int kAChunk = kSparse ? 8192 : 16384;           // weight values per chunk
+  static constexpr int kMChunk = kSparse ? 2048 : 0;               // metadata per chunk
+  static constexpr int kBChunk = kBN * 128;                        // activation codes per chunk
+  static constexpr int kOffA = kCPS * kBChunk;                     // stage layout: B | A | M | SFA | SFB
+  static constexpr int kOffM = kOffA + kCPS * kAChunk;
+  static constexpr int kOffSFA = kOffM + kCPS * kMChunk;
+  static constexpr int kOffSFB = kOffSFA + kKbps * 512;
+  static constexpr int kStage = (kOffSFB + kKbps * 512 + 1023) / 1024 * 1024;
+  static constexpr int kMetaCols = kSparse ? 4 * kCPS : 0;         // TMEM set: meta | SFA | SFB
+  static constexpr int kColSFA = kMetaCols;
+  static constexpr int kColSFB = kMetaCols + 4 * kKbps;
+  static constexpr int kSetUsed = kMetaCols + 8 * kKbps;
+  static constexpr uint32_t kBStep = kSparse ? 64 : 32;            // B bytes per row per MMA
+  static constexpr int kBoxH = kBN < 32 ? kBN : 32;                // token rows per TMA box
+  static constexpr int kAccStride = kBN < 32 ? 32 : kBN;
+  static_assert(kSetUsed <= (int)kSetCols, "TMEM set too small");
+};
+
+template <bool kSparse, int kBN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams p) {
+grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ CUtensorMap tmap_sfb,
+                    const GemmParams p) {
+  using G = Geo<kSparse, kBN>;
   extern __shared__ uint8_t smem_raw[];
-  constexpr int kKbLogical = kSparse ? 128 : 64;       // logical K per MMA
-  constexpr int kKbPerStage = kChunkK / kKbLogical;    // MMAs per stage: 2 sparse, 4 dense
-  constexpr int kABytes = kSparse ? 8192 : 16384;      // weight values per stage
-  constexpr int kMetaBytes = kSparse ? 2048 : 0;
-  constexpr int kSfBytes = kKbPerStage * 512;
-  constexpr uint32_t kBStep = kSparse ? 64 : 32;       // B bytes per row consumed by one MMA
-
-  const int BN = p.BN, E = p.E, NT = p.N / kTileN, KC = p.K / kChunkK;
-  const int KBt = p.K / kKbLogical;
+  const int E = p.E, NT = p.N / kTileN, KC = p.K / kChunkK;
+  const int KBt = p.K / G::kKbLogical;
+  const int S = p.stages, NACC = p.nacc;
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int S = p.stages;
-  uint8_t* stage0 = base;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + (size_t)S * p.stage_bytes);
-  // bars: full[S], empty[S], accf[2], acce[2], drain
-  Ctl* ctl = reinterpret_cast<Ctl*>(bars + 2 * S + 5);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + (size_t)S * G::kStage);
+  // bars: full[S], empty[S], tfull[kNSets], accf[NACC], acce[NACC], drain
+  const int nbars = 2 * S + kNSets + 2 * NACC + 1;
+  Ctl* ctl = reinterpret_cast<Ctl*>(bars + nbars);
   int* offs = reinterpret_cast<int*>(ctl + 1);   // [E+1]
   int* pref = offs + (E + 1);                    // [E+1]
+  float* wsc = reinterpret_cast<float*>(pref + (E + 1));   // [E]
   volatile int* abort_flag = &ctl->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t bar0 = smem_u32(bars);
+  const uint32_t sbase = smem_u32(base);
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (S + s); };
-  auto accf_bar = [&](int a) { return bar0 + 8u * (2 * S + a); };
-  auto acce_bar = [&](int a) { return bar0 + 8u * (2 * S + 2 + a); };
-  const uint32_t drain_bar = bar0 + 8u * (2 * S + 4);
+  auto tfull_bar = [&](int s) { return bar0 + 8u * (2 * S + s); };
+  auto accf_bar = [&](int a) { return bar0 + 8u * (2 * S + kNSets + a); };
+  auto acce_bar = [&](int a) { return bar0 + 8u * (2 * S + kNSets + NACC + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * S + kNSets + 2 * NACC);
 
-  // ---- set-up: barriers, TMEM, tile schedule
+  // ---- set-up: barriers, TMEM, tile schedule, tensor scales
   if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(accf_bar(a), 1);
-      mbar_init(acce_bar(a), 4);
-    }
+    for (int s = 0; s < S; ++s) { mbar_init(full_bar(s), 2); mbar_init(empty_bar(s), 1); }
+    for (int s = 0; s < kNSets; ++s) mbar_init(tfull_bar(s), 4);
+    for (int a = 0; a < NACC; ++a) { mbar_init(accf_bar(a), 1); mbar_init(acce_bar(a), 4); }
     mbar_init(drain_bar, 1);
     ctl->abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -232,13 +307,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  // expert offsets (clamped to [0, R] and made monotone so a corrupt array can never send a
-  // copy or a store out of bounds) and the per-expert tile prefix
+  // expert offsets, clamped to [0, R] so a corrupt array can never send a copy or a store out
+  // of bounds (a decreasing pair makes that expert empty, see below)
   bool bad = false;
   for (int i = threadIdx.x; i <= E; i += blockDim.x) {
     int v = __ldg(p.off + i);
     if (v < 0 || v > p.R) { bad = true; v = v < 0 ? 0 : p.R; }
     offs[i] = v;
+    if (i < E) wsc[i] = __ldg(p.w_scale + i);
   }
   __syncthreads();
   {
@@ -249,7 +325,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams
     for (int e = e0; e < e1; ++e) {
       int rows = offs[e + 1] - offs[e];
       if (rows < 0) { bad = true; rows = 0; }
-      local += ((rows + BN - 1) / BN) * NT;
+      local += ((rows + kBN - 1) / kBN) * NT;
     }
     int incl = local;
 #pragma unroll
@@ -267,7 +343,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams
       pref[e] = run;
       int rows = offs[e + 1] - offs[e];
       if (rows < 0) rows = 0;
-      run += ((rows + BN - 1) / BN) * NT;
+      run += ((rows + kBN - 1) / kBN) * NT;
     }
     if (threadIdx.x == kGemmThreads - 1) pref[E] = before + incl;
   }
@@ -275,135 +351,181 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  // a decreasing offset makes that expert empty (its count is clamped to 0 above); keep the
-  // row arithmetic below consistent with that
   const int total_tiles = pref[E];
   const uint32_t tmem = ctl->tmem_base;
 
-  if (warp == 0) {
-    // =============================== producer
-    if (lane == 0) {
-      const uint32_t tx_bytes = (uint32_t)(BN * 128 + kABytes + kMetaBytes + 2 * kSfBytes);
-      int stage = 0;
-      uint32_t phase = 0;
-      int issued = 0;
-      for (int t = blockIdx.x; t < total_tiles && !*abort_flag; t += gridDim.x) {
-        const TileCoord c = decode_tile(t, pref, offs, E, NT, BN);
-        const int r0 = offs[c.e] + c.mt * BN;
-        const size_t tile = (size_t)c.e * NT + c.nt;
-        const uint8_t* av = p.w_vals + tile * KBt * 4096;
-        const uint8_t* am = kSparse ? p.w_meta + tile * KC * 2048 : nullptr;
-        const uint8_t* as = p.w_scales + tile * KBt * 512;
-        bool ok = true;
-        for (int kc = 0; kc < KC; ++kc) {
-          if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, p.status)) { ok = false; break; }
-          uint8_t* sb = stage0 + (size_t)stage * p.stage_bytes;
-          const uint32_t sB = smem_u32(sb);
-          const uint32_t sA = sB + BN * 128;
-          const uint32_t sM = sA + kABytes;
-          const uint32_t sSFA = sM + kMetaBytes;
-          const uint32_t sSFB = sSFA + kSfBytes;
-          const uint32_t fb = full_bar(stage);
-          mbar_arrive_expect_tx(fb, tx_bytes);
-          bulk_g2s(sA, av + (size_t)kc * kABytes, kABytes, fb);
-          if (kSparse) bulk_g2s(sM, am + (size_t)kc * 2048, 2048, fb);
-          bulk_g2s(sSFA, as + (size_t)kc * kSfBytes, kSfBytes, fb);
-          tma_load_2d(sB, &tmap_b, kc * 128, r0, fb);
-#pragma unroll
-          for (int h = 0; h < kKbPerStage; ++h) {
-            const size_t kb = (size_t)kc * kKbPerStage + h;
-            bulk_g2s(sSFB + h * 512, p.a_scales + (kb * p.rcap + r0) * 16, 512, fb);
-          }
-          ++issued;
-          if (++stage == S) { stage = 0; phase ^= 1u; }
+  if (warp == 0 || warp == 2) {
+    // =============================== producers: warp 0 weights, warp 2 activations
+    const bool wprod = warp == 0;
+    int s = 0, issued = 0;
+    uint32_t ph = 0;
+    TileCursor cur;
+    for (int t = blockIdx.x; t < total_tiles && !*abort_flag; t += gridDim.x) {
+      const TileCoord c = cur.next(t, pref, offs, kBN);
+      const size_t tile = (size_t)c.e * NT + c.nt;
+      const uint8_t* av = p.w_vals + tile * KBt * 4096;
+      const uint8_t* am = kSparse ? p.w_meta + tile * KC * 2048 : nullptr;
+      const uint8_t* as = p.w_scales + tile * KBt * 512;
+      const int r0 = offs[c.e] + c.mt * kBN;
+      const int valid = min(kBN, offs[c.e + 1] - r0);
+      const int nbox = (valid + G::kBoxH - 1) / G::kBoxH;
+      bool ok = true;
+      for (int kc = 0; kc < KC; kc += G::kCPS) {
+        const int nch = KC - kc >= G::kCPS ? G::kCPS : KC - kc;
+        if (!wait_warp(empty_bar(s), ph ^ 1u, abort_flag, p.status)) { ok = false; break; }
+        const uint32_t st = sbase + (uint32_t)s * G::kStage;
+        const uint32_t fb = full_bar(s);
+        if (wprod) {
+          mbar_arrive_expect_tx(fb, (uint32_t)(nch * (G::kAChunk + G::kMChunk + G::kKbPerChunk * 512)));
+          bulk_g2s(st + G::kOffA, av + (size_t)kc * G::kAChunk, nch * G::kAChunk, fb);
+          if (kSparse) bulk_g2s(st + G::kOffM, am + (size_t)kc * G::kMChunk, nch * G::kMChunk, fb);
+          bulk_g2s(st + G::kOffSFA, as + (size_t)kc * G::kKbPerChunk * 512, nch * G::kKbPerChunk * 512, fb);
+        } else {
+          mbar_arrive_expect_tx(fb, (uint32_t)(nch * nbox * G::kBoxH * 128 + G::kKbps * 512));
+          for (int ch = 0; ch < nch; ++ch)
+            for (int b = 0; b < nbox; ++b)
+              tma_load_2d(st + ch * G::kBChunk + b * G::kBoxH * 128, &tmap_b, (kc + ch) * 128, r0 + b * G::kBoxH, fb);
+          tma_load_3d(st + G::kOffSFB, &tmap_sfb, 0, r0, kc * G::kKbPerChunk, fb);
         }
-        if (!ok) break;
+        ++issued;
+        if (++s == S) { s = 0; ph ^= 1u; }
       }
-      if (*abort_flag) {
-        // drain: wait for the copies this thread issued into the last min(S, issued) stages
-        int s = stage;
-        uint32_t ph = phase;
-        for (int i = 0; i < S && i < issued; ++i) {
-          if (--s < 0) { s = S - 1; ph ^= 1u; }
-          const uint64_t t0 = globaltimer_ns();
-          while (!mbar_try_wait(full_bar(s), ph) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
-          }
+      if (!ok) break;
+    }
+    if (*abort_flag && lane == 0) {
+      // wait (2 s in all) for copies still landing in the stages this warp filled
+      const uint64_t t0 = globaltimer_ns();
+      for (int i = 0; i < S && i < issued; ++i) {
+        if (--s < 0) { s = S - 1; ph ^= 1u; }
+        while (!mbar_try_wait(full_bar(s), ph) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
         }
       }
     }
-  } else if (warp == 1) {
-    // =============================== MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc = make_idesc(kSparse, BN);
-      int stage = 0;
-      uint32_t phase = 0;
-      int acc = 0;
-      uint32_t acc_phase = 0;
-      bool any = false;
-      for (int t = blockIdx.x; t < total_tiles && !*abort_flag; t += gridDim.x) {
-        if (!wait_bounded(acce_bar(acc), acc_phase ^ 1u, abort_flag, p.status)) break;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem + (acc ? kColAcc1 : 0u);
-        bool ok = true;
-        for (int kc = 0; kc < KC; ++kc) {
-          if (!wait_bounded(full_bar(stage), phase, abort_flag, p.status)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t sB = smem_u32(stage0 + (size_t)stage * p.stage_bytes);
-          const uint32_t sA = sB + BN * 128;
-          const uint32_t sM = sA + kABytes;
-          const uint32_t sSFA = sM + kMetaBytes;
-          const uint32_t sSFB = sSFA + kSfBytes;
-          if (kSparse) tc_cp_128x128b(tmem + kColMeta, smem_desc(sM, 128, 128, 0));
-#pragma unroll
-          for (int h = 0; h < kKbPerStage; ++h) {
-            tc_cp_32x128b_x4(tmem + kColSFA + 4 * h, smem_desc(sSFA + 512 * h, 128, 128, 0));
-            tc_cp_32x128b_x4(tmem + kColSFB + 4 * h, smem_desc(sSFB + 512 * h, 128, 128, 0));
-          }
-#pragma unroll
-          for (int h = 0; h < kKbPerStage; ++h) {
-            const uint64_t adesc = smem_desc(sA + 4096u * h, 128, 256, 0);
-            const uint64_t bdesc = smem_desc(sB + kBStep * h, 16, 1024, 2);
-            const uint32_t accum = (kc | h) != 0 ? 1u : 0u;
-            if (kSparse)
-              tc_mma_sparse(d_tmem, adesc, bdesc, idesc, accum, tmem + kColSFA + 4 * h, tmem + kColSFB + 4 * h,
-                            tmem + kColMeta + 2 * h);
-            else
-              tc_mma_dense(d_tmem, adesc, bdesc, idesc, accum, tmem + kColSFA + 4 * h, tmem + kColSFB + 4 * h);
-          }
-          tc_commit(empty_bar(stage));
-          any = true;
-          if (++stage == S) { stage = 0; phase ^= 1u; }
+  } else if (warp >= 7) {
+    // =============================== metadata / scale loaders (TMEM quadrant q = warp % 4)
+    const int q = warp & 3;
+    const int row = 32 * q + lane;
+    const uint32_t tlane = (uint32_t)(32 * q) << 16;
+    int s = 0, set = 0, i = 0;
+    uint32_t ph = 0;
+    TileCursor cur;
+    for (int t = blockIdx.x; t < total_tiles && !*abort_flag; t += gridDim.x) {
+      cur.next(t, pref, offs, kBN);
+      bool ok = true;
+      for (int kc = 0; kc < KC; kc += G::kCPS) {
+        const int nch = KC - kc >= G::kCPS ? G::kCPS : KC - kc;
+        // the TMEM set is free once the MMAs of the stage that last used it have completed
+        if (i >= kNSets) {
+          const int j = i - kNSets;
+          if (!wait_warp(empty_bar(j % S), (uint32_t)(j / S) & 1u, abort_flag, p.status)) { ok = false; break; }
         }
-        if (!ok) break;
-        tc_commit(accf_bar(acc));
-        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        if (!wait_warp(full_bar(s), ph, abort_flag, p.status)) { ok = false; break; }
+        const uint32_t st = sbase + (uint32_t)s * G::kStage;
+        uint32_t r[G::kSetUsed];
+        if (kSparse) {
+#pragma unroll
+          for (int ch = 0; ch < G::kCPS; ++ch)
+            if (ch < nch) lds128(st + G::kOffM + ch * G::kMChunk + row * 16, r[4 * ch], r[4 * ch + 1], r[4 * ch + 2], r[4 * ch + 3]);
+        }
+#pragma unroll
+        for (int kb = 0; kb < G::kKbps; ++kb) {
+          if (kb < nch * G::kKbPerChunk) {
+            lds128(st + G::kOffSFA + kb * 512 + lane * 16, r[G::kColSFA + 4 * kb], r[G::kColSFA + 4 * kb + 1],
+                   r[G::kColSFA + 4 * kb + 2], r[G::kColSFA + 4 * kb + 3]);
+            lds128(st + G::kOffSFB + kb * 512 + lane * 16, r[G::kColSFB + 4 * kb], r[G::kColSFB + 4 * kb + 1],
+                   r[G::kColSFB + 4 * kb + 2], r[G::kColSFB + 4 * kb + 3]);
+          }
+        }
+        tc_st_cols<G::kSetUsed>(tmem + tlane + (uint32_t)set * kSetCols, r);
+        tc_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tfull_bar(set));
+        ++i;
+        if (++set == kNSets) set = 0;
+        if (++s == S) { s = 0; ph ^= 1u; }
       }
-      if (any) {
-        // all MMAs issued by this thread have completed once the drain barrier fires
-        tc_commit(drain_bar);
-        const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(drain_bar, 0) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
+      if (!ok) break;
+    }
+  } else if (warp == 1) {
+    // =============================== MMA issuer (whole warp, one elected lane issues)
+    int s = 0, set = 0, i = 0, it = 0;
+    uint32_t ph = 0;
+    bool any = false;
+    TileCursor cur;
+    for (int t = blockIdx.x; t < total_tiles && !*abort_flag; t += gridDim.x, ++it) {
+      const TileCoord c = cur.next(t, pref, offs, kBN);
+      const int r0 = offs[c.e] + c.mt * kBN;
+      const int valid = min(kBN, offs[c.e + 1] - r0);
+      const uint32_t idesc = make_idesc(kSparse, (valid + 15) & ~15);
+      const int acc = it % NACC;
+      if (!wait_warp(acce_bar(acc), ((uint32_t)(it / NACC) & 1u) ^ 1u, abort_flag, p.status)) break;
+      tc_fence_after();
+      const uint32_t d_tmem = tmem + kColAcc + (uint32_t)(acc * G::kAccStride);
+      bool ok = true;
+      for (int kc = 0; kc < KC; kc += G::kCPS) {
+        const int nch = KC - kc >= G::kCPS ? G::kCPS : KC - kc;
+        if (!wait_warp(full_bar(s), ph, abort_flag, p.status) ||
+            !wait_warp(tfull_bar(set), (uint32_t)(i / kNSets) & 1u, abort_flag, p.status)) {
+          ok = false;
+          break;
         }
+        tc_fence_after();
+        const uint32_t st = sbase + (uint32_t)s * G::kStage;
+        const uint32_t tset = tmem + (uint32_t)set * kSetCols;
+#pragma unroll
+        for (int ch = 0; ch < G::kCPS; ++ch) {
+          if (ch < nch) {
+#pragma unroll
+            for (int h = 0; h < G::kKbPerChunk; ++h) {
+              const int kbi = ch * G::kKbPerChunk + h;
+              const uint64_t adesc = smem_desc(st + G::kOffA + ch * G::kAChunk + 4096u * h, 128, 256, 0);
+              const uint64_t bdesc = smem_desc(st + ch * G::kBChunk + G::kBStep * h, 16, 1024, 2);
+              const uint32_t accum = (kc | ch | h) != 0 ? 1u : 0u;
+              if (kSparse)
+                tc_mma_sparse(d_tmem, adesc, bdesc, idesc, accum, tset + G::kColSFA + 4 * kbi,
+                              tset + G::kColSFB + 4 * kbi, tset + 2 * kbi);
+              else
+                tc_mma_dense(d_tmem, adesc, bdesc, idesc, accum, tset + G::kColSFA + 4 * kbi,
+                             tset + G::kColSFB + 4 * kbi);
+            }
+          }
+        }
+        tc_commit(empty_bar(s));
+        any = true;
+        ++i;
+        if (++set == kNSets) set = 0;
+        if (++s == S) { s = 0; ph ^= 1u; }
+      }
+      if (!ok) break;
+      tc_commit(accf_bar(acc));
+    }
+    __syncwarp();
+    if (any) {
+      // all MMAs issued by this warp have completed once the drain barrier fires
+      tc_commit(drain_bar);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(drain_bar, 0) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
       }
     }
   } else {
-    // =============================== epilogue (warps 2..5 -> TMEM lane quadrants 2,3,0,1)
+    // =============================== epilogue (warps 3..6 -> TMEM lane quadrants 3,0,1,2)
     const int q = warp & 3;
     const int row = 32 * q + lane;
-    int acc = 0;
-    uint32_t acc_phase = 0;
     const float sx = __ldg(p.x_scale);
-    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
-      const TileCoord c = decode_tile(t, pref, offs, E, NT, BN);
-      const int r0 = offs[c.e] + c.mt * BN;
-      const int valid = min(BN, offs[c.e + 1] - r0);
-      if (!wait_bounded(accf_bar(acc), acc_phase, abort_flag, p.status)) break;
+    int it = 0;
+    TileCursor cur;
+    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++it) {
+      const TileCoord c = cur.next(t, pref, offs, kBN);
+      const int r0 = offs[c.e] + c.mt * kBN;
+      const int valid = min(kBN, offs[c.e + 1] - r0);
+      const int acc = it % NACC;
+      if (!wait_warp(accf_bar(acc), (uint32_t)(it / NACC) & 1u, abort_flag, p.status)) break;
       tc_fence_after();
-      const float scale = __fmul_rn(sx, __ldg(p.w_scale + c.e));
+      const float scale = __fmul_rn(sx, wsc[c.e]);
       const int n = c.nt * kTileN + row;
-      const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + (acc ? kColAcc1 : 0u);
-      for (int c0 = 0; c0 < BN; c0 += 16) {
-        if (c0 >= valid) break;
+      const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + kColAcc + (uint32_t)(acc * G::kAccStride);
+      for (int c0 = 0; c0 < valid; c0 += 16) {
         float v[16];
         tc_ld_16(taddr + c0, v);
         if (p.y_f32) {
@@ -421,7 +543,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acce_bar(acc));
-      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
   }
 
@@ -435,10 +556,29 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const GemmParams
 }
 
 // ------------------------------------------------------------------ host side
-int gemm_stage_bytes(bool sparse, int BN) {
-  const int a = sparse ? 8192 : 16384, m = sparse ? 2048 : 0, sf = (sparse ? 2 : 4) * 512;
-  const int b = BN * 128 + a + m + 2 * sf;
-  return (b + 1023) / 1024 * 1024;
+struct GemmPlan {
+  int BN, cps, stage, stages, nacc;
+  size_t smem;
+};
+
+constexpr int kSmemBudget = 200 * 1024;
+
+static GemmPlan make_plan(bool sparse, int BN, int E) {
+  GemmPlan g;
+  g.BN = BN;
+  g.cps = (sparse ? BN <= 64 : BN <= 32) ? 2 : 1;
+  const int kbpc = sparse ? 2 : 4;
+  const int kbps = g.cps * kbpc;
+  const int body = g.cps * BN * 128 + g.cps * (sparse ? 8192 + 2048 : 16384) + 2 * kbps * 512;
+  g.stage = (body + 1023) / 1024 * 1024;
+  g.stages = kSmemBudget / g.stage;
+  if (g.stages > 12) g.stages = 12;
+  const int acc_stride = BN < 32 ? 32 : BN;
+  g.nacc = (int)((kTmemCols - kColAcc) / acc_stride);
+  if (g.nacc > kMaxAcc) g.nacc = kMaxAcc;
+  const int nbars = 2 * g.stages + kNSets + 2 * g.nacc + 1;
+  g.smem = 1024 + (size_t)g.stages * g.stage + nbars * 8 + sizeof(Ctl) + (size_t)(3 * E + 2) * 4;
+  return g;
 }
 
 int gemm_pick_bn(int max_rows) {
@@ -447,19 +587,6 @@ int gemm_pick_bn(int max_rows) {
   if (max_rows <= 32) return 32;
   if (max_rows <= 64) return 64;
   return 128;
-}
-
-constexpr int kSmemBudget = 200 * 1024;
-
-int gemm_stages(bool sparse, int BN) {
-  int s = kSmemBudget / gemm_stage_bytes(sparse, BN);
-  if (s > 16) s = 16;
-  return s;
-}
-
-size_t gemm_smem_bytes(bool sparse, int BN, int E) {
-  const int S = gemm_stages(sparse, BN);
-  return 1024 + (size_t)S * gemm_stage_bytes(sparse, BN) + (2 * S + 5) * 8 + sizeof(Ctl) + (size_t)2 * (E + 1) * 4;
 }
 
 bool gemm_supported(int E) { return E >= 1 && E <= kMaxE; }
@@ -480,16 +607,35 @@ static EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
+template <bool kSparse, int kBN>
+static cudaError_t set_attr_one(int bytes) {
+  return cudaFuncSetAttribute(grouped_gemm_kernel<kSparse, kBN>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
 cudaError_t gemm_set_smem_attrs() {
   int maxb = 0;
   for (int bn = 16; bn <= 128; bn *= 2) {
-    const int a = (int)gemm_smem_bytes(true, bn, kMaxE), b = (int)gemm_smem_bytes(false, bn, kMaxE);
+    const int a = (int)make_plan(true, bn, kMaxE).smem, b = (int)make_plan(false, bn, kMaxE).smem;
     if (a > maxb) maxb = a;
     if (b > maxb) maxb = b;
   }
-  cudaError_t e1 = cudaFuncSetAttribute(grouped_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxb);
-  cudaError_t e2 = cudaFuncSetAttribute(grouped_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, maxb);
-  return e1 != cudaSuccess ? e1 : e2;
+  cudaError_t errs[8] = {set_attr_one<true, 16>(maxb),  set_attr_one<true, 32>(maxb),  set_attr_one<true, 64>(maxb),
+                         set_attr_one<true, 128>(maxb), set_attr_one<false, 16>(maxb), set_attr_one<false, 32>(maxb),
+                         set_attr_one<false, 64>(maxb), set_attr_one<false, 128>(maxb)};
+  for (cudaError_t e : errs)
+    if (e != cudaSuccess) return e;
+  return cudaSuccess;
+}
+
+template <bool kSparse>
+static void launch_bn(int BN, int grid, size_t smem, cudaStream_t stream, const CUtensorMap& tb,
+                      const CUtensorMap& ts, const GemmParams& p) {
+  switch (BN) {
+    case 16: grouped_gemm_kernel<kSparse, 16><<<grid, kGemmThreads, smem, stream>>>(tb, ts, p); break;
+    case 32: grouped_gemm_kernel<kSparse, 32><<<grid, kGemmThreads, smem, stream>>>(tb, ts, p); break;
+    case 64: grouped_gemm_kernel<kSparse, 64><<<grid, kGemmThreads, smem, stream>>>(tb, ts, p); break;
+    default: grouped_gemm_kernel<kSparse, 128><<<grid, kGemmThreads, smem, stream>>>(tb, ts, p); break;
+  }
 }
 
 // returns 0 ok, 1 cuda error, 2 tensor map failure
@@ -499,27 +645,42 @@ int launch_gemm(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, co
                 int num_sms, cudaStream_t stream) {
   EncodeTiledFn enc = get_encode_fn();
   if (enc == nullptr) return 2;
-  const int BN = gemm_pick_bn(max_rows);
-  CUtensorMap tmap;
-  cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)R};
-  cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
-  cuuint32_t box[2] = {128u, (cuuint32_t)BN};
-  cuuint32_t estr[2] = {1u, 1u};
-  CUresult cr = enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a_codes), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (cr != CUDA_SUCCESS) return 2;
+  const GemmPlan g = make_plan(sparse, gemm_pick_bn(max_rows), E);
+  const int box_h = g.BN < 32 ? g.BN : 32;
+  const int kbps = g.cps * (sparse ? 2 : 4);
+  const int rcap = R + kActScalePadRows;
+  const int KBa = K / (sparse ? 128 : 64);
+  CUtensorMap tb, ts;
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)R};
+    cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+    cuuint32_t box[2] = {128u, (cuuint32_t)box_h};
+    cuuint32_t estr[2] = {1u, 1u};
+    if (enc(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a_codes), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return 2;
+  }
+  {
+    // activation scale quad entries as a [KBa][rcap][16 B] tensor; one box = the stage's atoms
+    cuuint64_t dims[3] = {16u, (cuuint64_t)rcap, (cuuint64_t)KBa};
+    cuuint64_t strides[2] = {16u, (cuuint64_t)rcap * 16u};
+    cuuint32_t box[3] = {16u, 32u, (cuuint32_t)kbps};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    if (enc(&ts, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(a_scales), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return 2;
+  }
   GemmParams p;
   p.a_scales = a_scales; p.x_scale = x_scale; p.w_vals = w_vals; p.w_meta = w_meta; p.w_scales = w_scales;
   p.w_scale = w_scale; p.off = off; p.Y = Y; p.status = status;
-  p.E = E; p.N = N; p.K = K; p.R = R; p.BN = BN; p.y_f32 = y_f32; p.rcap = R + kActScalePadRows;
-  p.stages = gemm_stages(sparse, BN);
-  p.stage_bytes = gemm_stage_bytes(sparse, BN);
-  const size_t smem = gemm_smem_bytes(sparse, BN, E);
+  p.E = E; p.N = N; p.K = K; p.R = R; p.y_f32 = y_f32; p.rcap = rcap;
+  p.stages = g.stages; p.nacc = g.nacc;
   if (sparse)
-    grouped_gemm_kernel<true><<<num_sms, kGemmThreads, smem, stream>>>(tmap, p);
+    launch_bn<true>(g.BN, num_sms, g.smem, stream, tb, ts, p);
   else
-    grouped_gemm_kernel<false><<<num_sms, kGemmThreads, smem, stream>>>(tmap, p);
+    launch_bn<false>(g.BN, num_sms, g.smem, stream, tb, ts, p);
   return cudaGetLastError() == cudaSuccess ? 0 : 1;
 }
 

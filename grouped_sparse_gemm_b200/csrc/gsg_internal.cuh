@@ -10,7 +10,7 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
-#include "../../include/gsg.h"
+#include "gsg.h"
 
 #if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
 #error "libgsg is written for sm_100a (Blackwell B200) only"
