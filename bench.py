@@ -138,29 +138,19 @@ class Workload:
         self.cfg, self.dev = cfg, dev
         E, N, K, T, k = cfg.E, cfg.N, cfg.K, cfg.T, cfg.top_k
         u8 = dict(dtype=torch.uint8, device=dev)
-        self.pw = gsg.PackedSparseWeights(values=torch.empty(E * N * K // 4, **u8),
-                                          meta=torch.empty(E * N * K // 16, **u8),
-                                          scales=torch.empty(E * N * K // 32, **u8),
+        L = gsg.lib()
+        self.pw = gsg.PackedSparseWeights(packed=torch.empty(L.gsg_sparse_packed_bytes(E, N, K), **u8),
                                           w_scale=torch.empty(E, dtype=torch.float32, device=dev), E=E, N=N, K=K)
         self.pd = None
         if with_dense:
-            self.pd = gsg.PackedDenseWeights(codes=torch.empty(E * N * K // 2, **u8),
-                                             scales=torch.empty(E * N * K // 16, **u8),
+            self.pd = gsg.PackedDenseWeights(packed=torch.empty(L.gsg_dense_packed_bytes(E, N, K), **u8),
                                              w_scale=torch.empty(E, dtype=torch.float32, device=dev), E=E, N=N, K=K)
         ws_pack = torch.empty(max(gsg.workspace_size(gsg.OP_PACK_SPARSE, 1, N, K), 16), **u8)
         for e in range(E):          # generate and pack one expert at a time (offline step)
             We = inputs.expert_weight(cfg, e, str(dev))[None]
-            vs, ms, ss = N * K // 4, N * K // 16, N * K // 32
-            sub = gsg.PackedSparseWeights(values=self.pw.values[e * vs:(e + 1) * vs], meta=self.pw.meta[e * ms:(e + 1) * ms],
-                                          scales=self.pw.scales[e * ss:(e + 1) * ss], w_scale=self.pw.w_scale[e:e + 1],
-                                          E=1, N=N, K=K)
-            gsg.pack_sparse_nvfp4(We, out=sub, workspace=ws_pack)
+            gsg.pack_sparse_nvfp4(We, out=self.pw.expert(e), workspace=ws_pack)
             if with_dense:
-                cs, ds = N * K // 2, N * K // 16
-                subd = gsg.PackedDenseWeights(codes=self.pd.codes[e * cs:(e + 1) * cs],
-                                              scales=self.pd.scales[e * ds:(e + 1) * ds],
-                                              w_scale=self.pd.w_scale[e:e + 1], E=1, N=N, K=K)
-                gsg.pack_dense_nvfp4(We, out=subd, workspace=ws_pack)
+                gsg.pack_dense_nvfp4(We, out=self.pd.expert(e), workspace=ws_pack)
             del We
         torch.cuda.synchronize()
         self.X_h = inputs.activations(cfg)

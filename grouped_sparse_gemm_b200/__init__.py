@@ -34,8 +34,8 @@ OUT_BF16, OUT_F32 = 0, 1
 ACT_SCALE_PAD_ROWS = 256
 
 EXPORTED_SYMBOLS = [
-    "gsg_sparse_values_bytes", "gsg_sparse_meta_bytes", "gsg_weight_scales_bytes",
-    "gsg_dense_codes_bytes", "gsg_act_codes_bytes", "gsg_act_scales_bytes", "gsg_workspace_size",
+    "gsg_sparse_packed_bytes", "gsg_dense_packed_bytes", "gsg_act_codes_bytes", "gsg_act_scales_bytes",
+    "gsg_workspace_size",
     "gsg_pack_sparse_nvfp4", "gsg_pack_dense_nvfp4", "gsg_moe_route_permute",
     "gsg_quantize_act_nvfp4", "gsg_grouped_sparse_gemm", "gsg_grouped_dense_gemm",
     "gsg_unpermute_scale", "gsg_get_device_status", "gsg_status_string", "gsg_version",
@@ -71,19 +71,17 @@ def load_library(build_if_missing: bool = False) -> ctypes.CDLL:
     L = ctypes.CDLL(path)
     vp, i, sz, fp = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
     sig = {
-        "gsg_sparse_values_bytes": (sz, [i, i, i]),
-        "gsg_sparse_meta_bytes": (sz, [i, i, i]),
-        "gsg_weight_scales_bytes": (sz, [i, i, i, i]),
-        "gsg_dense_codes_bytes": (sz, [i, i, i]),
+        "gsg_sparse_packed_bytes": (sz, [i, i, i]),
+        "gsg_dense_packed_bytes": (sz, [i, i, i]),
         "gsg_act_codes_bytes": (sz, [i, i]),
         "gsg_act_scales_bytes": (sz, [i, i, i]),
         "gsg_workspace_size": (sz, [i, i, i, i, i, i]),
-        "gsg_pack_sparse_nvfp4": (i, [vp, i, i, i, vp, vp, vp, fp, vp, sz, vp]),
-        "gsg_pack_dense_nvfp4": (i, [vp, i, i, i, vp, vp, fp, vp, sz, vp]),
+        "gsg_pack_sparse_nvfp4": (i, [vp, i, i, i, vp, fp, vp, sz, vp]),
+        "gsg_pack_dense_nvfp4": (i, [vp, i, i, i, vp, fp, vp, sz, vp]),
         "gsg_moe_route_permute": (i, [vp, i, i, i, vp, vp, vp, vp, sz, vp]),
         "gsg_quantize_act_nvfp4": (i, [vp, i, i, i, vp, i, vp, vp, vp, vp, vp, sz, vp]),
-        "gsg_grouped_sparse_gemm": (i, [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, i, vp]),
-        "gsg_grouped_dense_gemm": (i, [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, i, vp]),
+        "gsg_grouped_sparse_gemm": (i, [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, i, vp]),
+        "gsg_grouped_dense_gemm": (i, [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, i, vp]),
         "gsg_unpermute_scale": (i, [vp, vp, vp, i, i, i, vp, vp]),
         "gsg_get_device_status": (i, [vp]),
         "gsg_status_string": (ctypes.c_char_p, [i]),
@@ -139,31 +137,41 @@ def _workspace(nbytes: int, device) -> torch.Tensor:
 
 
 # ------------------------------------------------------------------ packed containers
+SPARSE_CHUNK_BYTES = 11264     # one (expert, n-tile, 256-wide K chunk) block: values | metadata | scales
+DENSE_CHUNK_BYTES = 18432
+
+
 @dataclass
 class PackedSparseWeights:
-    values: torch.Tensor   # uint8 [E*N*K/4]
-    meta: torch.Tensor     # uint8 [E*N*K/16]
-    scales: torch.Tensor   # uint8 [E*N*K/32]
+    packed: torch.Tensor   # uint8 [E*N*K*11/32], chunk blocks (see include/gsg.h)
     w_scale: torch.Tensor  # fp32 [E]
     E: int
     N: int
     K: int
 
     def nbytes(self) -> int:
-        return self.values.numel() + self.meta.numel() + self.scales.numel()
+        return self.packed.numel()
+
+    def expert(self, e: int) -> "PackedSparseWeights":
+        """View of expert e alone (E = 1)."""
+        n = self.packed.numel() // self.E
+        return PackedSparseWeights(self.packed[e * n:(e + 1) * n], self.w_scale[e:e + 1], 1, self.N, self.K)
 
 
 @dataclass
 class PackedDenseWeights:
-    codes: torch.Tensor    # uint8 [E*N*K/2]
-    scales: torch.Tensor   # uint8 [E*N*K/16]
+    packed: torch.Tensor   # uint8 [E*N*K*9/16]
     w_scale: torch.Tensor  # fp32 [E]
     E: int
     N: int
     K: int
 
     def nbytes(self) -> int:
-        return self.codes.numel() + self.scales.numel()
+        return self.packed.numel()
+
+    def expert(self, e: int) -> "PackedDenseWeights":
+        n = self.packed.numel() // self.E
+        return PackedDenseWeights(self.packed[e * n:(e + 1) * n], self.w_scale[e:e + 1], 1, self.N, self.K)
 
 
 @dataclass
@@ -197,15 +205,12 @@ def pack_sparse_nvfp4(W: torch.Tensor, out: Optional[PackedSparseWeights] = None
     dev = W.device
     if out is None:
         out = PackedSparseWeights(
-            values=torch.empty(L.gsg_sparse_values_bytes(E, N, K), dtype=torch.uint8, device=dev),
-            meta=torch.empty(L.gsg_sparse_meta_bytes(E, N, K), dtype=torch.uint8, device=dev),
-            scales=torch.empty(L.gsg_weight_scales_bytes(E, N, K, 32), dtype=torch.uint8, device=dev),
+            packed=torch.empty(L.gsg_sparse_packed_bytes(E, N, K), dtype=torch.uint8, device=dev),
             w_scale=torch.empty(E, dtype=torch.float32, device=dev), E=E, N=N, K=K)
     need = workspace_size(OP_PACK_SPARSE, E, N, K)
     ws = workspace if workspace is not None else _workspace(need, dev)
     _check("gsg_pack_sparse_nvfp4", L.gsg_pack_sparse_nvfp4(
-        _ptr(W), E, N, K, _ptr(out.values), _ptr(out.meta), _ptr(out.scales), _ptr(out.w_scale),
-        _ptr(ws), ws.numel(), _stream(stream)))
+        _ptr(W), E, N, K, _ptr(out.packed), _ptr(out.w_scale), _ptr(ws), ws.numel(), _stream(stream)))
     return out
 
 
@@ -219,14 +224,12 @@ def pack_dense_nvfp4(W: torch.Tensor, out: Optional[PackedDenseWeights] = None,
     dev = W.device
     if out is None:
         out = PackedDenseWeights(
-            codes=torch.empty(L.gsg_dense_codes_bytes(E, N, K), dtype=torch.uint8, device=dev),
-            scales=torch.empty(L.gsg_weight_scales_bytes(E, N, K, 16), dtype=torch.uint8, device=dev),
+            packed=torch.empty(L.gsg_dense_packed_bytes(E, N, K), dtype=torch.uint8, device=dev),
             w_scale=torch.empty(E, dtype=torch.float32, device=dev), E=E, N=N, K=K)
     need = workspace_size(OP_PACK_DENSE, E, N, K)
     ws = workspace if workspace is not None else _workspace(need, dev)
     _check("gsg_pack_dense_nvfp4", L.gsg_pack_dense_nvfp4(
-        _ptr(W), E, N, K, _ptr(out.codes), _ptr(out.scales), _ptr(out.w_scale),
-        _ptr(ws), ws.numel(), _stream(stream)))
+        _ptr(W), E, N, K, _ptr(out.packed), _ptr(out.w_scale), _ptr(ws), ws.numel(), _stream(stream)))
     return out
 
 
@@ -282,9 +285,8 @@ def grouped_sparse_gemm(act: QuantizedActivations, w: PackedSparseWeights, offse
         out = torch.empty(max(act.R, 1), w.N, dtype=out_dtype, device=act.codes.device)
     ydt = OUT_F32 if out.dtype == torch.float32 else OUT_BF16
     _check("gsg_grouped_sparse_gemm", lib().gsg_grouped_sparse_gemm(
-        _ptr(act.codes), _ptr(act.scales), _ptr(act.x_scale), _ptr(w.values), _ptr(w.meta),
-        _ptr(w.scales), _ptr(w.w_scale), _ptr(offsets), w.E, w.N, w.K, act.R, max_rows_per_expert,
-        _ptr(out), ydt, _stream(stream)))
+        _ptr(act.codes), _ptr(act.scales), _ptr(act.x_scale), _ptr(w.packed), _ptr(w.w_scale),
+        _ptr(offsets), w.E, w.N, w.K, act.R, max_rows_per_expert, _ptr(out), ydt, _stream(stream)))
     return out
 
 
@@ -298,9 +300,8 @@ def grouped_dense_gemm(act: QuantizedActivations, w: PackedDenseWeights, offsets
         out = torch.empty(max(act.R, 1), w.N, dtype=out_dtype, device=act.codes.device)
     ydt = OUT_F32 if out.dtype == torch.float32 else OUT_BF16
     _check("gsg_grouped_dense_gemm", lib().gsg_grouped_dense_gemm(
-        _ptr(act.codes), _ptr(act.scales), _ptr(act.x_scale), _ptr(w.codes), _ptr(w.scales),
-        _ptr(w.w_scale), _ptr(offsets), w.E, w.N, w.K, act.R, max_rows_per_expert,
-        _ptr(out), ydt, _stream(stream)))
+        _ptr(act.codes), _ptr(act.scales), _ptr(act.x_scale), _ptr(w.packed), _ptr(w.w_scale),
+        _ptr(offsets), w.E, w.N, w.K, act.R, max_rows_per_expert, _ptr(out), ydt, _stream(stream)))
     return out
 
 

@@ -57,12 +57,12 @@ bool weight_shape_ok(int E, int N, int K) {
 
 extern "C" {
 
-size_t gsg_sparse_values_bytes(int E, int N, int K) { return (size_t)E * N * K / 4; }
-size_t gsg_sparse_meta_bytes(int E, int N, int K) { return (size_t)E * N * K / 16; }
-size_t gsg_weight_scales_bytes(int E, int N, int K, int sf_block) {
-  return sf_block > 0 ? (size_t)E * N * K / sf_block : 0;
+size_t gsg_sparse_packed_bytes(int E, int N, int K) {
+  return (size_t)E * (N / gsg::kTileN) * (K / gsg::kChunkK) * gsg::kSparseChunkBytes;
 }
-size_t gsg_dense_codes_bytes(int E, int N, int K) { return (size_t)E * N * K / 2; }
+size_t gsg_dense_packed_bytes(int E, int N, int K) {
+  return (size_t)E * (N / gsg::kTileN) * (K / gsg::kChunkK) * gsg::kDenseChunkBytes;
+}
 size_t gsg_act_codes_bytes(int R, int K) { return (size_t)R * K / 2; }
 size_t gsg_act_scales_bytes(int R, int K, int sf_block) {
   if (sf_block <= 0) return 0;
@@ -86,30 +86,29 @@ size_t gsg_workspace_size(int op, int E, int N, int K, int T, int k) {
   }
 }
 
-static gsg_status_t pack_common(bool sparse, const float* W, int E, int N, int K, uint8_t* values, uint8_t* meta,
-                                uint8_t* scales, float* w_tensor_scale, void* ws, size_t ws_bytes, void* stream) {
-  if (!W || !values || !scales || !w_tensor_scale || (sparse && !meta)) return GSG_ERR_INVALID_ARG;
+static gsg_status_t pack_common(bool sparse, const float* W, int E, int N, int K, uint8_t* packed,
+                                float* w_tensor_scale, void* ws, size_t ws_bytes, void* stream) {
+  if (!W || !packed || !w_tensor_scale) return GSG_ERR_INVALID_ARG;
   if (!weight_shape_ok(E, N, K)) return GSG_ERR_UNSUPPORTED_SHAPE;
   if (E > 65535) return GSG_ERR_UNSUPPORTED_SHAPE;
-  if (!aligned16(W) || !aligned16(values) || (sparse && !aligned16(meta))) return GSG_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(packed)) return GSG_ERR_INVALID_ARG;
   const size_t need = gsg_workspace_size(sparse ? GSG_OP_PACK_SPARSE : GSG_OP_PACK_DENSE, E, N, K, 0, 1);
   if (ws == nullptr || ws_bytes < need) return GSG_ERR_WORKSPACE;
   DeviceState* d = nullptr;
   gsg_status_t st = device_state(&d);
   if (st != GSG_OK) return st;
-  return from_cuda(gsg::launch_pack(sparse, W, E, N, K, values, meta, scales, w_tensor_scale,
-                                    static_cast<float*>(ws), d->status, as_stream(stream)));
+  return from_cuda(gsg::launch_pack(sparse, W, E, N, K, packed, w_tensor_scale, static_cast<float*>(ws), d->status,
+                                    as_stream(stream)));
 }
 
-gsg_status_t gsg_pack_sparse_nvfp4(const float* W, int E, int N, int K, uint8_t* values, uint8_t* meta,
-                                   uint8_t* scales, float* w_tensor_scale, void* workspace, size_t workspace_bytes,
-                                   void* stream) {
-  return pack_common(true, W, E, N, K, values, meta, scales, w_tensor_scale, workspace, workspace_bytes, stream);
+gsg_status_t gsg_pack_sparse_nvfp4(const float* W, int E, int N, int K, uint8_t* w_packed, float* w_tensor_scale,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+  return pack_common(true, W, E, N, K, w_packed, w_tensor_scale, workspace, workspace_bytes, stream);
 }
 
-gsg_status_t gsg_pack_dense_nvfp4(const float* W, int E, int N, int K, uint8_t* codes, uint8_t* scales,
-                                  float* w_tensor_scale, void* workspace, size_t workspace_bytes, void* stream) {
-  return pack_common(false, W, E, N, K, codes, nullptr, scales, w_tensor_scale, workspace, workspace_bytes, stream);
+gsg_status_t gsg_pack_dense_nvfp4(const float* W, int E, int N, int K, uint8_t* w_packed, float* w_tensor_scale,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+  return pack_common(false, W, E, N, K, w_packed, w_tensor_scale, workspace, workspace_bytes, stream);
 }
 
 gsg_status_t gsg_moe_route_permute(const int32_t* topk_ids, int T, int k, int E, int32_t* expert_offsets,
@@ -153,41 +152,37 @@ gsg_status_t gsg_quantize_act_nvfp4(const uint16_t* X, int T, int K, int sf_bloc
 }
 
 static gsg_status_t gemm_common(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, const float* x_scale,
-                                const uint8_t* w_vals, const uint8_t* w_meta, const uint8_t* w_scales,
-                                const float* w_scale, const int32_t* off, int E, int N, int K, int R, int max_rows,
-                                void* Y, int y_dtype, void* stream) {
+                                const uint8_t* w_packed, const float* w_scale, const int32_t* off, int E, int N,
+                                int K, int R, int max_rows, void* Y, int y_dtype, void* stream) {
   if (R < 0 || (y_dtype != GSG_OUT_BF16 && y_dtype != GSG_OUT_F32)) return GSG_ERR_INVALID_ARG;
   if (!weight_shape_ok(E, N, K) || !gsg::gemm_supported(E)) return GSG_ERR_UNSUPPORTED_SHAPE;
   if ((long long)R > (1ll << 30)) return GSG_ERR_UNSUPPORTED_SHAPE;
-  if (!off || !w_vals || !w_scales || !w_scale || !x_scale || (sparse && !w_meta)) return GSG_ERR_INVALID_ARG;
+  if (!off || !w_packed || !w_scale || !x_scale) return GSG_ERR_INVALID_ARG;
   if (R == 0) return GSG_OK;  // nothing routed: nothing to compute or write
   if (!a_codes || !a_scales || !Y) return GSG_ERR_INVALID_ARG;
-  if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(w_vals) || !aligned16(w_scales) ||
-      (sparse && !aligned16(w_meta)))
-    return GSG_ERR_INVALID_ARG;
+  if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(w_packed)) return GSG_ERR_INVALID_ARG;
   DeviceState* d = nullptr;
   gsg_status_t st = device_state(&d);
   if (st != GSG_OK) return st;
-  const int rc = gsg::launch_gemm(sparse, a_codes, a_scales, x_scale, w_vals, w_meta, w_scales, w_scale, off, E, N,
-                                  K, R, max_rows, Y, y_dtype == GSG_OUT_F32 ? 1 : 0, d->status, d->num_sms,
-                                  as_stream(stream));
+  const int rc = gsg::launch_gemm(sparse, a_codes, a_scales, x_scale, w_packed, w_scale, off, E, N, K, R, max_rows,
+                                  Y, y_dtype == GSG_OUT_F32 ? 1 : 0, d->status, d->num_sms, as_stream(stream));
   return rc == 0 ? GSG_OK : GSG_ERR_CUDA;
 }
 
 gsg_status_t gsg_grouped_sparse_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* x_tensor_scale,
-                                     const uint8_t* w_values, const uint8_t* w_meta, const uint8_t* w_scales,
-                                     const float* w_tensor_scale, const int32_t* expert_offsets, int E, int N, int K,
-                                     int R, int max_rows_per_expert, void* Y, int y_dtype, void* stream) {
-  return gemm_common(true, a_codes, a_scales, x_tensor_scale, w_values, w_meta, w_scales, w_tensor_scale,
-                     expert_offsets, E, N, K, R, max_rows_per_expert, Y, y_dtype, stream);
+                                     const uint8_t* w_packed, const float* w_tensor_scale,
+                                     const int32_t* expert_offsets, int E, int N, int K, int R,
+                                     int max_rows_per_expert, void* Y, int y_dtype, void* stream) {
+  return gemm_common(true, a_codes, a_scales, x_tensor_scale, w_packed, w_tensor_scale, expert_offsets, E, N, K, R,
+                     max_rows_per_expert, Y, y_dtype, stream);
 }
 
 gsg_status_t gsg_grouped_dense_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* x_tensor_scale,
-                                    const uint8_t* w_codes, const uint8_t* w_scales, const float* w_tensor_scale,
+                                    const uint8_t* w_packed, const float* w_tensor_scale,
                                     const int32_t* expert_offsets, int E, int N, int K, int R,
                                     int max_rows_per_expert, void* Y, int y_dtype, void* stream) {
-  return gemm_common(false, a_codes, a_scales, x_tensor_scale, w_codes, nullptr, w_scales, w_tensor_scale,
-                     expert_offsets, E, N, K, R, max_rows_per_expert, Y, y_dtype, stream);
+  return gemm_common(false, a_codes, a_scales, x_tensor_scale, w_packed, w_tensor_scale, expert_offsets, E, N, K, R,
+                     max_rows_per_expert, Y, y_dtype, stream);
 }
 
 gsg_status_t gsg_unpermute_scale(const uint16_t* Y, const int32_t* inv_perm, const float* gates, int T, int k, int N,

@@ -8,7 +8,7 @@
 //
 // One CTA per SM, 352 threads (11 warps), warp-specialised around one shared-memory ring whose
 // stages hold 256 or 512 logical K of one tile (weights, activation codes and both scales):
-//   warp 0      weight producer: three bulk copies per stage (pre-tiled values, metadata, scales).
+//   warp 0      weight producer: one bulk copy per stage of the interleaved packed weight blocks.
 //   warp 2      activation producer: tensor-map TMA boxes (128B swizzle) of only the token rows the
 //               tile holds, and one 3-D TMA box of the activation scale atoms.
 //   warps 7..10 scale/metadata loaders, one per TMEM lane quadrant: read the stage's metadata and
@@ -19,7 +19,8 @@
 //   warps 3..6  epilogue: tcgen05.ld accumulator lanes, multiply by s_x * s_w[e], store rows of Y.
 // Every TMA and tcgen05 instruction is issued by an elected lane of a converged warp.
 // Tiles are (expert e, 128 weight rows nt, token tile mt) in e -> nt -> mt order; CTAs take
-// tiles round-robin.  Experts with no rows produce no tiles.  Every mbarrier wait is bounded:
+// tiles round-robin and decode their own tile list into shared memory once, at set-up.
+// Experts with no rows produce no tiles.  Every mbarrier wait is bounded:
 // on expiry the kernel records GSG_ERR_DEVICE_TIMEOUT, drains its own copies and MMAs, frees
 // TMEM and returns.
 #include <cuda.h>
@@ -40,15 +41,13 @@ constexpr uint32_t kColAcc = kNSets * kSetCols;       // first accumulator (192)
 struct GemmParams {
   const uint8_t* a_scales;
   const float* x_scale;
-  const uint8_t* w_vals;
-  const uint8_t* w_meta;
-  const uint8_t* w_scales;
+  const uint8_t* w_packed;
   const float* w_scale;
   const int32_t* off;
   void* Y;
   int* status;
   int E, N, K, R, y_f32, rcap;
-  int stages, nacc;
+  int stages, nacc, tcap;
 };
 
 // ------------------------------------------------------------------ PTX wrappers
@@ -217,25 +216,38 @@ __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatil
   return __all_sync(0xffffffffu, ok);
 }
 
-struct TileCoord {
-  int e, nt, mt;
+// One tile of this CTA: expert, n-tile, first routed row and number of rows.
+struct TileDesc {
+  int e, nt, r0, valid;
 };
 
-// Tiles are visited in increasing order, so the owning expert only moves forward: a linear
-// scan from the previous expert replaces a search.  pref[E] = total tiles > t ends the scan.
-struct TileCursor {
-  int e = 0;
-  __device__ __forceinline__ TileCoord next(int t, const int* pref, const int* offs, int BN) {
-    while (pref[e + 1] <= t) ++e;
-    TileCoord c;
-    c.e = e;
-    const int local = t - pref[e];
-    const int mte = (offs[e + 1] - offs[e] + BN - 1) / BN;
-    c.nt = local / mte;
-    c.mt = local % mte;
-    return c;
+// Largest e with pref[e] <= t (pref[0] = 0, pref[E] = total tiles), then the tile's rows.
+__device__ __forceinline__ TileDesc decode_tile(int t, const int* pref, const int* offs, int E, int BN) {
+  int lo = 0, hi = E;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (pref[mid] <= t) lo = mid; else hi = mid;
   }
-};
+  const int local = t - pref[lo];
+  const int mte = (offs[lo + 1] - offs[lo] + BN - 1) / BN;
+  TileDesc d;
+  d.e = lo;
+  d.nt = local / mte;
+  d.r0 = offs[lo] + (local % mte) * BN;
+  d.valid = min(BN, offs[lo + 1] - d.r0);
+  return d;
+}
+
+// The j-th tile of this CTA (tile index blockIdx.x + j * gridDim.x): from the shared-memory
+// table filled at set-up, or decoded on the spot past its capacity.
+__device__ __forceinline__ TileDesc my_tile(int j, const int4* table, int tcap, const int* pref, const int* offs,
+                                            int E, int BN) {
+  if (j < tcap) {
+    const int4 v = table[j];
+    return TileDesc{v.x, v.y, v.z, v.w};
+  }
+  return decode_tile(blockIdx.x + j * (int)gridDim.x, pref, offs, E, BN);
+}
 
 // Compile-time stage geometry of one (sparse/dense, token tile) instantiation.
 template <bool kSparse, int kBN>
@@ -244,13 +256,12 @@ struct Geo {
   static constexpr int kKbPerChunk = kChunkK / kKbLogical;         // 2 sparse, 4 dense
   static constexpr int kCPS = (kSparse ? kBN <= 64 : kBN <= 32) ? 2 : 1;   // 256-wide chunks per stage
   static constexpr int kKbps = kCPS * kKbPerChunk;                 // MMAs per stage
-  static constexpr int kAChunk = kSparse ? 8192 : 16384;           // weight values per chunk
-  static constexpr int kMChunk = kSparse ? 2048 : 0;               // metadata per chunk
+  static constexpr int kCB = kSparse ? kSparseChunkBytes : kDenseChunkBytes;   // packed chunk block
+  static constexpr int kCBMeta = 8192;                             // metadata offset in a chunk block
+  static constexpr int kCBScale = kSparse ? 10240 : 16384;         // scale atoms offset in a chunk block
   static constexpr int kBChunk = kBN * 128;                        // activation codes per chunk
-  static constexpr int kOffA = kCPS * kBChunk;                     // stage layout: B | A | M | SFA | SFB
-  static constexpr int kOffM = kOffA + kCPS * kAChunk;
-  static constexpr int kOffSFA = kOffM + kCPS * kMChunk;
-  static constexpr int kOffSFB = kOffSFA + kKbps * 512;
+  static constexpr int kOffW = kCPS * kBChunk;                     // stage layout: B chunks | W blocks | SFB
+  static constexpr int kOffSFB = kOffW + kCPS * kCB;
   static constexpr int kStage = (kOffSFB + kKbps * 512 + 1023) / 1024 * 1024;
   static constexpr int kMetaCols = kSparse ? 4 * kCPS : 0;         // TMEM set: meta | SFA | SFB
   static constexpr int kColSFA = kMetaCols;
@@ -269,7 +280,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
   using G = Geo<kSparse, kBN>;
   extern __shared__ uint8_t smem_raw[];
   const int E = p.E, NT = p.N / kTileN, KC = p.K / kChunkK;
-  const int KBt = p.K / G::kKbLogical;
   const int S = p.stages, NACC = p.nacc;
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + (size_t)S * G::kStage);
@@ -279,6 +289,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
   int* offs = reinterpret_cast<int*>(ctl + 1);   // [E+1]
   int* pref = offs + (E + 1);                    // [E+1]
   float* wsc = reinterpret_cast<float*>(pref + (E + 1));   // [E]
+  int4* ttab = reinterpret_cast<int4*>((reinterpret_cast<uintptr_t>(wsc + E) + 15) & ~uintptr_t(15));   // [tcap]
   volatile int* abort_flag = &ctl->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -348,10 +359,17 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
     if (threadIdx.x == kGemmThreads - 1) pref[E] = before + incl;
   }
   if (bad) set_status(p.status, GSG_ERR_BAD_ROUTING);
+  __syncthreads();
+  const int total_tiles = pref[E];
+  // this CTA's tiles, decoded once
+  const int n_my = (int)blockIdx.x < total_tiles ? (total_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+  for (int j = threadIdx.x; j < n_my && j < p.tcap; j += blockDim.x) {
+    const TileDesc d = decode_tile((int)blockIdx.x + j * (int)gridDim.x, pref, offs, E, kBN);
+    ttab[j] = make_int4(d.e, d.nt, d.r0, d.valid);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const int total_tiles = pref[E];
   const uint32_t tmem = ctl->tmem_base;
 
   if (warp == 0 || warp == 2) {
@@ -359,16 +377,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
     const bool wprod = warp == 0;
     int s = 0, issued = 0;
     uint32_t ph = 0;
-    TileCursor cur;
-    for (int t = blockIdx.x; t < total_tiles && !*abort_flag; t += gridDim.x) {
-      const TileCoord c = cur.next(t, pref, offs, kBN);
-      const size_t tile = (size_t)c.e * NT + c.nt;
-      const uint8_t* av = p.w_vals + tile * KBt * 4096;
-      const uint8_t* am = kSparse ? p.w_meta + tile * KC * 2048 : nullptr;
-      const uint8_t* as = p.w_scales + tile * KBt * 512;
-      const int r0 = offs[c.e] + c.mt * kBN;
-      const int valid = min(kBN, offs[c.e + 1] - r0);
-      const int nbox = (valid + G::kBoxH - 1) / G::kBoxH;
+    for (int j = 0; j < n_my && !*abort_flag; ++j) {
+      const TileDesc c = my_tile(j, ttab, p.tcap, pref, offs, E, kBN);
+      const uint8_t* wsrc = p.w_packed + ((size_t)c.e * NT + c.nt) * KC * G::kCB;
+      const int r0 = c.r0;
+      const int nbox = (c.valid + G::kBoxH - 1) / G::kBoxH;
       bool ok = true;
       for (int kc = 0; kc < KC; kc += G::kCPS) {
         const int nch = KC - kc >= G::kCPS ? G::kCPS : KC - kc;
@@ -376,10 +389,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
         const uint32_t st = sbase + (uint32_t)s * G::kStage;
         const uint32_t fb = full_bar(s);
         if (wprod) {
-          mbar_arrive_expect_tx(fb, (uint32_t)(nch * (G::kAChunk + G::kMChunk + G::kKbPerChunk * 512)));
-          bulk_g2s(st + G::kOffA, av + (size_t)kc * G::kAChunk, nch * G::kAChunk, fb);
-          if (kSparse) bulk_g2s(st + G::kOffM, am + (size_t)kc * G::kMChunk, nch * G::kMChunk, fb);
-          bulk_g2s(st + G::kOffSFA, as + (size_t)kc * G::kKbPerChunk * 512, nch * G::kKbPerChunk * 512, fb);
+          mbar_arrive_expect_tx(fb, (uint32_t)(nch * G::kCB));
+          bulk_g2s(st + G::kOffW, wsrc + (size_t)kc * G::kCB, nch * G::kCB, fb);
         } else {
           mbar_arrive_expect_tx(fb, (uint32_t)(nch * nbox * G::kBoxH * 128 + G::kKbps * 512));
           for (int ch = 0; ch < nch; ++ch)
@@ -408,9 +419,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
     const uint32_t tlane = (uint32_t)(32 * q) << 16;
     int s = 0, set = 0, i = 0;
     uint32_t ph = 0;
-    TileCursor cur;
-    for (int t = blockIdx.x; t < total_tiles && !*abort_flag; t += gridDim.x) {
-      cur.next(t, pref, offs, kBN);
+    for (int j = 0; j < n_my && !*abort_flag; ++j) {
       bool ok = true;
       for (int kc = 0; kc < KC; kc += G::kCPS) {
         const int nch = KC - kc >= G::kCPS ? G::kCPS : KC - kc;
@@ -425,12 +434,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
         if (kSparse) {
 #pragma unroll
           for (int ch = 0; ch < G::kCPS; ++ch)
-            if (ch < nch) lds128(st + G::kOffM + ch * G::kMChunk + row * 16, r[4 * ch], r[4 * ch + 1], r[4 * ch + 2], r[4 * ch + 3]);
+            if (ch < nch)
+              lds128(st + G::kOffW + ch * G::kCB + G::kCBMeta + row * 16, r[4 * ch], r[4 * ch + 1], r[4 * ch + 2],
+                     r[4 * ch + 3]);
         }
 #pragma unroll
         for (int kb = 0; kb < G::kKbps; ++kb) {
           if (kb < nch * G::kKbPerChunk) {
-            lds128(st + G::kOffSFA + kb * 512 + lane * 16, r[G::kColSFA + 4 * kb], r[G::kColSFA + 4 * kb + 1],
+            const uint32_t sfa = st + G::kOffW + (kb / G::kKbPerChunk) * G::kCB + G::kCBScale + (kb % G::kKbPerChunk) * 512;
+            lds128(sfa + lane * 16, r[G::kColSFA + 4 * kb], r[G::kColSFA + 4 * kb + 1],
                    r[G::kColSFA + 4 * kb + 2], r[G::kColSFA + 4 * kb + 3]);
             lds128(st + G::kOffSFB + kb * 512 + lane * 16, r[G::kColSFB + 4 * kb], r[G::kColSFB + 4 * kb + 1],
                    r[G::kColSFB + 4 * kb + 2], r[G::kColSFB + 4 * kb + 3]);
@@ -452,12 +464,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
     int s = 0, set = 0, i = 0, it = 0;
     uint32_t ph = 0;
     bool any = false;
-    TileCursor cur;
-    for (int t = blockIdx.x; t < total_tiles && !*abort_flag; t += gridDim.x, ++it) {
-      const TileCoord c = cur.next(t, pref, offs, kBN);
-      const int r0 = offs[c.e] + c.mt * kBN;
-      const int valid = min(kBN, offs[c.e + 1] - r0);
-      const uint32_t idesc = make_idesc(kSparse, (valid + 15) & ~15);
+    for (int j = 0; j < n_my && !*abort_flag; ++j, ++it) {
+      const TileDesc c = my_tile(j, ttab, p.tcap, pref, offs, E, kBN);
+      const uint32_t idesc = make_idesc(kSparse, (c.valid + 15) & ~15);
       const int acc = it % NACC;
       if (!wait_warp(acce_bar(acc), ((uint32_t)(it / NACC) & 1u) ^ 1u, abort_flag, p.status)) break;
       tc_fence_after();
@@ -479,7 +488,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
 #pragma unroll
             for (int h = 0; h < G::kKbPerChunk; ++h) {
               const int kbi = ch * G::kKbPerChunk + h;
-              const uint64_t adesc = smem_desc(st + G::kOffA + ch * G::kAChunk + 4096u * h, 128, 256, 0);
+              const uint64_t adesc = smem_desc(st + G::kOffW + ch * G::kCB + 4096u * h, 128, 256, 0);
               const uint64_t bdesc = smem_desc(st + ch * G::kBChunk + G::kBStep * h, 16, 1024, 2);
               const uint32_t accum = (kc | ch | h) != 0 ? 1u : 0u;
               if (kSparse)
@@ -514,11 +523,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
     const int row = 32 * q + lane;
     const float sx = __ldg(p.x_scale);
     int it = 0;
-    TileCursor cur;
-    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++it) {
-      const TileCoord c = cur.next(t, pref, offs, kBN);
-      const int r0 = offs[c.e] + c.mt * kBN;
-      const int valid = min(kBN, offs[c.e + 1] - r0);
+    for (int j = 0; j < n_my; ++j, ++it) {
+      const TileDesc c = my_tile(j, ttab, p.tcap, pref, offs, E, kBN);
+      const int r0 = c.r0, valid = c.valid;
       const int acc = it % NACC;
       if (!wait_warp(accf_bar(acc), (uint32_t)(it / NACC) & 1u, abort_flag, p.status)) break;
       tc_fence_after();
@@ -557,29 +564,34 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
 
 // ------------------------------------------------------------------ host side
 struct GemmPlan {
-  int BN, cps, stage, stages, nacc;
+  int BN, cps, stage, stages, nacc, tcap;
   size_t smem;
 };
 
 constexpr int kSmemBudget = 200 * 1024;
 
-static GemmPlan make_plan(bool sparse, int BN, int E) {
+// tcap: capacity of the per-CTA tile table (tiles beyond it are decoded on the fly); an upper
+// bound on a CTA's tiles is ceil((ceil(R/BN) + E) * NT / grid).
+static GemmPlan make_plan(bool sparse, int BN, int E, int tcap) {
   GemmPlan g;
   g.BN = BN;
+  g.tcap = tcap;
   g.cps = (sparse ? BN <= 64 : BN <= 32) ? 2 : 1;
-  const int kbpc = sparse ? 2 : 4;
-  const int kbps = g.cps * kbpc;
-  const int body = g.cps * BN * 128 + g.cps * (sparse ? 8192 + 2048 : 16384) + 2 * kbps * 512;
+  const int kbps = g.cps * (sparse ? 2 : 4);
+  const int body = g.cps * BN * 128 + g.cps * (sparse ? kSparseChunkBytes : kDenseChunkBytes) + kbps * 512;
   g.stage = (body + 1023) / 1024 * 1024;
-  g.stages = kSmemBudget / g.stage;
+  g.stages = (kSmemBudget - tcap * 16) / g.stage;
   if (g.stages > 12) g.stages = 12;
   const int acc_stride = BN < 32 ? 32 : BN;
   g.nacc = (int)((kTmemCols - kColAcc) / acc_stride);
   if (g.nacc > kMaxAcc) g.nacc = kMaxAcc;
   const int nbars = 2 * g.stages + kNSets + 2 * g.nacc + 1;
-  g.smem = 1024 + (size_t)g.stages * g.stage + nbars * 8 + sizeof(Ctl) + (size_t)(3 * E + 2) * 4;
+  g.smem = 1024 + (size_t)g.stages * g.stage + nbars * 8 + sizeof(Ctl) + (size_t)(3 * E + 2) * 4 + 16 +
+           (size_t)tcap * 16;
   return g;
 }
+
+constexpr int kMaxTableTiles = 1024;
 
 int gemm_pick_bn(int max_rows) {
   if (max_rows <= 0) return 128;
@@ -613,17 +625,17 @@ static cudaError_t set_attr_one(int bytes) {
 }
 
 cudaError_t gemm_set_smem_attrs() {
-  int maxb = 0;
-  for (int bn = 16; bn <= 128; bn *= 2) {
-    const int a = (int)make_plan(true, bn, kMaxE).smem, b = (int)make_plan(false, bn, kMaxE).smem;
-    if (a > maxb) maxb = a;
-    if (b > maxb) maxb = b;
-  }
+  // every plan stays below the opt-in limit (200 KB of stages + at most 16 KB of tile table)
+  int dev = 0, maxb = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&maxb, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  if (e != cudaSuccess) return e;
+  maxb -= 1024;   // room for the kernels' static shared memory
   cudaError_t errs[8] = {set_attr_one<true, 16>(maxb),  set_attr_one<true, 32>(maxb),  set_attr_one<true, 64>(maxb),
                          set_attr_one<true, 128>(maxb), set_attr_one<false, 16>(maxb), set_attr_one<false, 32>(maxb),
                          set_attr_one<false, 64>(maxb), set_attr_one<false, 128>(maxb)};
-  for (cudaError_t e : errs)
-    if (e != cudaSuccess) return e;
+  for (cudaError_t x : errs)
+    if (x != cudaSuccess) return x;
   return cudaSuccess;
 }
 
@@ -640,12 +652,15 @@ static void launch_bn(int BN, int grid, size_t smem, cudaStream_t stream, const 
 
 // returns 0 ok, 1 cuda error, 2 tensor map failure
 int launch_gemm(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, const float* x_scale,
-                const uint8_t* w_vals, const uint8_t* w_meta, const uint8_t* w_scales, const float* w_scale,
-                const int32_t* off, int E, int N, int K, int R, int max_rows, void* Y, int y_f32, int* status,
-                int num_sms, cudaStream_t stream) {
+                const uint8_t* w_packed, const float* w_scale, const int32_t* off, int E, int N, int K, int R,
+                int max_rows, void* Y, int y_f32, int* status, int num_sms, cudaStream_t stream) {
   EncodeTiledFn enc = get_encode_fn();
   if (enc == nullptr) return 2;
-  const GemmPlan g = make_plan(sparse, gemm_pick_bn(max_rows), E);
+  const int BN = gemm_pick_bn(max_rows);
+  const long long bound = (((long long)R + BN - 1) / BN + E) * (N / kTileN);
+  long long tcap = (bound + num_sms - 1) / num_sms;
+  if (tcap > kMaxTableTiles) tcap = kMaxTableTiles;
+  const GemmPlan g = make_plan(sparse, BN, E, (int)tcap);
   const int box_h = g.BN < 32 ? g.BN : 32;
   const int kbps = g.cps * (sparse ? 2 : 4);
   const int rcap = R + kActScalePadRows;
@@ -673,10 +688,10 @@ int launch_gemm(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, co
       return 2;
   }
   GemmParams p;
-  p.a_scales = a_scales; p.x_scale = x_scale; p.w_vals = w_vals; p.w_meta = w_meta; p.w_scales = w_scales;
+  p.a_scales = a_scales; p.x_scale = x_scale; p.w_packed = w_packed;
   p.w_scale = w_scale; p.off = off; p.Y = Y; p.status = status;
   p.E = E; p.N = N; p.K = K; p.R = R; p.y_f32 = y_f32; p.rcap = rcap;
-  p.stages = g.stages; p.nacc = g.nacc;
+  p.stages = g.stages; p.nacc = g.nacc; p.tcap = g.tcap;
   if (sparse)
     launch_bn<true>(g.BN, num_sms, g.smem, stream, tb, ts, p);
   else

@@ -21,6 +21,8 @@ namespace gsg {
 constexpr int kTileN = 128;            // weight rows per tile (MMA M)
 constexpr int kChunkK = 256;           // logical K per pipeline stage / metadata chunk
 constexpr int kActScalePadRows = 256;  // extra zero rows of the quad activation-scale layout
+constexpr int kSparseChunkBytes = 11264;  // packed weight chunk block: values 8192 | meta 2048 | scales 1024
+constexpr int kDenseChunkBytes = 18432;   // dense control chunk block: codes 16384 | scales 2048
 constexpr float kTensorScaleDen = 2688.0f;  // 6 * 448
 
 // ------------------------------------------------------------------ status word

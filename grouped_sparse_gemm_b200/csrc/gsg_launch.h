@@ -9,8 +9,8 @@ namespace gsg {
 
 // gsg_pack.cu
 int pack_partials_per_expert(int N, int K);
-cudaError_t launch_pack(bool sparse, const float* W, int E, int N, int K, uint8_t* values, uint8_t* meta,
-                        uint8_t* scales, float* w_tensor_scale, float* partial, int* status, cudaStream_t stream);
+cudaError_t launch_pack(bool sparse, const float* W, int E, int N, int K, uint8_t* packed, float* w_tensor_scale,
+                        float* partial, int* status, cudaStream_t stream);
 
 // gsg_quant.cu
 int quant_partials(long long n_elems);
@@ -35,8 +35,7 @@ bool gemm_supported(int E);
 int gemm_pick_bn(int max_rows);
 cudaError_t gemm_set_smem_attrs();
 int launch_gemm(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, const float* x_scale,
-                const uint8_t* w_vals, const uint8_t* w_meta, const uint8_t* w_scales, const float* w_scale,
-                const int32_t* off, int E, int N, int K, int R, int max_rows, void* Y, int y_f32, int* status,
-                int num_sms, cudaStream_t stream);
+                const uint8_t* w_packed, const float* w_scale, const int32_t* off, int E, int N, int K, int R,
+                int max_rows, void* Y, int y_f32, int* status, int num_sms, cudaStream_t stream);
 
 }  // namespace gsg

@@ -9,8 +9,8 @@
 // (fp32, ties to the lower pair); the per-expert fp32 tensor scale is amax / 2688.
 //
 // Two launches per call: (1) per-expert partial amax of the kept weights, (2) one thread per
-// 32-block (sparse) or 16-block (dense) writes codes, metadata and the scale directly in the
-// tile-major layout the grouped GEMM streams (see include/gsg.h).
+// 32-block (sparse) or 16-block (dense) writes codes, metadata and the scale directly into the
+// interleaved tile-major chunk blocks the grouped GEMM streams (see include/gsg.h).
 #include "gsg_internal.cuh"
 
 namespace gsg {
@@ -104,8 +104,7 @@ __device__ float expert_scale_from_partials(const float* partial, int e, int npa
 // (2a) sparse encode: one thread per 32-block (4 groups, 16 retained values).
 __global__ void __launch_bounds__(kPackThreads)
 pack_sparse_encode_kernel(const float* __restrict__ W, int N, int K, const float* __restrict__ partial,
-                          int nparts, uint8_t* __restrict__ values, uint8_t* __restrict__ meta,
-                          uint8_t* __restrict__ scales, float* __restrict__ w_tensor_scale) {
+                          int nparts, uint8_t* __restrict__ packed, float* __restrict__ w_tensor_scale) {
   __shared__ float red[32];
   const int e = blockIdx.y;
   const float s = expert_scale_from_partials(partial, e, nparts, red);
@@ -113,7 +112,7 @@ pack_sparse_encode_kernel(const float* __restrict__ W, int N, int K, const float
   const float six_s = __fmul_rn(6.0f, s);
   const int blocks_per_row = K / 32;
   const long long nblk = (long long)N * blocks_per_row;
-  const int NT = N / kTileN, KB = K / 128, KC = K / kChunkK;
+  const int NT = N / kTileN, KC = K / kChunkK;
   for (long long bi = (long long)blockIdx.x * blockDim.x + threadIdx.x; bi < nblk;
        bi += (long long)gridDim.x * blockDim.x) {
     const int n = int(bi / blocks_per_row), b = int(bi % blocks_per_row);
@@ -141,26 +140,23 @@ pack_sparse_encode_kernel(const float* __restrict__ W, int N, int K, const float
     for (int i = 0; i < 16; ++i)
       codes |= uint64_t(e2m1_encode(__fmul_rn(kept[i], bs.inv))) << (4 * i);
     const int nt = n / kTileN, r = n % kTileN;
-    const size_t tile = (size_t)e * NT + nt;
-    // values: k-block b/4, stored values 16*(b%4) .. +15 -> bytes 8*(b%4) .. +7 of the row
-    const int kb = b >> 2, q = b & 3;
-    const size_t vpos = (tile * KB + kb) * 4096 + (r >> 3) * 256 + (q >> 1) * 128 + (r & 7) * 16 + (q & 1) * 8;
-    *reinterpret_cast<uint64_t*>(values + vpos) = codes;
-    // metadata: chunk b/8, groups 4*(b%8) .. +3 -> bytes 2*(b%8), +1 of the row
-    const int kc = b >> 3, g8 = b & 7;
-    const size_t mpos = (tile * KC + kc) * 2048 + (size_t)r * 16 + 2 * g8;
+    // chunk block of (e, nt, chunk b/8); k-block h = (b/4)%2 of the chunk, 32-block q = b%4
+    const int kc = b >> 3, h = (b >> 2) & 1, q = b & 3, g8 = b & 7;
+    uint8_t* cb = packed + (((size_t)e * NT + nt) * KC + kc) * kSparseChunkBytes;
+    // values: stored values 16*q .. +15 of the k-block -> bytes 8*q .. +7 of the row
+    *reinterpret_cast<uint64_t*>(cb + h * 4096 + (r >> 3) * 256 + (q >> 1) * 128 + (r & 7) * 16 + (q & 1) * 8) = codes;
+    // metadata: groups 4*(b%8) .. +3 of the chunk -> bytes 2*(b%8), +1 of the row
     const uint32_t m16 = pat[0] | (pat[1] << 4) | (pat[2] << 8) | (pat[3] << 12);
-    *reinterpret_cast<uint16_t*>(meta + mpos) = uint16_t(m16);
-    // scale: atom of k-block b/4, block j = b%4
-    scales[(tile * KB + kb) * 512 + 16 * (r & 31) + 4 * (r >> 5) + q] = uint8_t(bs.sc);
+    *reinterpret_cast<uint16_t*>(cb + 8192 + r * 16 + 2 * g8) = uint16_t(m16);
+    // scale atom of k-block h
+    cb[10240 + h * 512 + 16 * (r & 31) + 4 * (r >> 5) + q] = uint8_t(bs.sc);
   }
 }
 
 // (2b) dense encode: one thread per 16-block.
 __global__ void __launch_bounds__(kPackThreads)
 pack_dense_encode_kernel(const float* __restrict__ W, int N, int K, const float* __restrict__ partial,
-                         int nparts, uint8_t* __restrict__ codes_out, uint8_t* __restrict__ scales,
-                         float* __restrict__ w_tensor_scale) {
+                         int nparts, uint8_t* __restrict__ packed, float* __restrict__ w_tensor_scale) {
   __shared__ float red[32];
   const int e = blockIdx.y;
   const float s = expert_scale_from_partials(partial, e, nparts, red);
@@ -168,7 +164,7 @@ pack_dense_encode_kernel(const float* __restrict__ W, int N, int K, const float*
   const float six_s = __fmul_rn(6.0f, s);
   const int blocks_per_row = K / 16;
   const long long nblk = (long long)N * blocks_per_row;
-  const int NT = N / kTileN, KB = K / 64;
+  const int NT = N / kTileN, KC = K / kChunkK;
   for (long long bi = (long long)blockIdx.x * blockDim.x + threadIdx.x; bi < nblk;
        bi += (long long)gridDim.x * blockDim.x) {
     const int n = int(bi / blocks_per_row), b = int(bi % blocks_per_row);
@@ -184,11 +180,11 @@ pack_dense_encode_kernel(const float* __restrict__ W, int N, int K, const float*
 #pragma unroll
     for (int i = 0; i < 16; ++i) c |= uint64_t(e2m1_encode(__fmul_rn(w[i], bs.inv))) << (4 * i);
     const int nt = n / kTileN, r = n % kTileN;
-    const size_t tile = (size_t)e * NT + nt;
-    const int kb = b >> 2, q = b & 3;
-    const size_t vpos = (tile * KB + kb) * 4096 + (r >> 3) * 256 + (q >> 1) * 128 + (r & 7) * 16 + (q & 1) * 8;
-    *reinterpret_cast<uint64_t*>(codes_out + vpos) = c;
-    scales[(tile * KB + kb) * 512 + 16 * (r & 31) + 4 * (r >> 5) + q] = uint8_t(bs.sc);
+    // chunk block of (e, nt, chunk b/16); k-block h = (b/4)%4 of the chunk (64 K each), q = b%4
+    const int kc = b >> 4, h = (b >> 2) & 3, q = b & 3;
+    uint8_t* cb = packed + (((size_t)e * NT + nt) * KC + kc) * kDenseChunkBytes;
+    *reinterpret_cast<uint64_t*>(cb + h * 4096 + (r >> 3) * 256 + (q >> 1) * 128 + (r & 7) * 16 + (q & 1) * 8) = c;
+    cb[16384 + h * 512 + 16 * (r & 31) + 4 * (r >> 5) + q] = uint8_t(bs.sc);
   }
 }
 
@@ -201,9 +197,8 @@ int pack_partials_per_expert(int N, int K) {
   return int(want);
 }
 
-cudaError_t launch_pack(bool sparse, const float* W, int E, int N, int K, uint8_t* values,
-                        uint8_t* meta, uint8_t* scales, float* w_tensor_scale, float* partial,
-                        int* status, cudaStream_t stream) {
+cudaError_t launch_pack(bool sparse, const float* W, int E, int N, int K, uint8_t* packed, float* w_tensor_scale,
+                        float* partial, int* status, cudaStream_t stream) {
   const int P = pack_partials_per_expert(N, K);
   const long long groups = (long long)N * K / 8;
   dim3 g1(P, E);
@@ -218,11 +213,9 @@ cudaError_t launch_pack(bool sparse, const float* W, int E, int N, int K, uint8_
   if (nb > 1024) nb = 1024;
   dim3 g2((unsigned)nb, E);
   if (sparse)
-    pack_sparse_encode_kernel<<<g2, kPackThreads, 0, stream>>>(W, N, K, partial, P, values, meta,
-                                                               scales, w_tensor_scale);
+    pack_sparse_encode_kernel<<<g2, kPackThreads, 0, stream>>>(W, N, K, partial, P, packed, w_tensor_scale);
   else
-    pack_dense_encode_kernel<<<g2, kPackThreads, 0, stream>>>(W, N, K, partial, P, values, scales,
-                                                              w_tensor_scale);
+    pack_dense_encode_kernel<<<g2, kPackThreads, 0, stream>>>(W, N, K, partial, P, packed, w_tensor_scale);
   return cudaGetLastError();
 }
 

@@ -22,16 +22,19 @@
  *     patterns.  Multi-dimensional buffers are dense, last index fastest.
  *   - Re-entrant across streams; the only global state is the device status word.
  *
- * Packed weight layouts (tile-major, the order the GEMM streams them; n-tile = 128 output
- * rows, NT = N/128; k-block = one MMA step = 64 stored 4-bit values per row):
- *   sparse values  [E][NT][K/128][4096 B]  row r (0..127), stored value v (0..63) of the k-block
- *                  -> byte c = v/2 (low nibble = even v) at (r/8)*256 + (c/16)*128 + (r%8)*16 + c%16.
- *                  Stored values are the four retained E2M1 codes of each 8-group in K order.
- *   sparse meta    [E][NT][K/256][2048 B] row r, 8-group g of the 256-wide chunk (0..31)
- *                  -> byte r*16 + g/2, low nibble = even g; nibble = i0 | i1 << 2 (kept pairs i0<i1).
- *   weight scales  [E][NT][K/(4*sf)][512 B] row r, block j (0..3) of the k-block
- *                  -> byte 16*(r%32) + 4*(r/32) + j.  UE4M3 codes; sf = 32 sparse, 16 dense.
- *   dense codes    [E][NT][K/64][4096 B]  same index function as sparse values, v = K index.
+ * Packed weight layout (one buffer, tile-major, the order the GEMM streams it): for expert e,
+ * n-tile nt (128 output rows, NT = N/128) and 256-wide K chunk kc, one contiguous chunk block
+ * at ((e*NT + nt)*(K/256) + kc) * CB holding, for the chunk's MMA k-blocks h (64 stored 4-bit
+ * values per row each: 128 logical K sparse, 64 dense):
+ *   values  h*4096 + (r/8)*256 + (c/16)*128 + (r%8)*16 + c%16 for row r (0..127) and byte
+ *           c = v/2 of stored value v (0..63) of the k-block, low nibble = even v.  Sparse: the
+ *           four retained E2M1 codes of each 8-group in K order; dense: every code.
+ *   meta    (sparse) 8192 + r*16 + g/2 for 8-group g (0..31) of the chunk, low nibble = even g;
+ *           nibble = i0 | i1 << 2 (the kept pairs, i0 < i1).
+ *   scales  V + h*512 + 16*(r%32) + 4*(r/32) + j for block j (0..3) of k-block h: UE4M3 codes,
+ *           one per 32 logical weights (sparse) or 16 (dense).
+ * Sparse: CB = 11264, V = 10240 (2 k-blocks, 2.75 bit/weight).  Dense: CB = 18432, V = 16384
+ * (4 k-blocks, 4.5 bit/weight).
  * Activation layouts (R routed rows; KBa = K/(4*sf)):
  *   codes  [R][K/2]  row-major E2M1, low nibble = even k.
  *   scales [KBa][R + 256][4][4 B]: entry (kb, r, c, j) = UE4M3 scale of block 4*kb + j of
@@ -74,10 +77,8 @@ enum { GSG_OUT_BF16 = 0, GSG_OUT_F32 = 1 };
 /* ----------------------------------------------------------------------------------------
  * Buffer sizes in bytes (host-only arithmetic, no GPU access).
  */
-size_t gsg_sparse_values_bytes(int E, int N, int K);          /* E*N*K/4                    */
-size_t gsg_sparse_meta_bytes(int E, int N, int K);            /* E*N*K/16                   */
-size_t gsg_weight_scales_bytes(int E, int N, int K, int sf_block); /* E*N*K/sf_block      */
-size_t gsg_dense_codes_bytes(int E, int N, int K);            /* E*N*K/2                    */
+size_t gsg_sparse_packed_bytes(int E, int N, int K);          /* E*N*K*11/32 (2.75 bit)     */
+size_t gsg_dense_packed_bytes(int E, int N, int K);           /* E*N*K*9/16 (4.5 bit)       */
 size_t gsg_act_codes_bytes(int R, int K);                     /* R*K/2                      */
 size_t gsg_act_scales_bytes(int R, int K, int sf_block);      /* K/(4 sf) * (R+256) * 16    */
 /* Workspace needed by `op` (0 when none).  T = tokens, k = experts per token. */
@@ -89,19 +90,18 @@ size_t gsg_workspace_size(int op, int E, int N, int K, int T, int k);
  * W fp32 [E][N][K] (K contiguous).  Per 8-group of K the two adjacent pairs with the largest
  * energy w0*w0 + w1*w1 (fp32, ties -> lower pair) are kept; s_w[e] = amax(kept W_e)/2688
  * (1 if 0); per 32-block b: sc = UE4M3(b / (6 s_w)), codes = E2M1(w / (dec(sc) s_w)),
- * round-to-nearest-even with saturation.  Writes values/meta/scales in the layouts above and
- * w_tensor_scale fp32 [E].  Non-finite W sets GSG_ERR_NONFINITE on the device.
+ * round-to-nearest-even with saturation.  Writes the packed layout above (w_packed, size
+ * gsg_sparse_packed_bytes) and w_tensor_scale fp32 [E].  Non-finite W sets GSG_ERR_NONFINITE.
  */
-gsg_status_t gsg_pack_sparse_nvfp4(const float* W, int E, int N, int K,
-                                   uint8_t* values, uint8_t* meta, uint8_t* scales,
+gsg_status_t gsg_pack_sparse_nvfp4(const float* W, int E, int N, int K, uint8_t* w_packed,
                                    float* w_tensor_scale,
                                    void* workspace, size_t workspace_bytes, void* stream);
 
 /* gsg_pack_dense_nvfp4 -- dense NVFP4 packer for the in-repo control GEMM (16-element
  * blocks, the block size the dense block-scaled MMA takes; §D.2, p.19: the control differs
- * from the sparse kernel only in sparsity).  codes [E][NT][K/64][4096], scales [E][NT][K/64][512]. */
-gsg_status_t gsg_pack_dense_nvfp4(const float* W, int E, int N, int K,
-                                  uint8_t* codes, uint8_t* scales, float* w_tensor_scale,
+ * from the sparse kernel only in sparsity).  Packed layout above, size gsg_dense_packed_bytes. */
+gsg_status_t gsg_pack_dense_nvfp4(const float* W, int E, int N, int K, uint8_t* w_packed,
+                                  float* w_tensor_scale,
                                   void* workspace, size_t workspace_bytes, void* stream);
 
 /* ----------------------------------------------------------------------------------------
@@ -139,7 +139,8 @@ gsg_status_t gsg_quantize_act_nvfp4(const uint16_t* X, int T, int K, int sf_bloc
  * weight as operand A; §2 (p.3): the sparse NVFP4 path peaks at 2x dense NVFP4.
  * For each expert e and routed row r in [off[e], off[e+1]):
  *     Y[r][n] = s_x * s_w[e] * sum_k a[r][k] * w[e][n][k]      (fp32 accumulation)
- * a_codes/a_scales from gsg_quantize_act_nvfp4 (sf_block 32); w_* from gsg_pack_sparse_nvfp4.
+ * a_codes/a_scales from gsg_quantize_act_nvfp4 (sf_block 32); w_packed and w_tensor_scale from
+ * gsg_pack_sparse_nvfp4.
  * expert_offsets int32 [E+1], monotone, off[0] = 0, off[E] <= R.  max_rows_per_expert is a
  * host-side hint that picks the token tile (<= 0: unknown).  Y [R][N] bf16 (y_dtype
  * GSG_OUT_BF16) or fp32 (GSG_OUT_F32); rows >= off[E] are not written.  No workspace.
@@ -148,8 +149,7 @@ gsg_status_t gsg_quantize_act_nvfp4(const uint16_t* X, int T, int K, int sf_bloc
  */
 gsg_status_t gsg_grouped_sparse_gemm(const uint8_t* a_codes, const uint8_t* a_scales,
                                      const float* x_tensor_scale,
-                                     const uint8_t* w_values, const uint8_t* w_meta,
-                                     const uint8_t* w_scales, const float* w_tensor_scale,
+                                     const uint8_t* w_packed, const float* w_tensor_scale,
                                      const int32_t* expert_offsets, int E, int N, int K, int R,
                                      int max_rows_per_expert, void* Y, int y_dtype, void* stream);
 
@@ -158,8 +158,7 @@ gsg_status_t gsg_grouped_sparse_gemm(const uint8_t* a_codes, const uint8_t* a_sc
  * gsg_pack_dense_nvfp4.  Same semantics as gsg_grouped_sparse_gemm. */
 gsg_status_t gsg_grouped_dense_gemm(const uint8_t* a_codes, const uint8_t* a_scales,
                                     const float* x_tensor_scale,
-                                    const uint8_t* w_codes, const uint8_t* w_scales,
-                                    const float* w_tensor_scale,
+                                    const uint8_t* w_packed, const float* w_tensor_scale,
                                     const int32_t* expert_offsets, int E, int N, int K, int R,
                                     int max_rows_per_expert, void* Y, int y_dtype, void* stream);
 

@@ -9,15 +9,17 @@ order its grouped GEMM consumes it, and this module restates those index
 functions independently of the CUDA code, so packed bytes can be compared
 bit for bit.  Constants: weight tiles of 128 output rows ("n-tiles"); an MMA
 k-block is 64 stored 4-bit values per row (128 logical K for the paired 4:8
-weight, 64 for the dense control); a metadata chunk is 256 logical K.
+weight, 64 for the dense control); a chunk is 256 logical K.
 
-Weight values   [E][NT][KB][4096 B]: in a k-block, row r (0..127), stored value
-                v (0..63): byte c = v // 2 (low nibble = even v) at
-                (r//8)*256 + (c//16)*128 + (r%8)*16 + c%16.
-Weight metadata [E][NT][KC][2048 B]: row r, 8-group g of the chunk (0..31):
-                byte r*16 + g//2, low nibble = even g.
-Block scales    [E][NT][KB][512 B]: row r, block j of the k-block (0..3):
-                byte 16*(r%32) + 4*(r//32) + j.
+The packed weight buffer is a sequence of chunk blocks, one per (expert,
+n-tile, chunk), each holding the chunk's values, then (sparse) its metadata,
+then its scale atoms:
+  values  k-block h, row r (0..127), stored value v (0..63): byte c = v // 2
+          (low nibble = even v) at h*4096 + (r//8)*256 + (c//16)*128 + (r%8)*16 + c%16
+  meta    8192 + r*16 + g//2 for 8-group g (0..31) of the chunk, low nibble = even g
+  scales  V + h*512 + 16*(r%32) + 4*(r//32) + j for block j (0..3) of k-block h
+Sparse blocks are 11264 bytes (2 k-blocks, V = 10240), dense 18432 (4 k-blocks,
+V = 16384).
 Activation codes  [R][K/2] row-major, low nibble = even k.
 Activation scales [KB][R + 256][4][4] ("quad" entries): entry (kb, r, c, j)
                 holds the scale of block 4*kb + j of routed row r + 32*c, or 0
@@ -128,6 +130,35 @@ def untile_scales(packed: np.ndarray, N: int, S: int) -> np.ndarray:
     kb, j = s // 4, s % 4
     pos = (nt * KB + kb) * 512 + 16 * (r % 32) + 4 * (r // 32) + j
     return flat[pos]
+
+
+SPARSE_CHUNK_BYTES = 11264
+DENSE_CHUNK_BYTES = 18432
+
+
+def packed_sparse(codes: np.ndarray, patterns: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """One expert's canonical parts -> its packed chunk blocks [NT, K/256, 11264].
+
+    codes [N, K/2] (retained values), patterns [N, K/8], scales [N, K/32].
+    """
+    N, Kh = codes.shape
+    K = 2 * Kh
+    NT, KC = N // TILE_N, K // 256
+    out = np.zeros((NT, KC, SPARSE_CHUNK_BYTES), dtype=np.uint8)
+    out[:, :, :8192] = tile_values_fast(codes).reshape(NT, KC, 8192)
+    out[:, :, 8192:10240] = tile_meta(patterns).reshape(NT, KC, 2048)
+    out[:, :, 10240:] = tile_scales(scales).reshape(NT, KC, 1024)
+    return out
+
+
+def packed_dense(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """One expert's dense control parts -> chunk blocks [NT, K/256, 18432] (codes [N, K], scales [N, K/16])."""
+    N, K = codes.shape
+    NT, KC = N // TILE_N, K // 256
+    out = np.zeros((NT, KC, DENSE_CHUNK_BYTES), dtype=np.uint8)
+    out[:, :, :16384] = tile_values_fast(codes).reshape(NT, KC, 16384)
+    out[:, :, 16384:] = tile_scales(scales).reshape(NT, KC, 2048)
+    return out
 
 
 def pack_act_codes(codes: np.ndarray) -> np.ndarray:

@@ -16,28 +16,24 @@ from oracle import route as oroute
 
 
 def oracle_pack_sparse(W: np.ndarray):
-    """W fp32 [E, N, K] -> (values, meta, scales) in the library's tiled layout + s_w [E] + canonical parts."""
-    vals, metas, scs, sws, canon = [], [], [], [], []
+    """W fp32 [E, N, K] -> (packed bytes in the library's layout, s_w [E], canonical parts per expert)."""
+    blocks, sws, canon = [], [], []
     for e in range(W.shape[0]):
         codes, pats, scales, s_w = opack.pack_sparse_expert(W[e])
-        vals.append(olayout.tile_values_fast(codes).reshape(-1))
-        metas.append(olayout.tile_meta(pats).reshape(-1))
-        scs.append(olayout.tile_scales(scales).reshape(-1))
+        blocks.append(olayout.packed_sparse(codes, pats, scales).reshape(-1))
         sws.append(s_w)
         canon.append((codes, pats, scales))
-    return (np.concatenate(vals), np.concatenate(metas), np.concatenate(scs),
-            np.array(sws, dtype=np.float32), canon)
+    return np.concatenate(blocks), np.array(sws, dtype=np.float32), canon
 
 
 def oracle_pack_dense(W: np.ndarray, sf_block: int = 16):
-    vals, scs, sws, canon = [], [], [], []
+    blocks, sws, canon = [], [], []
     for e in range(W.shape[0]):
         codes, scales, s_w = opack.pack_dense_expert(W[e], sf_block)
-        vals.append(olayout.tile_values_fast(codes).reshape(-1))
-        scs.append(olayout.tile_scales(scales).reshape(-1))
+        blocks.append(olayout.packed_dense(codes, scales).reshape(-1))
         sws.append(s_w)
         canon.append((codes, scales))
-    return np.concatenate(vals), np.concatenate(scs), np.array(sws, dtype=np.float32), canon
+    return np.concatenate(blocks), np.array(sws, dtype=np.float32), canon
 
 
 def oracle_act(x: np.ndarray, sf_block: int, perm_src, top_k: int, s_x=None):

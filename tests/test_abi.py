@@ -35,10 +35,8 @@ def test_every_declared_symbol_is_exported(L):
 
 def test_sizes(L):
     E, N, K = 3, 256, 512
-    total = L.gsg_sparse_values_bytes(E, N, K) + L.gsg_sparse_meta_bytes(E, N, K) + \
-        L.gsg_weight_scales_bytes(E, N, K, 32)
-    assert total * 8 == 2.75 * E * N * K                       # 2.75 bit per weight
-    assert L.gsg_dense_codes_bytes(E, N, K) + L.gsg_weight_scales_bytes(E, N, K, 16) == 4.5 * E * N * K / 8
+    assert L.gsg_sparse_packed_bytes(E, N, K) * 8 == 2.75 * E * N * K     # 2.75 bit per weight
+    assert L.gsg_dense_packed_bytes(E, N, K) * 8 == 4.5 * E * N * K
     assert L.gsg_act_codes_bytes(10, 256) == 1280
     assert L.gsg_act_scales_bytes(10, 256, 32) == 2 * (10 + 256) * 16
     assert L.gsg_workspace_size(gsg.OP_ROUTE, 384, 0, 0, 64, 8) == 0          # single-launch routing
@@ -56,15 +54,15 @@ P = ctypes.c_void_p(16)   # a non-NULL, 16-byte aligned placeholder never derefe
 
 def test_host_argument_checks(L):
     # bad shapes (K % 256, N % 128) -> unsupported shape, no launch
-    assert L.gsg_pack_sparse_nvfp4(P, 1, 128, 100, P, P, P, P, P, 1 << 20, None) == -2
-    assert L.gsg_pack_sparse_nvfp4(P, 1, 100, 256, P, P, P, P, P, 1 << 20, None) == -2
-    assert L.gsg_pack_sparse_nvfp4(None, 1, 128, 256, P, P, P, P, P, 1 << 20, None) == -1
-    assert L.gsg_pack_sparse_nvfp4(P, 1, 128, 256, P, P, P, P, None, 0, None) == -7
-    assert L.gsg_grouped_sparse_gemm(P, P, P, P, P, P, P, P, 4, 128, 300, 8, -1, P, 0, None) == -2
-    assert L.gsg_grouped_sparse_gemm(P, P, P, P, P, P, P, P, 4, 128, 256, 8, -1, P, 7, None) == -1
-    assert L.gsg_grouped_sparse_gemm(P, P, P, P, P, P, P, P, 2000, 128, 256, 8, -1, P, 0, None) == -2
-    assert L.gsg_grouped_sparse_gemm(P, P, P, P, None, P, P, P, 4, 128, 256, 8, -1, P, 0, None) == -1
-    assert L.gsg_grouped_sparse_gemm(P, P, P, P, P, P, P, P, 4, 128, 256, 0, -1, P, 0, None) == 0  # R = 0
+    assert L.gsg_pack_sparse_nvfp4(P, 1, 128, 100, P, P, P, 1 << 20, None) == -2
+    assert L.gsg_pack_sparse_nvfp4(P, 1, 100, 256, P, P, P, 1 << 20, None) == -2
+    assert L.gsg_pack_sparse_nvfp4(None, 1, 128, 256, P, P, P, 1 << 20, None) == -1
+    assert L.gsg_pack_sparse_nvfp4(P, 1, 128, 256, P, P, None, 0, None) == -7
+    assert L.gsg_grouped_sparse_gemm(P, P, P, P, P, P, 4, 128, 300, 8, -1, P, 0, None) == -2
+    assert L.gsg_grouped_sparse_gemm(P, P, P, P, P, P, 4, 128, 256, 8, -1, P, 7, None) == -1
+    assert L.gsg_grouped_sparse_gemm(P, P, P, P, P, P, 2000, 128, 256, 8, -1, P, 0, None) == -2
+    assert L.gsg_grouped_sparse_gemm(P, P, P, None, P, P, 4, 128, 256, 8, -1, P, 0, None) == -1
+    assert L.gsg_grouped_sparse_gemm(P, P, P, P, P, P, 4, 128, 256, 0, -1, P, 0, None) == 0  # R = 0
     assert L.gsg_moe_route_permute(P, 4, 2, 0, P, P, P, None, 0, None) == -2
     assert L.gsg_moe_route_permute(P, 4, 2, 5000, P, P, P, None, 0, None) == -2
     assert L.gsg_moe_route_permute(P, 8192, 8, 16, P, P, P, None, 0, None) == -7

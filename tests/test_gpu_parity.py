@@ -40,10 +40,8 @@ def test_pack_sparse_bit_exact(gsg, E, N, K):
     if E > 1:
         W[1].mul_(1e-3)                # a small-magnitude expert
     pw = gsg.pack_sparse_nvfp4(W.to(DEV))
-    vals, meta, scs, sws, _ = tl.oracle_pack_sparse(W.numpy())
-    np.testing.assert_array_equal(pw.values.cpu().numpy(), vals)
-    np.testing.assert_array_equal(pw.meta.cpu().numpy(), meta)
-    np.testing.assert_array_equal(pw.scales.cpu().numpy(), scs)
+    packed, sws, _ = tl.oracle_pack_sparse(W.numpy())
+    np.testing.assert_array_equal(pw.packed.cpu().numpy(), packed)
     np.testing.assert_array_equal(pw.w_scale.cpu().numpy(), sws)
     _status_ok(gsg)
 
@@ -54,9 +52,8 @@ def test_pack_dense_bit_exact(gsg, E, N, K):
     W = inputs.all_weights(cfg)
     W[0, 1] = 0.0
     pw = gsg.pack_dense_nvfp4(W.to(DEV))
-    vals, scs, sws, _ = tl.oracle_pack_dense(W.numpy(), 16)
-    np.testing.assert_array_equal(pw.codes.cpu().numpy(), vals)
-    np.testing.assert_array_equal(pw.scales.cpu().numpy(), scs)
+    packed, sws, _ = tl.oracle_pack_dense(W.numpy(), 16)
+    np.testing.assert_array_equal(pw.packed.cpu().numpy(), packed)
     np.testing.assert_array_equal(pw.w_scale.cpu().numpy(), sws)
 
 
@@ -151,11 +148,10 @@ def _gemm_case(counts, N, K, seed=0, sparse=True):
     sf = 32 if sparse else 16
     a_codes, a_quad, s_x, q, sc = tl.oracle_act(X, sf, None, 1)
     if sparse:
-        vals, meta, scs, sws, canon = tl.oracle_pack_sparse(W)
-        w = dict(values=vals, meta=meta, scales=scs, w_scale=sws)
+        packed, sws, canon = tl.oracle_pack_sparse(W)
     else:
-        vals, scs, sws, canon = tl.oracle_pack_dense(W, 16)
-        w = dict(codes=vals, scales=scs, w_scale=sws)
+        packed, sws, canon = tl.oracle_pack_dense(W, 16)
+    w = dict(packed=packed, w_scale=sws)
     return dict(E=E, N=N, K=K, R=int(off[-1]), off=off, a_codes=a_codes, a_quad=a_quad, s_x=s_x, q=q, sc=sc,
                 w=w, canon=canon, sws=sws, sf=sf)
 
@@ -167,11 +163,11 @@ def _run_gemm(gsg, c, sparse, hint, out_dtype):
                                    R=c["R"], K=c["K"], sf_block=c["sf"])
     off = t(c["off"])
     if sparse:
-        w = gsg.PackedSparseWeights(values=t(c["w"]["values"]), meta=t(c["w"]["meta"]), scales=t(c["w"]["scales"]),
-                                    w_scale=t(c["w"]["w_scale"]), E=c["E"], N=c["N"], K=c["K"])
+        w = gsg.PackedSparseWeights(packed=t(c["w"]["packed"]), w_scale=t(c["w"]["w_scale"]), E=c["E"], N=c["N"],
+                                    K=c["K"])
         return gsg.grouped_sparse_gemm(act, w, off, max_rows_per_expert=hint, out_dtype=out_dtype)
-    w = gsg.PackedDenseWeights(codes=t(c["w"]["codes"]), scales=t(c["w"]["scales"]), w_scale=t(c["w"]["w_scale"]),
-                               E=c["E"], N=c["N"], K=c["K"])
+    w = gsg.PackedDenseWeights(packed=t(c["w"]["packed"]), w_scale=t(c["w"]["w_scale"]), E=c["E"], N=c["N"],
+                               K=c["K"])
     return gsg.grouped_dense_gemm(act, w, off, max_rows_per_expert=hint, out_dtype=out_dtype)
 
 
@@ -224,17 +220,16 @@ def test_dense_and_sparse_agree_on_48_weights(gsg):
     counts, N, K = [20, 9], 128, 512
     c = _gemm_case(counts, N, K, sparse=True)
     # dense weights: scatter the retained codes with +0 at pruned slots; duplicate each 32-block scale
-    dv, ds = [], []
+    dblocks = []
     for (codes, pats, scales) in c["canon"]:
         full = np.zeros((N, K // 8, 4, 2), dtype=np.uint8)
         np.put_along_axis(full, opack.pattern_pairs(pats)[..., None].repeat(2, axis=-1),
                           codes.reshape(N, K // 8, 2, 2), axis=-2)
-        dv.append(olayout.tile_values_fast(full.reshape(N, K)).reshape(-1))
-        ds.append(olayout.tile_scales(np.repeat(scales, 2, axis=1)).reshape(-1))
+        dblocks.append(olayout.packed_dense(full.reshape(N, K), np.repeat(scales, 2, axis=1)).reshape(-1))
     # activations with 16-blocks carrying the same scale as their 32-block
     q, sc = c["q"], c["sc"]
     d = dict(c)
-    d["w"] = dict(codes=np.concatenate(dv), scales=np.concatenate(ds), w_scale=c["sws"])
+    d["w"] = dict(packed=np.concatenate(dblocks), w_scale=c["sws"])
     d["a_quad"] = olayout.quad_act_scales(np.repeat(sc, 2, axis=1)).reshape(-1)
     d["sf"] = 16
     y_sparse = _run_gemm(gsg, c, True, -1, torch.float32)
@@ -290,9 +285,7 @@ def test_gemm_full_size_sampled_30b_up(gsg):
     cfg = inputs.CONFIGS["30b_up_prefill"]
     E, N, K = cfg.E, cfg.N, cfg.K
     pw = gsg.PackedSparseWeights(
-        values=torch.empty(E * N * K // 4, dtype=torch.uint8, device=DEV),
-        meta=torch.empty(E * N * K // 16, dtype=torch.uint8, device=DEV),
-        scales=torch.empty(E * N * K // 32, dtype=torch.uint8, device=DEV),
+        packed=torch.empty(gsg.lib().gsg_sparse_packed_bytes(E, N, K), dtype=torch.uint8, device=DEV),
         w_scale=torch.empty(E, dtype=torch.float32, device=DEV), E=E, N=N, K=K)
     ids = inputs.routing(cfg)
     off, ps, ip = tl.route_np(ids, E)
@@ -301,18 +294,13 @@ def test_gemm_full_size_sampled_30b_up(gsg):
     canon, sws = {}, np.zeros(E, dtype=np.float32)
     for e in range(E):
         We = inputs.expert_weight(cfg, e, DEV)
-        sub = gsg.PackedSparseWeights(values=pw.values[e * N * K // 4:(e + 1) * N * K // 4],
-                                      meta=pw.meta[e * N * K // 16:(e + 1) * N * K // 16],
-                                      scales=pw.scales[e * N * K // 32:(e + 1) * N * K // 32],
-                                      w_scale=pw.w_scale[e:e + 1], E=1, N=N, K=K)
+        sub = pw.expert(e)
         gsg.pack_sparse_nvfp4(We[None], out=sub)
         if e in sample_e:
             codes, pats, scales, s_w = opack.pack_sparse_expert(We.cpu().numpy())
             canon[e] = (codes, pats, scales)
             sws[e] = s_w
-            np.testing.assert_array_equal(sub.values.cpu().numpy(), olayout.tile_values_fast(codes).reshape(-1))
-            np.testing.assert_array_equal(sub.meta.cpu().numpy(), olayout.tile_meta(pats).reshape(-1))
-            np.testing.assert_array_equal(sub.scales.cpu().numpy(), olayout.tile_scales(scales).reshape(-1))
+            np.testing.assert_array_equal(sub.packed.cpu().numpy(), olayout.packed_sparse(codes, pats, scales).reshape(-1))
             assert sub.w_scale.item() == s_w
     X = inputs.activations(cfg)
     r = gsg.moe_route_permute(ids.to(DEV), E)
