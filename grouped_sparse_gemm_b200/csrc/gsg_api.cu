@@ -135,6 +135,7 @@ gsg_status_t gsg_quantize_act_nvfp4(const uint16_t* X, int T, int K, int sf_bloc
   if (T < 0 || k < 1 || (sf_block != 16 && sf_block != 32)) return GSG_ERR_INVALID_ARG;
   if (K < 256 || K % 256 != 0) return GSG_ERR_UNSUPPORTED_SHAPE;
   if ((long long)T * k > (1ll << 30)) return GSG_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)T * (K / 16) >= (1ll << 31)) return GSG_ERR_UNSUPPORTED_SHAPE;  // 32-bit unit index
   if (inv_perm == nullptr && k != 1) return GSG_ERR_INVALID_ARG;
   if (!scales || !x_tensor_scale_out) return GSG_ERR_INVALID_ARG;
   if (T > 0 && (!X || !codes)) return GSG_ERR_INVALID_ARG;
@@ -160,7 +161,7 @@ static gsg_status_t gemm_common(bool sparse, const uint8_t* a_codes, const uint8
   if (!off || !w_packed || !w_scale || !x_scale) return GSG_ERR_INVALID_ARG;
   if (R == 0) return GSG_OK;  // nothing routed: nothing to compute or write
   if (!a_codes || !a_scales || !Y) return GSG_ERR_INVALID_ARG;
-  if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(w_packed)) return GSG_ERR_INVALID_ARG;
+  if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(w_packed) || !aligned16(Y)) return GSG_ERR_INVALID_ARG;
   DeviceState* d = nullptr;
   gsg_status_t st = device_state(&d);
   if (st != GSG_OK) return st;

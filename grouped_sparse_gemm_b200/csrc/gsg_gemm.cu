@@ -37,6 +37,7 @@ constexpr uint32_t kSetCols = 64;
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;   // 2 s
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColAcc = kNSets * kSetCols;       // first accumulator (192)
+constexpr int kOutStageBytes = 16 * 32 * 4;           // epilogue transpose buffer per warp
 
 struct GemmParams {
   const uint8_t* a_scales;
@@ -290,6 +291,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
   int* pref = offs + (E + 1);                    // [E+1]
   float* wsc = reinterpret_cast<float*>(pref + (E + 1));   // [E]
   int4* ttab = reinterpret_cast<int4*>((reinterpret_cast<uintptr_t>(wsc + E) + 15) & ~uintptr_t(15));   // [tcap]
+  // per-epilogue-warp staging buffer for 16 tokens x 32 output features (fp32 worst case)
+  uint8_t* ostage = reinterpret_cast<uint8_t*>(ttab + p.tcap);   // [4][kOutStageBytes]
   volatile int* abort_flag = &ctl->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -520,7 +523,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
   } else {
     // =============================== epilogue (warps 3..6 -> TMEM lane quadrants 3,0,1,2)
     const int q = warp & 3;
-    const int row = 32 * q + lane;
     const float sx = __ldg(p.x_scale);
     int it = 0;
     for (int j = 0; j < n_my; ++j, ++it) {
@@ -530,22 +532,50 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
       if (!wait_warp(accf_bar(acc), (uint32_t)(it / NACC) & 1u, abort_flag, p.status)) break;
       tc_fence_after();
       const float scale = __fmul_rn(sx, wsc[c.e]);
-      const int n = c.nt * kTileN + row;
       const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + kColAcc + (uint32_t)(acc * G::kAccStride);
+      // Each 16-token chunk: TMEM lane (= output feature) -> registers, scale, transpose through
+      // the warp's shared buffer into [token][32 features], then 16-byte stores of whole row
+      // segments (64 B bf16 / 128 B fp32 per token).
+      uint8_t* obuf = ostage + (size_t)(warp - 3) * kOutStageBytes;
+      const uint32_t obuf_s = smem_u32(obuf);
+      const size_t col0 = (size_t)c.nt * kTileN + 32 * q;       // first feature of this warp
       for (int c0 = 0; c0 < valid; c0 += 16) {
         float v[16];
         tc_ld_16(taddr + c0, v);
         if (p.y_f32) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            asm volatile("st.shared.f32 [%0], %1;" ::"r"(obuf_s + (uint32_t)(j * 128 + lane * 4)), "f"(__fmul_rn(v[j], scale)) : "memory");
+          __syncwarp();
           float* Y = static_cast<float*>(p.Y);
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (c0 + j < valid) Y[(size_t)(r0 + c0 + j) * p.N + n] = __fmul_rn(v[j], scale);
+          for (int k = 0; k < 4; ++k) {          // 16 tokens x 8 chunks of 16 B
+            const int ci = lane + 32 * k, tok = ci >> 3, part = ci & 7;
+            if (c0 + tok < valid) {
+              uint32_t a, b, cc, d;
+              lds128(obuf_s + (uint32_t)(tok * 128 + part * 16), a, b, cc, d);
+              *reinterpret_cast<uint4*>(Y + (size_t)(r0 + c0 + tok) * p.N + col0 + part * 4) = make_uint4(a, b, cc, d);
+            }
+          }
         } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const unsigned short h = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(v[j], scale)));
+            asm volatile("st.shared.u16 [%0], %1;" ::"r"(obuf_s + (uint32_t)(j * 64 + lane * 2)), "h"(h) : "memory");
+          }
+          __syncwarp();
           __nv_bfloat16* Y = static_cast<__nv_bfloat16*>(p.Y);
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (c0 + j < valid) Y[(size_t)(r0 + c0 + j) * p.N + n] = __float2bfloat16_rn(__fmul_rn(v[j], scale));
+          for (int k = 0; k < 2; ++k) {          // 16 tokens x 4 chunks of 16 B
+            const int ci = lane + 32 * k, tok = ci >> 2, part = ci & 3;
+            if (c0 + tok < valid) {
+              uint32_t a, b, cc, d;
+              lds128(obuf_s + (uint32_t)(tok * 64 + part * 16), a, b, cc, d);
+              *reinterpret_cast<uint4*>(Y + (size_t)(r0 + c0 + tok) * p.N + col0 + part * 8) = make_uint4(a, b, cc, d);
+            }
+          }
         }
+        __syncwarp();
       }
       tc_fence_before();
       __syncwarp();
@@ -568,7 +598,7 @@ struct GemmPlan {
   size_t smem;
 };
 
-constexpr int kSmemBudget = 200 * 1024;
+constexpr int kSmemBudget = 192 * 1024;
 
 // tcap: capacity of the per-CTA tile table (tiles beyond it are decoded on the fly); an upper
 // bound on a CTA's tiles is ceil((ceil(R/BN) + E) * NT / grid).
@@ -587,7 +617,7 @@ static GemmPlan make_plan(bool sparse, int BN, int E, int tcap) {
   if (g.nacc > kMaxAcc) g.nacc = kMaxAcc;
   const int nbars = 2 * g.stages + kNSets + 2 * g.nacc + 1;
   g.smem = 1024 + (size_t)g.stages * g.stage + nbars * 8 + sizeof(Ctl) + (size_t)(3 * E + 2) * 4 + 16 +
-           (size_t)tcap * 16;
+           (size_t)tcap * 16 + 4 * kOutStageBytes;
   return g;
 }
 

@@ -95,8 +95,9 @@ act_quant_kernel(QuantParams p) {
   for (long long base = (long long)gwarp * 32; base < U; base += (long long)nwarps * 32) {
     const long long unit = base + lane;
     const bool valid = unit < U;
-    const int t = valid ? int(unit / units_per_row) : 0;
-    const int c16 = valid ? int(unit % units_per_row) : 0;
+    const unsigned u32 = (unsigned)unit;   // U = T*K/16 < 2^31 is checked on the host
+    const int t = valid ? int(u32 / (unsigned)units_per_row) : 0;
+    const int c16 = valid ? int(u32 % (unsigned)units_per_row) : 0;
     float x[16];
     float amax = 0.0f;
     if (valid) {
@@ -137,19 +138,25 @@ act_quant_kernel(QuantParams p) {
       writer = (lane & 3) == 0;
     }
     if (!valid) continue;
-    for (int j = 0; j < p.k; ++j) {
-      int row = t;
-      if (p.inv_perm != nullptr) {
-        row = __ldg(p.inv_perm + (size_t)t * p.k + j);
-        if (row < 0 || row >= p.R) { set_status(p.status, GSG_ERR_BAD_ROUTING); continue; }
-      }
-      *reinterpret_cast<uint64_t*>(p.codes + (size_t)row * (p.K / 2) + (size_t)c16 * 8) = codes;
-      if (writer) {
-        uint32_t* sw = reinterpret_cast<uint32_t*>(p.scales);
+    // the token's destination rows, all loaded before any store (up to 16 at a time)
+    for (int j0 = 0; j0 < p.k; j0 += 16) {
+      int rows[16];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int rr = row - 32 * c;
-          if (rr >= 0) sw[((size_t)kb * p.rcap + rr) * 4 + c] = word;
+      for (int j = 0; j < 16; ++j)
+        rows[j] = (j0 + j < p.k) ? (p.inv_perm != nullptr ? __ldg(p.inv_perm + (size_t)t * p.k + j0 + j) : t) : -1;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        if (j0 + j >= p.k) break;
+        const int row = rows[j];
+        if (row < 0 || row >= p.R) { set_status(p.status, GSG_ERR_BAD_ROUTING); continue; }
+        *reinterpret_cast<uint64_t*>(p.codes + (size_t)row * (p.K / 2) + (size_t)c16 * 8) = codes;
+        if (writer) {
+          uint32_t* sw = reinterpret_cast<uint32_t*>(p.scales);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int rr = row - 32 * c;
+            if (rr >= 0) sw[((size_t)kb * p.rcap + rr) * 4 + c] = word;
+          }
         }
       }
     }

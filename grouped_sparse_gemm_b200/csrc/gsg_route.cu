@@ -18,44 +18,54 @@ constexpr int kRouteThreads = 1024;
 constexpr int kRouteChunk = 8192;
 constexpr int kRouteMaxE = 1024;
 
-// Per-warp histogram of the warp's sub-chunk [f0, f1).  hist row = this warp's E counters.
-__device__ void warp_histogram(const int32_t* __restrict__ ids, int f0, int f1, int E, int* hist,
-                               int* status) {
+// A warp's sub-chunk holds at most kRouteChunk / 32 = 256 flat indices: eight per lane, loaded
+// once into registers (all loads in flight together) and reused by both passes.
+constexpr int kPerLane = kRouteChunk / (32 * 32);
+
+__device__ __forceinline__ void warp_load_ids(const int32_t* __restrict__ ids, int f0, int f1, int E,
+                                              int x[kPerLane], int* status) {
   const int lane = threadIdx.x & 31;
-  for (int base = f0; base < f1; base += 32) {
-    const int f = base + lane;
-    int x = -1;
-    if (f < f1) {
-      x = __ldg(ids + f);
-      if (x < 0 || x >= E) { set_status(status, GSG_ERR_BAD_ROUTING); x = -1; }
-    }
-    const unsigned mask = __match_any_sync(0xffffffffu, x);
-    if (x >= 0 && lane == __ffs(mask) - 1) hist[x] += __popc(mask);
+  bool bad = false;
+#pragma unroll
+  for (int i = 0; i < kPerLane; ++i) {
+    const int f = f0 + 32 * i + lane;
+    x[i] = f < f1 ? __ldg(ids + f) : -1;
+  }
+#pragma unroll
+  for (int i = 0; i < kPerLane; ++i) {
+    const int f = f0 + 32 * i + lane;
+    if (f < f1 && (x[i] < 0 || x[i] >= E)) { bad = true; x[i] = -1; }
+  }
+  if (bad && status != nullptr) set_status(status, GSG_ERR_BAD_ROUTING);
+}
+
+// Per-warp histogram of the warp's ids.  hist row = this warp's E counters.
+__device__ __forceinline__ void warp_histogram(const int x[kPerLane], int* hist) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int i = 0; i < kPerLane; ++i) {
+    const unsigned mask = __match_any_sync(0xffffffffu, x[i]);
+    if (x[i] >= 0 && lane == __ffs(mask) - 1) hist[x[i]] += __popc(mask);
     __syncwarp();
   }
 }
 
-// Stable scatter of the warp's sub-chunk; base[x] = first row of id x for this warp (advanced).
-__device__ void warp_scatter(const int32_t* __restrict__ ids, int f0, int f1, int E, int* base,
-                             int32_t* perm_src, int32_t* inv_perm) {
+// Stable scatter of the warp's ids; base[x] = first row of id x for this warp (advanced).
+__device__ __forceinline__ void warp_scatter(const int x[kPerLane], int f0, int* base, int32_t* perm_src,
+                                             int32_t* inv_perm) {
   const int lane = threadIdx.x & 31;
   const unsigned lt = (1u << lane) - 1u;
-  for (int b = f0; b < f1; b += 32) {
-    const int f = b + lane;
-    int x = -1;
-    if (f < f1) {
-      x = __ldg(ids + f);
-      if (x < 0 || x >= E) x = -1;
-    }
-    const unsigned mask = __match_any_sync(0xffffffffu, x);
-    int pos = 0;
-    if (x >= 0) {
-      pos = base[x] + __popc(mask & lt);
+#pragma unroll
+  for (int i = 0; i < kPerLane; ++i) {
+    const int f = f0 + 32 * i + lane;
+    const unsigned mask = __match_any_sync(0xffffffffu, x[i]);
+    if (x[i] >= 0) {
+      const int pos = base[x[i]] + __popc(mask & lt);
       perm_src[pos] = f;
       inv_perm[f] = pos;
     }
     __syncwarp();
-    if (x >= 0 && lane == __ffs(mask) - 1) base[x] += __popc(mask);
+    if (x[i] >= 0 && lane == __ffs(mask) - 1) base[x[i]] += __popc(mask);
     __syncwarp();
   }
 }
@@ -106,25 +116,27 @@ route_single_kernel(const int32_t* __restrict__ ids, int R, int E, int32_t* off,
   const int warp = threadIdx.x >> 5;
   int f0, f1;
   sub_chunk(0, R, f0, f1);
-  warp_histogram(ids, f0, f1, E, hist + warp * E, status);
+  int x[kPerLane];
+  warp_load_ids(ids, f0, f1, E, x, status);
+  warp_histogram(x, hist + warp * E);
   __syncthreads();
-  const int x = threadIdx.x;
+  const int ex = threadIdx.x;
   int tot = 0;
-  if (x < E)
-    for (int w = 0; w < 32; ++w) tot += hist[w * E + x];
+  if (ex < E)
+    for (int w = 0; w < 32; ++w) tot += hist[w * E + ex];
   const int start = block_exclusive_scan(tot, warp_sums, &total);
-  if (x < E) {
-    off[x] = start;
+  if (ex < E) {
+    off[ex] = start;
     int run = start;
     for (int w = 0; w < 32; ++w) {
-      int c = hist[w * E + x];
-      hist[w * E + x] = run;
+      int c = hist[w * E + ex];
+      hist[w * E + ex] = run;
       run += c;
     }
   }
-  if (x == 0) off[E] = total;
+  if (ex == 0) off[E] = total;
   __syncthreads();
-  warp_scatter(ids, f0, f1, E, hist + warp * E, perm_src, inv_perm);
+  warp_scatter(x, f0, hist + warp * E, perm_src, inv_perm);
 }
 
 // Multi-chunk path, launch 1: per-chunk histograms -> ws_hist[chunk][E].
@@ -136,7 +148,9 @@ route_hist_kernel(const int32_t* __restrict__ ids, int R, int E, int* ws_hist, i
   const int c0 = blockIdx.x * kRouteChunk, c1 = min(c0 + kRouteChunk, R);
   int f0, f1;
   sub_chunk(c0, c1, f0, f1);
-  warp_histogram(ids, f0, f1, E, hist + (threadIdx.x >> 5) * E, status);
+  int x[kPerLane];
+  warp_load_ids(ids, f0, f1, E, x, status);
+  warp_histogram(x, hist + (threadIdx.x >> 5) * E);
   __syncthreads();
   for (int x = threadIdx.x; x < E; x += blockDim.x) {
     int s = 0;
@@ -178,7 +192,9 @@ route_scatter_kernel(const int32_t* __restrict__ ids, int R, int E, const int* w
   int f0, f1;
   sub_chunk(c0, c1, f0, f1);
   const int warp = threadIdx.x >> 5;
-  warp_histogram(ids, f0, f1, E, hist + warp * E, nullptr);
+  int x[kPerLane];
+  warp_load_ids(ids, f0, f1, E, x, nullptr);
+  warp_histogram(x, hist + warp * E);
   __syncthreads();
   for (int x = threadIdx.x; x < E; x += blockDim.x) {
     int run = ws_base[(size_t)blockIdx.x * E + x];
@@ -189,7 +205,7 @@ route_scatter_kernel(const int32_t* __restrict__ ids, int R, int E, const int* w
     }
   }
   __syncthreads();
-  warp_scatter(ids, f0, f1, E, hist + warp * E, perm_src, inv_perm);
+  warp_scatter(x, f0, hist + warp * E, perm_src, inv_perm);
 }
 
 int route_chunks(int R) { return R <= kRouteChunk ? 1 : (R + kRouteChunk - 1) / kRouteChunk; }

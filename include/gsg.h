@@ -126,6 +126,7 @@ gsg_status_t gsg_moe_route_permute(const int32_t* topk_ids, int T, int k, int E,
  * as the weights) and written to each of its k routed rows inv_perm[t*k + j]
  * (inv_perm NULL: row t, and k must be 1).  sf_block: 32 (sparse GEMM) or 16 (dense control).
  * Outputs: codes [R][K/2], scales in the quad layout above (R = T*k), x_tensor_scale_out fp32[1].
+ * Limits: T*k <= 2^30 and T*K/16 < 2^31, else GSG_ERR_UNSUPPORTED_SHAPE.
  */
 gsg_status_t gsg_quantize_act_nvfp4(const uint16_t* X, int T, int K, int sf_block,
                                     const int32_t* inv_perm, int k,
