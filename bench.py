@@ -99,6 +99,12 @@ class ClockSampler:
                                        "-i", str(gpu_index), "-lms", "50"], stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.p = None
+        # the first query initialises NVML and can stall the device briefly: wait for it to land
+        # before the timed region starts
+        t0 = time.time()
+        while self.p is not None and time.time() - t0 < 10.0 and os.path.getsize(self.f.name) == 0:
+            time.sleep(0.05)
+        time.sleep(0.2)
 
     def stop(self):
         if self.p is None:
