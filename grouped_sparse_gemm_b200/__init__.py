@@ -23,7 +23,8 @@ from . import _build
 __all__ = [
     "GsgError", "lib", "load_library", "library_path",
     "PackedSparseWeights", "PackedDenseWeights", "Routing", "QuantizedActivations",
-    "pack_sparse_nvfp4", "pack_dense_nvfp4", "moe_route_permute", "quantize_act_nvfp4",
+    "pack_sparse_nvfp4", "pack_dense_nvfp4", "moe_route_permute", "moe_route_permute_noalloc",
+    "quantize_act_nvfp4",
     "grouped_sparse_gemm", "grouped_dense_gemm", "unpermute_scale", "get_device_status",
     "act_scales_bytes", "workspace_size", "OP_PACK_SPARSE", "OP_PACK_DENSE", "OP_ROUTE",
     "OP_QUANTIZE", "OP_GEMM", "EXPORTED_SYMBOLS",
@@ -39,6 +40,7 @@ EXPORTED_SYMBOLS = [
     "gsg_pack_sparse_nvfp4", "gsg_pack_dense_nvfp4", "gsg_moe_route_permute",
     "gsg_quantize_act_nvfp4", "gsg_grouped_sparse_gemm", "gsg_grouped_dense_gemm",
     "gsg_unpermute_scale", "gsg_get_device_status", "gsg_status_string", "gsg_version",
+    "gsg_moe_route_permute_noalloc",
 ]
 
 _STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported shape", -3: "CUDA error",
@@ -86,6 +88,7 @@ def load_library(build_if_missing: bool = False) -> ctypes.CDLL:
         "gsg_get_device_status": (i, [vp]),
         "gsg_status_string": (ctypes.c_char_p, [i]),
         "gsg_version": (i, []),
+        "gsg_moe_route_permute_noalloc": (i, [vp, i, i, i, vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -249,6 +252,18 @@ def moe_route_permute(topk_ids: torch.Tensor, E: int, out: Optional[Routing] = N
     _check("gsg_moe_route_permute", lib().gsg_moe_route_permute(
         _ptr(topk_ids), T, k, E, _ptr(out.offsets), _ptr(out.perm_src), _ptr(out.inv_perm),
         _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+    return out
+
+
+def moe_route_permute_noalloc(topk_ids: torch.Tensor, E: int, out: Routing, stream=None) -> Routing:
+    """gsg_moe_route_permute_noalloc: the same routing with the library's fixed scratch instead of
+    a workspace, for callers that may not allocate device memory at this point (outputs in `out`
+    are caller-allocated; nothing is allocated here)."""
+    _need_cuda(topk_ids, out.offsets, out.perm_src, out.inv_perm)
+    assert topk_ids.dtype == torch.int32 and topk_ids.dim() == 2
+    T, k = topk_ids.shape
+    _check("gsg_moe_route_permute_noalloc", lib().gsg_moe_route_permute_noalloc(
+        _ptr(topk_ids), T, k, E, _ptr(out.offsets), _ptr(out.perm_src), _ptr(out.inv_perm), _stream(stream)))
     return out
 
 

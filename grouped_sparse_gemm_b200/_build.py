@@ -10,7 +10,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libgsg.so")
-SOURCES = ["gsg_api.cu", "gsg_pack.cu", "gsg_quant.cu", "gsg_route.cu", "gsg_unpermute.cu", "gsg_gemm.cu"]
+SOURCES = ["gsg_api.cu", "gsg_pack.cu", "gsg_quant.cu", "gsg_route.cu", "gsg_unpermute.cu", "gsg_gemm.cu",
+           "gsg_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -55,6 +55,18 @@ bool weight_shape_ok(int E, int N, int K) {
 
 }  // namespace
 
+namespace gsg {
+// The library's per-device set-up and status word, for entry points defined in other files.
+gsg_status_t device_setup(int** status, int* num_sms) {
+  DeviceState* d = nullptr;
+  gsg_status_t st = device_state(&d);
+  if (st != GSG_OK) return st;
+  *status = d->status;
+  *num_sms = d->num_sms;
+  return GSG_OK;
+}
+}  // namespace gsg
+
 extern "C" {
 
 size_t gsg_sparse_packed_bytes(int E, int N, int K) {

@@ -5,7 +5,12 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include "gsg.h"
+
 namespace gsg {
+
+// gsg_api.cu: per-device set-up (first call on a device), device status word and SM count
+gsg_status_t device_setup(int** status, int* num_sms);
 
 // gsg_pack.cu
 int pack_partials_per_expert(int N, int K);

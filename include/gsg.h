@@ -174,6 +174,27 @@ gsg_status_t gsg_unpermute_scale(const uint16_t* Y, const int32_t* inv_perm, con
                                  int T, int k, int N, uint16_t* out, void* stream);
 
 /* ----------------------------------------------------------------------------------------
+ * gsg_moe_route_permute_noalloc -- gsg_moe_route_permute for callers that cannot allocate.
+ * The paper has no counterpart: this is a library convenience, not a step of the method.
+ * Who needs it: code that may not call cudaMalloc or any allocating routine when it routes
+ * tokens (its device memory is owned and pre-carved by another component, or it must not grow
+ * its footprint after start-up), so it cannot supply the routing workspace.  Same inputs,
+ * outputs, result and errors as gsg_moe_route_permute; the workspace is replaced by a fixed
+ * 256 KiB device array inside the library, which every GPU that loads the library holds until
+ * the process exits.  The call allocates nothing.
+ * Limit: R = T*k <= 8192 needs no scratch; above that ceil(R/8192) * E <= 32768
+ * (E = 384: R <= 696,320; E = 128: R <= 2,097,152), else GSG_ERR_UNSUPPORTED_SHAPE with no
+ * launch.  The first call on a device sets up that device (the library's per-device set-up and
+ * the scratch's device address); make that first call before any stream capture begins.
+ * All calls on a device share the one array and it keeps the last call's contents (nothing in
+ * it needs to start at zero); calls whose launches overlap on the GPU (unordered streams) race
+ * on it and must be serialised by the caller.
+ */
+gsg_status_t gsg_moe_route_permute_noalloc(const int32_t* topk_ids, int T, int k, int E,
+                                           int32_t* expert_offsets, int32_t* perm_src,
+                                           int32_t* inv_perm, void* stream);
+
+/* ----------------------------------------------------------------------------------------
  * Status.  gsg_get_device_status synchronizes `stream`, returns the device status word of the
  * current device and clears it.  gsg_status_string never returns NULL.
  */
