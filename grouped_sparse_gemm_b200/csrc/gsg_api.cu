@@ -147,7 +147,7 @@ gsg_status_t gsg_quantize_act_nvfp4(const uint16_t* X, int T, int K, int sf_bloc
   if (T < 0 || k < 1 || (sf_block != 16 && sf_block != 32)) return GSG_ERR_INVALID_ARG;
   if (K < 256 || K % 256 != 0) return GSG_ERR_UNSUPPORTED_SHAPE;
   if ((long long)T * k > (1ll << 30)) return GSG_ERR_UNSUPPORTED_SHAPE;
-  if ((long long)T * (K / 16) >= (1ll << 31)) return GSG_ERR_UNSUPPORTED_SHAPE;  // 32-bit unit index
+  if ((long long)T * (K / 8) >= (1ll << 31)) return GSG_ERR_UNSUPPORTED_SHAPE;  // 32-bit unit index
   if (inv_perm == nullptr && k != 1) return GSG_ERR_INVALID_ARG;
   if (!scales || !x_tensor_scale_out) return GSG_ERR_INVALID_ARG;
   if (T > 0 && (!X || !codes)) return GSG_ERR_INVALID_ARG;
@@ -202,6 +202,7 @@ gsg_status_t gsg_unpermute_scale(const uint16_t* Y, const int32_t* inv_perm, con
                                  uint16_t* out, void* stream) {
   if (T < 0 || k < 1 || N < 8 || N % 8 != 0) return GSG_ERR_INVALID_ARG;
   if ((long long)T * k > (1ll << 30)) return GSG_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)T * (N / 8) >= (1ll << 31)) return GSG_ERR_UNSUPPORTED_SHAPE;
   if (T == 0) return GSG_OK;
   if (!Y || !inv_perm || !gates || !out) return GSG_ERR_INVALID_ARG;
   if (!aligned16(Y) || !aligned16(out)) return GSG_ERR_INVALID_ARG;

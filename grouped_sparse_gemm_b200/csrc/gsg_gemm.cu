@@ -255,7 +255,7 @@ template <bool kSparse, int kBN>
 struct Geo {
   static constexpr int kKbLogical = kSparse ? 128 : 64;            // logical K per MMA
   static constexpr int kKbPerChunk = kChunkK / kKbLogical;         // 2 sparse, 4 dense
-  static constexpr int kCPS = (kSparse ? kBN <= 64 : kBN <= 32) ? 2 : 1;   // 256-wide chunks per stage
+  static constexpr int kCPS = (kSparse || kBN <= 32) ? 2 : 1;     // 256-wide chunks per stage
   static constexpr int kKbps = kCPS * kKbPerChunk;                 // MMAs per stage
   static constexpr int kCB = kSparse ? kSparseChunkBytes : kDenseChunkBytes;   // packed chunk block
   static constexpr int kCBMeta = 8192;                             // metadata offset in a chunk block
@@ -464,14 +464,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
     }
   } else if (warp == 1) {
     // =============================== MMA issuer (whole warp, one elected lane issues)
-    int s = 0, set = 0, i = 0, it = 0;
-    uint32_t ph = 0;
+    int s = 0, set = 0, i = 0, acc = 0;
+    uint32_t ph = 0, aph = 0;   // ring phase, accumulator phase
     bool any = false;
-    for (int j = 0; j < n_my && !*abort_flag; ++j, ++it) {
+    for (int j = 0; j < n_my && !*abort_flag; ++j) {
       const TileDesc c = my_tile(j, ttab, p.tcap, pref, offs, E, kBN);
       const uint32_t idesc = make_idesc(kSparse, (c.valid + 15) & ~15);
-      const int acc = it % NACC;
-      if (!wait_warp(acce_bar(acc), ((uint32_t)(it / NACC) & 1u) ^ 1u, abort_flag, p.status)) break;
+      if (!wait_warp(acce_bar(acc), aph ^ 1u, abort_flag, p.status)) break;
       tc_fence_after();
       const uint32_t d_tmem = tmem + kColAcc + (uint32_t)(acc * G::kAccStride);
       bool ok = true;
@@ -511,6 +510,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
       }
       if (!ok) break;
       tc_commit(accf_bar(acc));
+      if (++acc == NACC) { acc = 0; aph ^= 1u; }
     }
     __syncwarp();
     if (any) {
@@ -524,12 +524,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
     // =============================== epilogue (warps 3..6 -> TMEM lane quadrants 3,0,1,2)
     const int q = warp & 3;
     const float sx = __ldg(p.x_scale);
-    int it = 0;
-    for (int j = 0; j < n_my; ++j, ++it) {
+    int acc = 0;
+    uint32_t aph = 0;
+    for (int j = 0; j < n_my; ++j) {
       const TileDesc c = my_tile(j, ttab, p.tcap, pref, offs, E, kBN);
       const int r0 = c.r0, valid = c.valid;
-      const int acc = it % NACC;
-      if (!wait_warp(accf_bar(acc), (uint32_t)(it / NACC) & 1u, abort_flag, p.status)) break;
+      if (!wait_warp(accf_bar(acc), aph, abort_flag, p.status)) break;
       tc_fence_after();
       const float scale = __fmul_rn(sx, wsc[c.e]);
       const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + kColAcc + (uint32_t)(acc * G::kAccStride);
@@ -580,6 +580,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acce_bar(acc));
+      if (++acc == NACC) { acc = 0; aph ^= 1u; }
     }
   }
 
@@ -598,7 +599,10 @@ struct GemmPlan {
   size_t smem;
 };
 
-constexpr int kSmemBudget = 192 * 1024;
+constexpr int kMaxStages = 12;
+constexpr int kStageBudget128 = 192 * 1024;   // 128-token tiles: a deeper ring only adds L2 pressure
+// opt-in dynamic shared memory per block minus room for static shared memory (set per device)
+static int g_smem_limit = 232448 - 1024;
 
 // tcap: capacity of the per-CTA tile table (tiles beyond it are decoded on the fly); an upper
 // bound on a CTA's tiles is ceil((ceil(R/BN) + E) * NT / grid).
@@ -606,12 +610,17 @@ static GemmPlan make_plan(bool sparse, int BN, int E, int tcap) {
   GemmPlan g;
   g.BN = BN;
   g.tcap = tcap;
-  g.cps = (sparse ? BN <= 64 : BN <= 32) ? 2 : 1;
+  g.cps = (sparse || BN <= 32) ? 2 : 1;
   const int kbps = g.cps * (sparse ? 2 : 4);
   const int body = g.cps * BN * 128 + g.cps * (sparse ? kSparseChunkBytes : kDenseChunkBytes) + kbps * 512;
   g.stage = (body + 1023) / 1024 * 1024;
-  g.stages = (kSmemBudget - tcap * 16) / g.stage;
-  if (g.stages > 12) g.stages = 12;
+  // everything but the stage ring and the tile table, at its largest
+  const int fixed = 1024 + (2 * kMaxStages + kNSets + 2 * kMaxAcc + 1) * 8 + (int)sizeof(Ctl) + (3 * E + 2) * 4 +
+                    16 + 4 * kOutStageBytes;
+  int budget = g_smem_limit - fixed;
+  if (BN == 128 && budget > kStageBudget128) budget = kStageBudget128;
+  g.stages = (budget - tcap * 16) / g.stage;
+  if (g.stages > kMaxStages) g.stages = kMaxStages;
   const int acc_stride = BN < 32 ? 32 : BN;
   g.nacc = (int)((kTmemCols - kColAcc) / acc_stride);
   if (g.nacc > kMaxAcc) g.nacc = kMaxAcc;
@@ -623,12 +632,14 @@ static GemmPlan make_plan(bool sparse, int BN, int E, int tcap) {
 
 constexpr int kMaxTableTiles = 1024;
 
-int gemm_pick_bn(int max_rows) {
-  if (max_rows <= 0) return 128;
-  if (max_rows <= 16) return 16;
-  if (max_rows <= 32) return 32;
-  if (max_rows <= 64) return 64;
-  return 128;
+// Token tile: the smallest of 16/32/64 that holds the largest expert; past 64 rows, 128 only when
+// experts average at least 64 rows (R / E), since a 128-row activation chunk takes shared memory
+// from the weight ring that the many small experts of a skewed routing would leave unused.
+int gemm_pick_bn(int max_rows, int R, int E) {
+  if (max_rows > 0 && max_rows <= 16) return 16;
+  if (max_rows > 0 && max_rows <= 32) return 32;
+  if (max_rows > 0 && max_rows <= 64) return 64;
+  return (long long)R >= 64ll * E ? 128 : 64;
 }
 
 bool gemm_supported(int E) { return E >= 1 && E <= kMaxE; }
@@ -655,12 +666,13 @@ static cudaError_t set_attr_one(int bytes) {
 }
 
 cudaError_t gemm_set_smem_attrs() {
-  // every plan stays below the opt-in limit (200 KB of stages + at most 16 KB of tile table)
+  // every plan stays below the opt-in limit (make_plan sizes the ring from it)
   int dev = 0, maxb = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&maxb, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   if (e != cudaSuccess) return e;
   maxb -= 1024;   // room for the kernels' static shared memory
+  g_smem_limit = maxb;
   cudaError_t errs[8] = {set_attr_one<true, 16>(maxb),  set_attr_one<true, 32>(maxb),  set_attr_one<true, 64>(maxb),
                          set_attr_one<true, 128>(maxb), set_attr_one<false, 16>(maxb), set_attr_one<false, 32>(maxb),
                          set_attr_one<false, 64>(maxb), set_attr_one<false, 128>(maxb)};
@@ -686,11 +698,12 @@ int launch_gemm(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, co
                 int max_rows, void* Y, int y_f32, int* status, int num_sms, cudaStream_t stream) {
   EncodeTiledFn enc = get_encode_fn();
   if (enc == nullptr) return 2;
-  const int BN = gemm_pick_bn(max_rows);
+  const int BN = gemm_pick_bn(max_rows, R, E);
   const long long bound = (((long long)R + BN - 1) / BN + E) * (N / kTileN);
   long long tcap = (bound + num_sms - 1) / num_sms;
   if (tcap > kMaxTableTiles) tcap = kMaxTableTiles;
   const GemmPlan g = make_plan(sparse, BN, E, (int)tcap);
+  if (g.stages < kNSets || g.smem > (size_t)g_smem_limit) return 1;   // ring too shallow: refuse, launch nothing
   const int box_h = g.BN < 32 ? g.BN : 32;
   const int kbps = g.cps * (sparse ? 2 : 4);
   const int rcap = R + kActScalePadRows;

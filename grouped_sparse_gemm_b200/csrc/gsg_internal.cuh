@@ -60,16 +60,12 @@ __device__ __forceinline__ uint32_t ue4m3_encode(float x) {
 
 // E2M1: magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6}; sign bit 3 copied from the input (-0 -> 0x8).
 __device__ __forceinline__ uint32_t e2m1_encode(float v) {
-  float a = fabsf(v);
-  uint32_t c;
-  if (a <= 0.25f) c = 0u;
-  else if (a < 0.75f) c = 1u;
-  else if (a <= 1.25f) c = 2u;
-  else if (a < 1.75f) c = 3u;
-  else if (a <= 2.5f) c = 4u;
-  else if (a < 3.5f) c = 5u;
-  else if (a <= 5.0f) c = 6u;
-  else c = 7u;
+  const float a = fabsf(v);
+  // code = number of decision thresholds below |v| (strict at the ties that round down to the
+  // even code, inclusive at those that round up); NaN saturates like the largest magnitude
+  uint32_t c = (uint32_t)(a > 0.25f) + (uint32_t)(a >= 0.75f) + (uint32_t)(a > 1.25f) + (uint32_t)(a >= 1.75f) +
+               (uint32_t)(a > 2.5f) + (uint32_t)(a >= 3.5f) + (uint32_t)(a > 5.0f);
+  if (a != a) c = 7u;
   return c | ((__float_as_uint(v) >> 28) & 8u);
 }
 

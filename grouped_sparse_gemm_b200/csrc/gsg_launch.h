@@ -24,7 +24,7 @@ cudaError_t launch_quant(const uint16_t* X, int T, int K, int sf, const int32_t*
                          cudaStream_t stream);
 
 // gsg_route.cu
-int route_chunks(int R);
+int route_chunks(int R, int E);
 size_t route_workspace_bytes(int R, int E);
 bool route_supported(int E);
 cudaError_t route_set_smem_attrs();
@@ -37,7 +37,7 @@ cudaError_t launch_unpermute(const uint16_t* Y, const int32_t* inv_perm, const f
 
 // gsg_gemm.cu
 bool gemm_supported(int E);
-int gemm_pick_bn(int max_rows);
+int gemm_pick_bn(int max_rows, int R, int E);
 cudaError_t gemm_set_smem_attrs();
 int launch_gemm(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, const float* x_scale,
                 const uint8_t* w_packed, const float* w_scale, const int32_t* off, int E, int N, int K, int R,

@@ -15,10 +15,11 @@
 // device address comes from cudaGetSymbolAddress, taken once per device (with that device
 // current) by the entry point's first call on that device.
 //
-// Limits: R <= 8192 uses no scratch.  Above that, the multi-chunk routing needs
-// 2 * ceil(R / 8192) * E int32 of scratch, so ceil(R / 8192) * E <= 32768 (E = 384: R up to
-// 696,320 rows; E = 128: R up to 2,097,152).  Larger requests return GSG_ERR_UNSUPPORTED_SHAPE
-// before anything is launched.
+// Limits: R <= 1024 uses no scratch.  Above that the routing needs the workspace that
+// gsg_workspace_size(GSG_OP_ROUTE, ...) reports: at most 128 KiB while it cuts R into 1024-row
+// chunks, else 2 * ceil(R / 8192) * E int32.  So a call is accepted when ceil(R / 8192) * E <=
+// 32768 (E = 384: R up to 696,320 rows; E = 128: R up to 2,097,152); larger requests return
+// GSG_ERR_UNSUPPORTED_SHAPE before anything is launched.
 //
 // Sharing: every call on a device uses the same array, which keeps the last call's contents.
 // Nothing in it has to start at zero: the histogram launch writes every [chunk][expert] count

@@ -7,10 +7,10 @@
 //
 // Launch 1 (skipped when the caller supplies s_x): partial max|X| per block, 128-bit loads,
 // warp-shuffle reductions.  Launch 2: every block folds the partials into s_x = amax/2688,
-// then each thread quantizes 16 consecutive elements of one token row (two 128-bit loads),
-// pairs of lanes combine their maxima into the 32-element block amax, eight lanes assemble
-// the four scales of one MMA k-block into a 32-bit word, and the token's codes and scale
-// words are written to each of its k routed rows (the dispatch).  The same launch zero-fills
+// then each thread quantizes 8 consecutive elements of one token row (one 128-bit load),
+// groups of 4 lanes (2 for 16-element blocks) combine their maxima into the block amax, the
+// four scales of one MMA k-block are gathered into a 32-bit word, and the token's codes and
+// scale words are written to each of its k routed rows (the dispatch).  The same launch zero-fills
 // the padding entries of the quad scale layout.
 #include "gsg_internal.cuh"
 
@@ -26,15 +26,24 @@ act_amax_kernel(const uint16_t* __restrict__ X, long long n8, float* __restrict_
   float mx = 0.0f;
   bool finite = true;
   const uint4* X4 = reinterpret_cast<const uint4*>(X);
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
-       i += (long long)gridDim.x * blockDim.x) {
-    uint4 v = __ldg(X4 + i);
-    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  // four independent 128-bit loads in flight per thread and round
+  for (long long i0 = (long long)blockIdx.x * blockDim.x + threadIdx.x; i0 < n8; i0 += 4 * stride) {
+    uint4 v[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      uint32_t lo = w[j] & 0xFFFFu, hi = w[j] >> 16;
-      finite &= ((lo & 0x7F80u) != 0x7F80u) && ((hi & 0x7F80u) != 0x7F80u);
-      mx = fmaxf(mx, fmaxf(fabsf(bf16_bits_to_f32(lo)), fabsf(bf16_bits_to_f32(hi))));
+    for (int u = 0; u < 4; ++u) {
+      const long long i = i0 + u * stride;
+      v[u] = i < n8 ? __ldg(X4 + i) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t lo = w[j] & 0xFFFFu, hi = w[j] >> 16;
+        finite &= ((lo & 0x7F80u) != 0x7F80u) && ((hi & 0x7F80u) != 0x7F80u);
+        mx = fmaxf(mx, fmaxf(fabsf(bf16_bits_to_f32(lo)), fabsf(bf16_bits_to_f32(hi))));
+      }
     }
   }
   if (!finite) set_status(status, GSG_ERR_NONFINITE);
@@ -86,57 +95,52 @@ act_quant_kernel(QuantParams p) {
   const float six_s = __fmul_rn(6.0f, s);
 
   const int lane = threadIdx.x & 31;
-  const int units_per_row = p.K / 16;
+  const int units_per_row = p.K / 8;
   const long long U = (long long)p.T * units_per_row;
   const int KBa = p.K / (4 * p.sf);
   const int gwarp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int nwarps = (gridDim.x * blockDim.x) >> 5;
-  // ---- main: warp-uniform loop so that the lane shuffles below always see the full warp
+  // ---- main: each lane quantizes 8 consecutive elements; a warp covers 256 elements of one row
+  // (K % 256 == 0), so a 32-element block is 4 lanes (16-element block: 2 lanes) and one MMA
+  // k-block's four scales sit in 16 lanes (8).  The loop is warp-uniform so the shuffles see the
+  // full warp.
   for (long long base = (long long)gwarp * 32; base < U; base += (long long)nwarps * 32) {
     const long long unit = base + lane;
     const bool valid = unit < U;
-    const unsigned u32 = (unsigned)unit;   // U = T*K/16 < 2^31 is checked on the host
+    const unsigned u32 = (unsigned)unit;   // U = T*K/8 < 2^31 is checked on the host
     const int t = valid ? int(u32 / (unsigned)units_per_row) : 0;
-    const int c16 = valid ? int(u32 % (unsigned)units_per_row) : 0;
-    float x[16];
+    const int c8 = valid ? int(u32 % (unsigned)units_per_row) : 0;
+    float x[8];
     float amax = 0.0f;
     if (valid) {
-      const uint4* src = reinterpret_cast<const uint4*>(p.X + (size_t)t * p.K + (size_t)c16 * 16);
-      uint4 a = __ldg(src), b = __ldg(src + 1);
-      uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+      const uint4 a = __ldg(reinterpret_cast<const uint4*>(p.X + (size_t)t * p.K + (size_t)c8 * 8));
+      const uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
+      for (int j = 0; j < 4; ++j) {
         x[2 * j] = bf16_bits_to_f32(w[j] & 0xFFFFu);
         x[2 * j + 1] = bf16_bits_to_f32(w[j] >> 16);
       }
 #pragma unroll
-      for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(x[j]));
+      for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(x[j]));
     } else {
 #pragma unroll
-      for (int j = 0; j < 16; ++j) x[j] = 0.0f;
+      for (int j = 0; j < 8; ++j) x[j] = 0.0f;
     }
-    if (p.sf == 32) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    if (p.sf == 32) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
     const BlockScale bs = block_scale(amax, six_s, s);
-    uint64_t codes = 0;
+    uint32_t codes = 0;
 #pragma unroll
-    for (int j = 0; j < 16; ++j) codes |= uint64_t(e2m1_encode(__fmul_rn(x[j], bs.inv))) << (4 * j);
-    // four scales of one MMA k-block -> one 32-bit word (sf 32: lanes g, g+2, g+4, g+6; sf 16: g..g+3)
-    uint32_t word;
-    int kb;
-    bool writer;
-    if (p.sf == 32) {
-      const int g = lane & ~7;
-      word = __shfl_sync(0xffffffffu, bs.sc, g) | (__shfl_sync(0xffffffffu, bs.sc, g + 2) << 8) |
-             (__shfl_sync(0xffffffffu, bs.sc, g + 4) << 16) | (__shfl_sync(0xffffffffu, bs.sc, g + 6) << 24);
-      kb = c16 >> 3;
-      writer = (lane & 7) == 0;
-    } else {
-      const int g = lane & ~3;
-      word = __shfl_sync(0xffffffffu, bs.sc, g) | (__shfl_sync(0xffffffffu, bs.sc, g + 1) << 8) |
-             (__shfl_sync(0xffffffffu, bs.sc, g + 2) << 16) | (__shfl_sync(0xffffffffu, bs.sc, g + 3) << 24);
-      kb = c16 >> 2;
-      writer = (lane & 3) == 0;
-    }
+    for (int j = 0; j < 8; ++j) codes |= e2m1_encode(__fmul_rn(x[j], bs.inv)) << (4 * j);
+    // four scales of one MMA k-block -> one 32-bit word (sf 32: lanes g, g+4, g+8, g+12;
+    // sf 16: g, g+2, g+4, g+6)
+    const int step = p.sf == 32 ? 4 : 2;
+    const int g = lane & ~(4 * step - 1);
+    const uint32_t word = __shfl_sync(0xffffffffu, bs.sc, g) | (__shfl_sync(0xffffffffu, bs.sc, g + step) << 8) |
+                          (__shfl_sync(0xffffffffu, bs.sc, g + 2 * step) << 16) |
+                          (__shfl_sync(0xffffffffu, bs.sc, g + 3 * step) << 24);
+    const int kb = p.sf == 32 ? (c8 >> 4) : (c8 >> 3);
+    const bool writer = (lane & (4 * step - 1)) == 0;
     if (!valid) continue;
     // the token's destination rows, all loaded before any store (up to 16 at a time)
     for (int j0 = 0; j0 < p.k; j0 += 16) {
@@ -149,7 +153,7 @@ act_quant_kernel(QuantParams p) {
         if (j0 + j >= p.k) break;
         const int row = rows[j];
         if (row < 0 || row >= p.R) { set_status(p.status, GSG_ERR_BAD_ROUTING); continue; }
-        *reinterpret_cast<uint64_t*>(p.codes + (size_t)row * (p.K / 2) + (size_t)c16 * 8) = codes;
+        *reinterpret_cast<uint32_t*>(p.codes + (size_t)row * (p.K / 2) + (size_t)c8 * 4) = codes;
         if (writer) {
           uint32_t* sw = reinterpret_cast<uint32_t*>(p.scales);
 #pragma unroll
@@ -163,14 +167,14 @@ act_quant_kernel(QuantParams p) {
   }
   // ---- zero the quad entries that refer to rows >= R
   const int r_lo = p.R > 96 ? p.R - 96 : 0;
-  const long long npad = (long long)KBa * (p.rcap - r_lo) * 4;
+  const int span = p.rcap - r_lo;                 // at most 352 rows
+  const int npad = KBa * span * 4;                // K / 128 * 352 * 4 < 2^31
   uint32_t* sw = reinterpret_cast<uint32_t*>(p.scales);
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < npad;
-       i += (long long)gridDim.x * blockDim.x) {
-    const int c = int(i & 3);
-    const long long rest = i >> 2;
-    const int rr = r_lo + int(rest % (p.rcap - r_lo));
-    const int kb = int(rest / (p.rcap - r_lo));
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < npad; i += gridDim.x * blockDim.x) {
+    const int c = i & 3;
+    const int rest = i >> 2;
+    const int rr = r_lo + rest % span;
+    const int kb = rest / span;
     if (rr + 32 * c >= p.R) sw[((size_t)kb * p.rcap + rr) * 4 + c] = 0u;
   }
 }
@@ -198,7 +202,7 @@ cudaError_t launch_quant(const uint16_t* X, int T, int K, int sf, const int32_t*
   p.X = X; p.inv_perm = inv_perm; p.s_in = s_in; p.partial = partial; p.nparts = P;
   p.T = T; p.K = K; p.sf = sf; p.k = k; p.R = T * k; p.rcap = T * k + kActScalePadRows;
   p.codes = codes; p.scales = scales; p.s_out = s_out; p.status = status;
-  const long long units = (long long)T * (K / 16);
+  const long long units = (long long)T * (K / 8);
   long long blocks = (units + kQuantThreads - 1) / kQuantThreads;
   if (blocks < 1) blocks = 1;
   if (blocks > (long long)num_sms * 8) blocks = (long long)num_sms * 8;

@@ -5,67 +5,90 @@
 // expert problems with different token counts together; §D.1 (p.19) -- dispatch/scatter.
 //
 // Routed pair (t, j) has flat index f = t*k + j; rows of expert e are [off[e], off[e+1]) in
-// ascending f.  Work is split into chunks of kRouteChunk flat indices, one 1024-thread block per
-// chunk and 32 sub-chunks (one per warp).  Within a warp, equal ids are ranked with
-// __match_any_sync; per-warp histograms live in shared memory (32 x E ints).  A single chunk
-// (R <= kRouteChunk) runs as one launch; larger R uses histogram -> scan -> scatter launches
-// with a [chunks x E] workspace.  The result is deterministic.
+// ascending f.  The flat indices are cut into chunks, one 1024-thread block per chunk: 1024
+// indices (one per thread) while ceil(R/1024) * E <= 16384 (a workspace of at most 128 KiB),
+// else 8192 (eight per thread).  Each warp owns a contiguous run of its chunk; lanes holding
+// the same id are found with one ballot per id bit, which gives each index its rank among equal
+// ids of its warp, and per-warp histograms live in shared memory (32 x E ints).  R <= 1024 is one launch; larger R is histogram -> scan -> scatter
+// over a [chunks x E] workspace.  Only integer arithmetic: the result is deterministic.
 #include "gsg_internal.cuh"
 
 namespace gsg {
 
 constexpr int kRouteThreads = 1024;
-constexpr int kRouteChunk = 8192;
 constexpr int kRouteMaxE = 1024;
+constexpr long long kSmallChunkMaxCells = 16384;   // chunks x experts of the 1024-index path
 
-// A warp's sub-chunk holds at most kRouteChunk / 32 = 256 flat indices: eight per lane, loaded
-// once into registers (all loads in flight together) and reused by both passes.
-constexpr int kPerLane = kRouteChunk / (32 * 32);
+int route_chunk_size(int R, int E) {
+  return ((long long)(R + 1023) / 1024) * E <= kSmallChunkMaxCells ? 1024 : 8192;
+}
 
+// Lanes of the warp holding the same key as this lane: one ballot per key bit (key = id + 1,
+// so the invalid id -1 is key 0 and needs no special case).  nbits = bit length of E.
+__device__ __forceinline__ unsigned peer_mask(int x, int nbits) {
+  const unsigned key = (unsigned)(x + 1);
+  unsigned m = 0xffffffffu;
+  for (int b = 0; b < nbits; ++b) {
+    const unsigned bit = (key >> b) & 1u;
+    const unsigned bal = __ballot_sync(0xffffffffu, bit);
+    m &= bit ? bal : ~bal;
+  }
+  return m;
+}
+
+__device__ __forceinline__ int key_bits(int E) { return 32 - __clz(E); }
+
+// The ids of this warp's run [f0, f1): kPer per lane, index f0 + 32*i + lane (-1 past the end or
+// out of range; an out-of-range id also records GSG_ERR_BAD_ROUTING when status is given).
+template <int kPer>
 __device__ __forceinline__ void warp_load_ids(const int32_t* __restrict__ ids, int f0, int f1, int E,
-                                              int x[kPerLane], int* status) {
+                                              int x[kPer], int* status) {
   const int lane = threadIdx.x & 31;
   bool bad = false;
 #pragma unroll
-  for (int i = 0; i < kPerLane; ++i) {
+  for (int i = 0; i < kPer; ++i) {
     const int f = f0 + 32 * i + lane;
     x[i] = f < f1 ? __ldg(ids + f) : -1;
   }
 #pragma unroll
-  for (int i = 0; i < kPerLane; ++i) {
+  for (int i = 0; i < kPer; ++i) {
     const int f = f0 + 32 * i + lane;
     if (f < f1 && (x[i] < 0 || x[i] >= E)) { bad = true; x[i] = -1; }
   }
   if (bad && status != nullptr) set_status(status, GSG_ERR_BAD_ROUTING);
 }
 
-// Per-warp histogram of the warp's ids.  hist row = this warp's E counters.
-__device__ __forceinline__ void warp_histogram(const int x[kPerLane], int* hist) {
+// Peer masks of the warp's ids and the warp's histogram (hist = this warp's E counters).
+template <int kPer>
+__device__ __forceinline__ void warp_histogram(const int x[kPer], unsigned m[kPer], int f0, int f1, int* hist,
+                                               int nbits) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
-  for (int i = 0; i < kPerLane; ++i) {
-    const unsigned mask = __match_any_sync(0xffffffffu, x[i]);
-    if (x[i] >= 0 && lane == __ffs(mask) - 1) hist[x[i]] += __popc(mask);
+  for (int i = 0; i < kPer; ++i) {
+    if (f0 + 32 * i >= f1) break;   // warp-uniform
+    m[i] = peer_mask(x[i], nbits);
+    if (x[i] >= 0 && lane == __ffs(m[i]) - 1) hist[x[i]] += __popc(m[i]);
     __syncwarp();
   }
 }
 
 // Stable scatter of the warp's ids; base[x] = first row of id x for this warp (advanced).
-__device__ __forceinline__ void warp_scatter(const int x[kPerLane], int f0, int* base, int32_t* perm_src,
-                                             int32_t* inv_perm) {
+template <int kPer>
+__device__ __forceinline__ void warp_scatter(const int x[kPer], const unsigned m[kPer], int f0, int f1, int* base,
+                                             int32_t* perm_src, int32_t* inv_perm) {
   const int lane = threadIdx.x & 31;
   const unsigned lt = (1u << lane) - 1u;
 #pragma unroll
-  for (int i = 0; i < kPerLane; ++i) {
+  for (int i = 0; i < kPer; ++i) {
+    if (f0 + 32 * i >= f1) break;   // warp-uniform
     const int f = f0 + 32 * i + lane;
-    const unsigned mask = __match_any_sync(0xffffffffu, x[i]);
     if (x[i] >= 0) {
-      const int pos = base[x[i]] + __popc(mask & lt);
+      const int pos = base[x[i]] + __popc(m[i] & lt);
       perm_src[pos] = f;
       inv_perm[f] = pos;
     }
     __syncwarp();
-    if (x[i] >= 0 && lane == __ffs(mask) - 1) base[x[i]] += __popc(mask);
+    if (x[i] >= 0 && lane == __ffs(m[i]) - 1) base[x[i]] += __popc(m[i]);
     __syncwarp();
   }
 }
@@ -96,15 +119,15 @@ __device__ int block_exclusive_scan(int v, int* warp_sums, int* total) {
   return warp_sums[warp] + incl - v;
 }
 
-__device__ __forceinline__ void sub_chunk(int c0, int c1, int& f0, int& f1) {
-  const int per = ((c1 - c0) + 31) / 32;
+// This warp's run of the chunk [c0, c1): 32*kPer indices starting at c0 + warp*32*kPer.
+template <int kPer>
+__device__ __forceinline__ void warp_run(int c0, int c1, int& f0, int& f1) {
   const int warp = threadIdx.x >> 5;
-  f0 = c0 + warp * per;
-  f1 = min(f0 + per, c1);
-  if (f0 > c1) f0 = c1;
+  f0 = min(c0 + warp * 32 * kPer, c1);
+  f1 = min(f0 + 32 * kPer, c1);
 }
 
-// One chunk holds everything: histogram, scan, scatter in one launch.
+// One chunk holds everything (R <= 1024): histogram, scan, scatter in one launch.
 __global__ void __launch_bounds__(kRouteThreads)
 route_single_kernel(const int32_t* __restrict__ ids, int R, int E, int32_t* off, int32_t* perm_src,
                     int32_t* inv_perm, int* status) {
@@ -112,13 +135,14 @@ route_single_kernel(const int32_t* __restrict__ ids, int R, int E, int32_t* off,
   __shared__ int warp_sums[32];
   __shared__ int total;
   for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) hist[i] = 0;
-  __syncthreads();
   const int warp = threadIdx.x >> 5;
   int f0, f1;
-  sub_chunk(0, R, f0, f1);
-  int x[kPerLane];
-  warp_load_ids(ids, f0, f1, E, x, status);
-  warp_histogram(x, hist + warp * E);
+  warp_run<1>(0, R, f0, f1);
+  int x[1];
+  unsigned m[1];
+  warp_load_ids<1>(ids, f0, f1, E, x, status);
+  __syncthreads();
+  warp_histogram<1>(x, m, f0, f1, hist + warp * E, key_bits(E));
   __syncthreads();
   const int ex = threadIdx.x;
   int tot = 0;
@@ -136,26 +160,28 @@ route_single_kernel(const int32_t* __restrict__ ids, int R, int E, int32_t* off,
   }
   if (ex == 0) off[E] = total;
   __syncthreads();
-  warp_scatter(x, f0, hist + warp * E, perm_src, inv_perm);
+  warp_scatter<1>(x, m, f0, f1, hist + warp * E, perm_src, inv_perm);
 }
 
 // Multi-chunk path, launch 1: per-chunk histograms -> ws_hist[chunk][E].
+template <int kPer>
 __global__ void __launch_bounds__(kRouteThreads)
 route_hist_kernel(const int32_t* __restrict__ ids, int R, int E, int* ws_hist, int* status) {
   extern __shared__ int hist[];
   for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) hist[i] = 0;
-  __syncthreads();
-  const int c0 = blockIdx.x * kRouteChunk, c1 = min(c0 + kRouteChunk, R);
+  const int c0 = blockIdx.x * 1024 * kPer, c1 = min(c0 + 1024 * kPer, R);
   int f0, f1;
-  sub_chunk(c0, c1, f0, f1);
-  int x[kPerLane];
-  warp_load_ids(ids, f0, f1, E, x, status);
-  warp_histogram(x, hist + (threadIdx.x >> 5) * E);
+  warp_run<kPer>(c0, c1, f0, f1);
+  int x[kPer];
+  unsigned m[kPer];
+  warp_load_ids<kPer>(ids, f0, f1, E, x, status);
   __syncthreads();
-  for (int x = threadIdx.x; x < E; x += blockDim.x) {
+  warp_histogram<kPer>(x, m, f0, f1, hist + (threadIdx.x >> 5) * E, key_bits(E));
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int s = 0;
-    for (int w = 0; w < 32; ++w) s += hist[w * E + x];
-    ws_hist[(size_t)blockIdx.x * E + x] = s;
+    for (int w = 0; w < 32; ++w) s += hist[w * E + e];
+    ws_hist[(size_t)blockIdx.x * E + e] = s;
   }
 }
 
@@ -164,54 +190,60 @@ __global__ void __launch_bounds__(kRouteThreads)
 route_scan_kernel(const int* ws_hist, int nchunks, int E, int32_t* off, int* ws_base) {
   __shared__ int warp_sums[32];
   __shared__ int total;
-  const int x = threadIdx.x;
+  const int e = threadIdx.x;
   int tot = 0;
-  if (x < E)
-    for (int b = 0; b < nchunks; ++b) tot += ws_hist[(size_t)b * E + x];
+  if (e < E)
+    for (int b = 0; b < nchunks; ++b) tot += ws_hist[(size_t)b * E + e];
   const int start = block_exclusive_scan(tot, warp_sums, &total);
-  if (x < E) {
-    off[x] = start;
+  if (e < E) {
+    off[e] = start;
     int run = start;
     for (int b = 0; b < nchunks; ++b) {
-      int c = ws_hist[(size_t)b * E + x];
-      ws_base[(size_t)b * E + x] = run;
+      int c = ws_hist[(size_t)b * E + e];
+      ws_base[(size_t)b * E + e] = run;
       run += c;
     }
   }
-  if (x == 0) off[E] = total;
+  if (e == 0) off[E] = total;
 }
 
 // Launch 3: per chunk, warp bases from the chunk base, then the stable scatter.
+template <int kPer>
 __global__ void __launch_bounds__(kRouteThreads)
 route_scatter_kernel(const int32_t* __restrict__ ids, int R, int E, const int* ws_base,
                      int32_t* perm_src, int32_t* inv_perm) {
   extern __shared__ int hist[];
   for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) hist[i] = 0;
-  __syncthreads();
-  const int c0 = blockIdx.x * kRouteChunk, c1 = min(c0 + kRouteChunk, R);
+  const int c0 = blockIdx.x * 1024 * kPer, c1 = min(c0 + 1024 * kPer, R);
   int f0, f1;
-  sub_chunk(c0, c1, f0, f1);
+  warp_run<kPer>(c0, c1, f0, f1);
   const int warp = threadIdx.x >> 5;
-  int x[kPerLane];
-  warp_load_ids(ids, f0, f1, E, x, nullptr);
-  warp_histogram(x, hist + warp * E);
+  int x[kPer];
+  unsigned m[kPer];
+  warp_load_ids<kPer>(ids, f0, f1, E, x, nullptr);
   __syncthreads();
-  for (int x = threadIdx.x; x < E; x += blockDim.x) {
-    int run = ws_base[(size_t)blockIdx.x * E + x];
+  warp_histogram<kPer>(x, m, f0, f1, hist + warp * E, key_bits(E));
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = ws_base[(size_t)blockIdx.x * E + e];
     for (int w = 0; w < 32; ++w) {
-      int c = hist[w * E + x];
-      hist[w * E + x] = run;
+      int c = hist[w * E + e];
+      hist[w * E + e] = run;
       run += c;
     }
   }
   __syncthreads();
-  warp_scatter(x, f0, hist + warp * E, perm_src, inv_perm);
+  warp_scatter<kPer>(x, m, f0, f1, hist + warp * E, perm_src, inv_perm);
 }
 
-int route_chunks(int R) { return R <= kRouteChunk ? 1 : (R + kRouteChunk - 1) / kRouteChunk; }
+int route_chunks(int R, int E) {
+  if (R <= 1024) return 1;
+  const int c = route_chunk_size(R, E);
+  return (R + c - 1) / c;
+}
 
 size_t route_workspace_bytes(int R, int E) {
-  const int nc = route_chunks(R);
+  const int nc = route_chunks(R, E);
   return nc <= 1 ? 0 : (size_t)2 * nc * E * sizeof(int);
 }
 
@@ -219,27 +251,36 @@ bool route_supported(int E) { return E >= 1 && E <= kRouteMaxE; }
 
 cudaError_t route_set_smem_attrs() {
   const int bytes = 32 * kRouteMaxE * (int)sizeof(int);
-  cudaError_t e1 = cudaFuncSetAttribute(route_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  cudaError_t e2 = cudaFuncSetAttribute(route_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  cudaError_t e3 = cudaFuncSetAttribute(route_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e1 != cudaSuccess) return e1;
-  if (e2 != cudaSuccess) return e2;
-  return e3;
+  const cudaError_t errs[5] = {
+      cudaFuncSetAttribute(route_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
+      cudaFuncSetAttribute(route_hist_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
+      cudaFuncSetAttribute(route_hist_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
+      cudaFuncSetAttribute(route_scatter_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
+      cudaFuncSetAttribute(route_scatter_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)};
+  for (cudaError_t e : errs)
+    if (e != cudaSuccess) return e;
+  return cudaSuccess;
 }
 
 cudaError_t launch_route(const int32_t* ids, int R, int E, int32_t* off, int32_t* perm_src,
                          int32_t* inv_perm, void* ws, int* status, cudaStream_t stream) {
   const size_t smem = (size_t)32 * E * sizeof(int);
-  const int nc = route_chunks(R);
+  const int nc = route_chunks(R, E);
   if (nc <= 1) {
     route_single_kernel<<<1, kRouteThreads, smem, stream>>>(ids, R, E, off, perm_src, inv_perm, status);
     return cudaGetLastError();
   }
   int* ws_hist = static_cast<int*>(ws);
   int* ws_base = ws_hist + (size_t)nc * E;
-  route_hist_kernel<<<nc, kRouteThreads, smem, stream>>>(ids, R, E, ws_hist, status);
-  route_scan_kernel<<<1, kRouteThreads, 0, stream>>>(ws_hist, nc, E, off, ws_base);
-  route_scatter_kernel<<<nc, kRouteThreads, smem, stream>>>(ids, R, E, ws_base, perm_src, inv_perm);
+  if (route_chunk_size(R, E) == 1024) {
+    route_hist_kernel<1><<<nc, kRouteThreads, smem, stream>>>(ids, R, E, ws_hist, status);
+    route_scan_kernel<<<1, kRouteThreads, 0, stream>>>(ws_hist, nc, E, off, ws_base);
+    route_scatter_kernel<1><<<nc, kRouteThreads, smem, stream>>>(ids, R, E, ws_base, perm_src, inv_perm);
+  } else {
+    route_hist_kernel<8><<<nc, kRouteThreads, smem, stream>>>(ids, R, E, ws_hist, status);
+    route_scan_kernel<<<1, kRouteThreads, 0, stream>>>(ws_hist, nc, E, off, ws_base);
+    route_scatter_kernel<8><<<nc, kRouteThreads, smem, stream>>>(ids, R, E, ws_base, perm_src, inv_perm);
+  }
   return cudaGetLastError();
 }
 

@@ -4,7 +4,8 @@
 // (paperlayer.ai summary), §D.1 (p.19): scatter after the expert GEMM.
 //   out[t][n] = bf16_rne( sum_{j<k} fp32(g[t][j] * Y[inv_perm[t*k + j]][n]) ),
 // products and the running sum in fp32 (starting at 0), j ascending.  One thread owns eight
-// consecutive outputs: 128-bit gathers of Y rows, 128-bit stores of out.
+// consecutive outputs: 128-bit gathers of Y rows (a token's rows all in flight at once),
+// 128-bit stores of out.
 #include "gsg_internal.cuh"
 
 namespace gsg {
@@ -15,24 +16,39 @@ __global__ void __launch_bounds__(kUnpermThreads)
 unpermute_kernel(const uint16_t* __restrict__ Y, const int32_t* __restrict__ inv_perm,
                  const float* __restrict__ gates, int T, int k, int N, int R, uint16_t* __restrict__ out,
                  int* status) {
-  const int n8 = N / 8;
-  const long long total = (long long)T * n8;
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (long long)gridDim.x * blockDim.x) {
+  const unsigned n8 = (unsigned)N / 8u;
+  const unsigned total = (unsigned)T * n8;   // T * N / 8 < 2^31 is checked on the host
+  for (unsigned i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
     const int t = int(i / n8), c = int(i % n8);
     float acc[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
-    for (int j = 0; j < k; ++j) {
-      const int row = __ldg(inv_perm + (size_t)t * k + j);
-      if (row < 0 || row >= R) { set_status(status, GSG_ERR_BAD_ROUTING); continue; }
-      const float g = __ldg(gates + (size_t)t * k + j);
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(Y + (size_t)row * N) + c);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    // up to eight routed rows at a time: every index, gate and row load is issued before the
+    // first use, then the products are summed in j order
+    for (int j0 = 0; j0 < k; j0 += 8) {
+      int row[8];
+      float g[8];
+      uint4 v[8];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        acc[2 * q] = __fadd_rn(acc[2 * q], __fmul_rn(g, __uint_as_float(w[q] << 16)));
-        acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], __fmul_rn(g, __uint_as_float(w[q] & 0xFFFF0000u)));
+      for (int jj = 0; jj < 8; ++jj) {
+        const bool in = j0 + jj < k;
+        row[jj] = in ? __ldg(inv_perm + (size_t)t * k + j0 + jj) : -1;
+        g[jj] = in ? __ldg(gates + (size_t)t * k + j0 + jj) : 0.0f;
+      }
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj)
+        v[jj] = (row[jj] >= 0 && row[jj] < R) ? __ldg(reinterpret_cast<const uint4*>(Y + (size_t)row[jj] * N) + c)
+                                              : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) {
+        if (j0 + jj >= k) break;
+        if (row[jj] < 0 || row[jj] >= R) { set_status(status, GSG_ERR_BAD_ROUTING); continue; }
+        const uint32_t w[4] = {v[jj].x, v[jj].y, v[jj].z, v[jj].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          acc[2 * q] = __fadd_rn(acc[2 * q], __fmul_rn(g[jj], __uint_as_float(w[q] << 16)));
+          acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], __fmul_rn(g[jj], __uint_as_float(w[q] & 0xFFFF0000u)));
+        }
       }
     }
     uint32_t o[4];

@@ -126,7 +126,7 @@ gsg_status_t gsg_moe_route_permute(const int32_t* topk_ids, int T, int k, int E,
  * as the weights) and written to each of its k routed rows inv_perm[t*k + j]
  * (inv_perm NULL: row t, and k must be 1).  sf_block: 32 (sparse GEMM) or 16 (dense control).
  * Outputs: codes [R][K/2], scales in the quad layout above (R = T*k), x_tensor_scale_out fp32[1].
- * Limits: T*k <= 2^30 and T*K/16 < 2^31, else GSG_ERR_UNSUPPORTED_SHAPE.
+ * Limits: T*k <= 2^30 and T*K/8 < 2^31, else GSG_ERR_UNSUPPORTED_SHAPE.
  */
 gsg_status_t gsg_quantize_act_nvfp4(const uint16_t* X, int T, int K, int sf_block,
                                     const int32_t* inv_perm, int k,
@@ -168,7 +168,8 @@ gsg_status_t gsg_grouped_dense_gemm(const uint8_t* a_codes, const uint8_t* a_sca
  * Paper: §D.1 (p.19): scatter after the expert GEMM.
  *     out[t][n] = bf16_rne( sum_{j<k} fp32(gates[t][j] * Y[inv_perm[t*k+j]][n]) )
  * fp32 products and running sum (starting at 0), j ascending.  Y bf16 [R][N],
- * gates fp32 [T][k], out bf16 [T][N].  N % 8 == 0.
+ * gates fp32 [T][k], out bf16 [T][N].  N % 8 == 0; T*k <= 2^30 and T*N/8 < 2^31, else
+ * GSG_ERR_UNSUPPORTED_SHAPE.
  */
 gsg_status_t gsg_unpermute_scale(const uint16_t* Y, const int32_t* inv_perm, const float* gates,
                                  int T, int k, int N, uint16_t* out, void* stream);
@@ -182,7 +183,7 @@ gsg_status_t gsg_unpermute_scale(const uint16_t* Y, const int32_t* inv_perm, con
  * outputs, result and errors as gsg_moe_route_permute; the workspace is replaced by a fixed
  * 256 KiB device array inside the library, which every GPU that loads the library holds until
  * the process exits.  The call allocates nothing.
- * Limit: R = T*k <= 8192 needs no scratch; above that ceil(R/8192) * E <= 32768
+ * Limit: R = T*k <= 1024 needs no scratch; above that ceil(R/8192) * E <= 32768
  * (E = 384: R <= 696,320; E = 128: R <= 2,097,152), else GSG_ERR_UNSUPPORTED_SHAPE with no
  * launch.  The first call on a device sets up that device (the library's per-device set-up and
  * the scratch's device address); make that first call before any stream capture begins.

@@ -2,7 +2,7 @@
 not allocate device memory) against gsg_moe_route_permute (caller-supplied workspace).
 
 Both calls go through the C ABI.  The GPU test routes two different problems in a row that both
-need the scratch (more than one 8192-row chunk), so the second call runs on the first one's
+need the scratch (more than one routing chunk), so the second call runs on the first one's
 leftover scratch contents; routing is integer work, so outputs must match bit for bit.  This file
 is collected last so that it runs both after the other tests and, alone, in a fresh process
 where its first call does the per-device set-up.
@@ -59,7 +59,7 @@ def test_noalloc_matches_workspace_routing_twice_in_a_row():
     L = gsg.load_library()
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     g = torch.Generator().manual_seed(77)
-    cases = [(8192, 8, 384), (3000, 7, 128)]     # R = 65536 (8 chunks), R = 21000 (3 chunks)
+    cases = [(8192, 8, 384), (3000, 7, 128)]     # R = 65536 (8 chunks of 8192), R = 21000 (21 of 1024)
     inputs = [torch.randint(0, E, (T, k), generator=g, dtype=torch.int32).cuda() for T, k, E in cases]
     got = [_route_noalloc(L, ids, E, stream) for ids, (_, _, E) in zip(inputs, cases)]
     want = [_route_with_workspace(L, ids, E, stream) for ids, (_, _, E) in zip(inputs, cases)]
