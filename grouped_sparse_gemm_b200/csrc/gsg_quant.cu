@@ -7,10 +7,11 @@
 //
 // Launch 1 (skipped when the caller supplies s_x): partial max|X| per block, 128-bit loads,
 // warp-shuffle reductions.  Launch 2: every block folds the partials into s_x = amax/2688,
-// then each thread quantizes 8 consecutive elements of one token row (one 128-bit load),
-// groups of 4 lanes (2 for 16-element blocks) combine their maxima into the block amax, the
-// four scales of one MMA k-block are gathered into a 32-bit word, and the token's codes and
-// scale words are written to each of its k routed rows (the dispatch).  The same launch zero-fills
+// then each warp quantizes 256 consecutive elements of one token row at a time (8 per lane, one
+// 128-bit load), groups of 4 lanes (2 for 16-element blocks) combine their maxima into the
+// block amax, the four scales of one MMA k-block are gathered into a 32-bit word, and the
+// token's codes and scale words are written to each of its k routed rows (the dispatch), the
+// rows read once per warp (lane j holds row j) and the scale words spread over the lanes.  The same launch zero-fills
 // the padding entries of the quad scale layout.
 #include "gsg_internal.cuh"
 
@@ -70,10 +71,37 @@ struct QuantParams {
   int* status;
 };
 
+// One warp-iteration covers 256 consecutive elements of one token row (K % 256 == 0): lane L
+// holds elements 8L..8L+7 of them, and lane j < k also holds the token's j-th routed row.
+struct QuantSlice {
+  uint4 x;
+  int myrow;
+};
+
+__device__ __forceinline__ void quant_fetch(const QuantParams& p, long long base, int units_per_row, int lane,
+                                            QuantSlice& q) {
+  const unsigned b32 = (unsigned)base;   // U = T*K/8 < 2^31 is checked on the host
+  const int t = int(b32 / (unsigned)units_per_row);
+  const int c8 = int(b32 % (unsigned)units_per_row) + lane;
+  q.x = __ldg(reinterpret_cast<const uint4*>(p.X + (size_t)t * p.K + (size_t)c8 * 8));
+  q.myrow = lane < p.k ? (p.inv_perm != nullptr ? __ldg(p.inv_perm + (size_t)t * p.k + lane) : t) : -1;
+}
+
 __global__ void __launch_bounds__(kQuantThreads)
 act_quant_kernel(QuantParams p) {
   __shared__ float red[kQuantThreads / 32];
   __shared__ float s_sh;
+  const int lane = threadIdx.x & 31;
+  const int units_per_row = p.K / 8;
+  const long long U = (long long)p.T * units_per_row;   // a multiple of 32
+  const int gwarp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  const long long wstep = (long long)nwarps * 32;
+  // the first slice's loads go out before the tensor scale is known (they do not depend on it)
+  long long base = (long long)gwarp * 32;
+  QuantSlice cur;
+  if (base < U) quant_fetch(p, base, units_per_row, lane, cur);
+
   // ---- tensor scale
   if (p.s_in != nullptr) {
     if (threadIdx.x == 0) s_sh = __ldg(p.s_in);
@@ -94,82 +122,73 @@ act_quant_kernel(QuantParams p) {
   if (blockIdx.x == 0 && threadIdx.x == 0) *p.s_out = s;
   const float six_s = __fmul_rn(6.0f, s);
 
-  const int lane = threadIdx.x & 31;
-  const int units_per_row = p.K / 8;
-  const long long U = (long long)p.T * units_per_row;
-  const int KBa = p.K / (4 * p.sf);
-  const int gwarp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int nwarps = (gridDim.x * blockDim.x) >> 5;
-  // ---- main: each lane quantizes 8 consecutive elements; a warp covers 256 elements of one row
-  // (K % 256 == 0), so a 32-element block is 4 lanes (16-element block: 2 lanes) and one MMA
-  // k-block's four scales sit in 16 lanes (8).  The loop is warp-uniform so the shuffles see the
-  // full warp.
-  for (long long base = (long long)gwarp * 32; base < U; base += (long long)nwarps * 32) {
-    const long long unit = base + lane;
-    const bool valid = unit < U;
-    const unsigned u32 = (unsigned)unit;   // U = T*K/8 < 2^31 is checked on the host
-    const int t = valid ? int(u32 / (unsigned)units_per_row) : 0;
-    const int c8 = valid ? int(u32 % (unsigned)units_per_row) : 0;
+  // a 32-element block is 4 lanes (16-element block: 2 lanes); one MMA k-block's four scales
+  // sit in 16 lanes (8), so a slice holds nkb = 2 (4) k-blocks
+  const int step = p.sf == 32 ? 4 : 2;
+  const int nkb = 8 / step;
+  uint32_t* sw = reinterpret_cast<uint32_t*>(p.scales);
+  for (; base < U; base += wstep) {
+    const QuantSlice q = cur;
+    if (base + wstep < U) quant_fetch(p, base + wstep, units_per_row, lane, cur);
+    const unsigned b32 = (unsigned)base;
+    const int t = int(b32 / (unsigned)units_per_row);
+    const int c80 = int(b32 % (unsigned)units_per_row);   // first unit of the slice in its row
     float x[8];
-    float amax = 0.0f;
-    if (valid) {
-      const uint4 a = __ldg(reinterpret_cast<const uint4*>(p.X + (size_t)t * p.K + (size_t)c8 * 8));
-      const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+    const uint32_t w[4] = {q.x.x, q.x.y, q.x.z, q.x.w};
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        x[2 * j] = bf16_bits_to_f32(w[j] & 0xFFFFu);
-        x[2 * j + 1] = bf16_bits_to_f32(w[j] >> 16);
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(x[j]));
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) x[j] = 0.0f;
+    for (int j = 0; j < 4; ++j) {
+      x[2 * j] = bf16_bits_to_f32(w[j] & 0xFFFFu);
+      x[2 * j + 1] = bf16_bits_to_f32(w[j] >> 16);
     }
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(x[j]));
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
     if (p.sf == 32) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
     const BlockScale bs = block_scale(amax, six_s, s);
     uint32_t codes = 0;
 #pragma unroll
     for (int j = 0; j < 8; ++j) codes |= e2m1_encode(__fmul_rn(x[j], bs.inv)) << (4 * j);
-    // four scales of one MMA k-block -> one 32-bit word (sf 32: lanes g, g+4, g+8, g+12;
-    // sf 16: g, g+2, g+4, g+6)
-    const int step = p.sf == 32 ? 4 : 2;
+    // four scales of one MMA k-block -> one 32-bit word, held by the k-block's first lane
     const int g = lane & ~(4 * step - 1);
     const uint32_t word = __shfl_sync(0xffffffffu, bs.sc, g) | (__shfl_sync(0xffffffffu, bs.sc, g + step) << 8) |
                           (__shfl_sync(0xffffffffu, bs.sc, g + 2 * step) << 16) |
                           (__shfl_sync(0xffffffffu, bs.sc, g + 3 * step) << 24);
-    const int kb = p.sf == 32 ? (c8 >> 4) : (c8 >> 3);
-    const bool writer = (lane & (4 * step - 1)) == 0;
-    if (!valid) continue;
-    // the token's destination rows, all loaded before any store (up to 16 at a time)
-    for (int j0 = 0; j0 < p.k; j0 += 16) {
-      int rows[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j)
-        rows[j] = (j0 + j < p.k) ? (p.inv_perm != nullptr ? __ldg(p.inv_perm + (size_t)t * p.k + j0 + j) : t) : -1;
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        if (j0 + j >= p.k) break;
-        const int row = rows[j];
-        if (row < 0 || row >= p.R) { set_status(p.status, GSG_ERR_BAD_ROUTING); continue; }
-        *reinterpret_cast<uint32_t*>(p.codes + (size_t)row * (p.K / 2) + (size_t)c8 * 4) = codes;
-        if (writer) {
-          uint32_t* sw = reinterpret_cast<uint32_t*>(p.scales);
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const int rr = row - 32 * c;
-            if (rr >= 0) sw[((size_t)kb * p.rcap + rr) * 4 + c] = word;
-          }
+    // dispatch: codes of the slice to each of the token's k routed rows (row j from lane j)
+    int myrow = q.myrow;
+    for (int j0 = 0; j0 < p.k; j0 += 32) {
+      if (j0 > 0)
+        myrow = j0 + lane < p.k ? (p.inv_perm != nullptr ? __ldg(p.inv_perm + (size_t)t * p.k + j0 + lane) : t) : -1;
+      const int jn = min(32, p.k - j0);
+      for (int j = 0; j < jn; ++j) {
+        const int row = __shfl_sync(0xffffffffu, myrow, j);
+        if (row < 0 || row >= p.R) {   // warp-uniform
+          if (lane == 0) set_status(p.status, GSG_ERR_BAD_ROUTING);
+          continue;
+        }
+        *reinterpret_cast<uint32_t*>(p.codes + (size_t)row * (p.K / 2) + (size_t)(c80 + lane) * 4) = codes;
+      }
+      // scale words: entry (j, c, kbw) of this row group, spread over the lanes
+      const int ng = jn * 4 * nkb;
+      for (int e0 = 0; e0 < ng; e0 += 32) {
+        const int e = e0 + lane;
+        const int jj = e / (4 * nkb), rem = e % (4 * nkb);
+        const int c = rem & 3, kbw = rem >> 2;
+        const int row = __shfl_sync(0xffffffffu, myrow, jj & 31);
+        const uint32_t wd = __shfl_sync(0xffffffffu, word, (kbw * 4 * step) & 31);
+        const int rr = row - 32 * c;
+        if (e < ng && row >= 0 && row < p.R && rr >= 0) {
+          const int kb = c80 / (4 * step) + kbw;
+          sw[((size_t)kb * p.rcap + rr) * 4 + c] = wd;
         }
       }
     }
   }
   // ---- zero the quad entries that refer to rows >= R
+  const int KBa = p.K / (4 * p.sf);
   const int r_lo = p.R > 96 ? p.R - 96 : 0;
   const int span = p.rcap - r_lo;                 // at most 352 rows
   const int npad = KBa * span * 4;                // K / 128 * 352 * 4 < 2^31
-  uint32_t* sw = reinterpret_cast<uint32_t*>(p.scales);
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < npad; i += gridDim.x * blockDim.x) {
     const int c = i & 3;
     const int rest = i >> 2;
@@ -203,7 +222,8 @@ cudaError_t launch_quant(const uint16_t* X, int T, int K, int sf, const int32_t*
   p.T = T; p.K = K; p.sf = sf; p.k = k; p.R = T * k; p.rcap = T * k + kActScalePadRows;
   p.codes = codes; p.scales = scales; p.s_out = s_out; p.status = status;
   const long long units = (long long)T * (K / 8);
-  long long blocks = (units + kQuantThreads - 1) / kQuantThreads;
+  const long long pad = (long long)(K / (4 * sf)) * (T * k + kActScalePadRows - (T * k > 96 ? T * k - 96 : 0)) * 4;
+  long long blocks = ((units > pad ? units : pad) + kQuantThreads - 1) / kQuantThreads;
   if (blocks < 1) blocks = 1;
   if (blocks > (long long)num_sms * 8) blocks = (long long)num_sms * 8;
   act_quant_kernel<<<(unsigned)blocks, kQuantThreads, 0, stream>>>(p);

@@ -9,8 +9,10 @@
 // indices (one per thread) while ceil(R/1024) * E <= 16384 (a workspace of at most 128 KiB),
 // else 8192 (eight per thread).  Each warp owns a contiguous run of its chunk; lanes holding
 // the same id are found with one ballot per id bit, which gives each index its rank among equal
-// ids of its warp, and per-warp histograms live in shared memory (32 x E ints).  R <= 1024 is one launch; larger R is histogram -> scan -> scatter
-// over a [chunks x E] workspace.  Only integer arithmetic: the result is deterministic.
+// ids of its warp, and per-warp histograms live in shared memory (32 x E ints).  R <= 1024 is
+// one launch; larger R is histogram -> (scan) -> scatter over a [chunks x E] workspace, the scan
+// folded into the scatter for 1024-index chunks.  Only integer arithmetic: the result is
+// deterministic.
 #include "gsg_internal.cuh"
 
 namespace gsg {
@@ -207,12 +209,34 @@ route_scan_kernel(const int* ws_hist, int nchunks, int E, int32_t* off, int* ws_
   if (e == 0) off[E] = total;
 }
 
-// Launch 3: per chunk, warp bases from the chunk base, then the stable scatter.
-template <int kPer>
+// Launch 3: per chunk, warp bases from the chunk base, then the stable scatter.  With kSelfScan
+// (1024-index chunks, where chunks x experts is small) there is no launch 2: every block sums the
+// chunk histograms itself (ws = ws_hist), block 0 writes the offsets.  Otherwise ws = ws_base.
+template <int kPer, bool kSelfScan>
 __global__ void __launch_bounds__(kRouteThreads)
-route_scatter_kernel(const int32_t* __restrict__ ids, int R, int E, const int* ws_base,
+route_scatter_kernel(const int32_t* __restrict__ ids, int R, int E, const int* ws, int nchunks, int32_t* off,
                      int32_t* perm_src, int32_t* inv_perm) {
   extern __shared__ int hist[];
+  __shared__ int warp_sums[32];
+  __shared__ int total;
+  int chunk_base = 0;
+  if (kSelfScan) {
+    // expert e's first row in this chunk: rows of experts < e, then of earlier chunks
+    const int e = threadIdx.x;
+    int tot = 0, before = 0;
+    if (e < E)
+      for (int b = 0; b < nchunks; ++b) {
+        const int c = ws[(size_t)b * E + e];
+        tot += c;
+        if (b < (int)blockIdx.x) before += c;
+      }
+    const int start = block_exclusive_scan(tot, warp_sums, &total);
+    chunk_base = start + before;
+    if (blockIdx.x == 0) {
+      if (e < E) off[e] = start;
+      if (e == 0) off[E] = total;
+    }
+  }
   for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) hist[i] = 0;
   const int c0 = blockIdx.x * 1024 * kPer, c1 = min(c0 + 1024 * kPer, R);
   int f0, f1;
@@ -225,7 +249,7 @@ route_scatter_kernel(const int32_t* __restrict__ ids, int R, int E, const int* w
   warp_histogram<kPer>(x, m, f0, f1, hist + warp * E, key_bits(E));
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int run = ws_base[(size_t)blockIdx.x * E + e];
+    int run = kSelfScan ? chunk_base : ws[(size_t)blockIdx.x * E + e];
     for (int w = 0; w < 32; ++w) {
       int c = hist[w * E + e];
       hist[w * E + e] = run;
@@ -255,8 +279,8 @@ cudaError_t route_set_smem_attrs() {
       cudaFuncSetAttribute(route_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
       cudaFuncSetAttribute(route_hist_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
       cudaFuncSetAttribute(route_hist_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
-      cudaFuncSetAttribute(route_scatter_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
-      cudaFuncSetAttribute(route_scatter_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)};
+      cudaFuncSetAttribute(route_scatter_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
+      cudaFuncSetAttribute(route_scatter_kernel<8, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes)};
   for (cudaError_t e : errs)
     if (e != cudaSuccess) return e;
   return cudaSuccess;
@@ -274,12 +298,13 @@ cudaError_t launch_route(const int32_t* ids, int R, int E, int32_t* off, int32_t
   int* ws_base = ws_hist + (size_t)nc * E;
   if (route_chunk_size(R, E) == 1024) {
     route_hist_kernel<1><<<nc, kRouteThreads, smem, stream>>>(ids, R, E, ws_hist, status);
-    route_scan_kernel<<<1, kRouteThreads, 0, stream>>>(ws_hist, nc, E, off, ws_base);
-    route_scatter_kernel<1><<<nc, kRouteThreads, smem, stream>>>(ids, R, E, ws_base, perm_src, inv_perm);
+    route_scatter_kernel<1, true><<<nc, kRouteThreads, smem, stream>>>(ids, R, E, ws_hist, nc, off, perm_src,
+                                                                       inv_perm);
   } else {
     route_hist_kernel<8><<<nc, kRouteThreads, smem, stream>>>(ids, R, E, ws_hist, status);
     route_scan_kernel<<<1, kRouteThreads, 0, stream>>>(ws_hist, nc, E, off, ws_base);
-    route_scatter_kernel<8><<<nc, kRouteThreads, smem, stream>>>(ids, R, E, ws_base, perm_src, inv_perm);
+    route_scatter_kernel<8, false><<<nc, kRouteThreads, smem, stream>>>(ids, R, E, ws_base, nc, off, perm_src,
+                                                                        inv_perm);
   }
   return cudaGetLastError();
 }

@@ -114,6 +114,20 @@ def test_quantize_matches_oracle(gsg, name, sf):
     _status_ok(gsg)
 
 
+@pytest.mark.parametrize("T,k,E,K,sf", [(5, 40, 64, 512, 32), (9, 33, 48, 256, 16), (3, 3, 3, 768, 32)])
+def test_quantize_many_routed_rows(gsg, T, k, E, K, sf):
+    # top-k above one warp's 32 lanes, the 16-element block path and a K of three 256-wide slices
+    cfg = inputs.custom_config("qk", E=E, K=K, N=128, T=T, top_k=k)
+    X = inputs.activations(cfg)
+    off, ps, ip = tl.route_np(inputs.routing(cfg), E)
+    qa = gsg.quantize_act_nvfp4(X.to(DEV), sf_block=sf, inv_perm=torch.from_numpy(ip).to(DEV), top_k=k)
+    codes, quad, s, _, _ = tl.oracle_act(X.float().numpy(), sf, ps, k)
+    assert qa.x_scale.item() == s
+    np.testing.assert_array_equal(qa.codes.cpu().numpy(), codes)
+    np.testing.assert_array_equal(qa.scales.cpu().numpy(), quad)
+    _status_ok(gsg)
+
+
 def test_quantize_identity_and_given_scale(gsg):
     cfg = inputs.custom_config("q", E=1, K=512, N=128, T=37, top_k=1, outlier_frac=0.01, outlier_scale=50.0)
     X = inputs.activations(cfg)
