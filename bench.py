@@ -195,7 +195,10 @@ class Workload:
         gsg.unpermute_scale(self.Y, self.route.inv_perm, self.gates, c.top_k, out=self.out)
 
     def launches_per_step(self) -> int:
-        route = 1 if self.cfg.R <= 8192 else 3
+        """Library kernels one step launches (the library's routing rule: one launch up to 1024
+        rows, histogram + scatter while ceil(R/1024)*E <= 16384, else histogram + scan + scatter)."""
+        R, E = self.cfg.R, self.cfg.E
+        route = 1 if R <= 1024 else (2 if -(-R // 1024) * E <= 16384 else 3)
         return route + 2 + 1 + 1        # route, amax + quantize, GEMM, scatter
 
     def gemm(self):
@@ -533,6 +536,27 @@ def gsg_token_tile(max_rows: int, R: int, E: int) -> int:
     return 128 if R >= 64 * E else 64
 
 
+def run_profile_steps(args, local):
+    """The step graph replayed warmup + steps times and nothing else, so that a profiler's launch
+    list holds only the step's kernels in step order."""
+    dev = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(dev)
+    gsg.load_library()
+    cfg = inputs.CONFIGS[args.config]
+    wl = Workload(cfg, dev, with_dense=False)
+    wl.step()
+    torch.cuda.synchronize()
+    g = capture(wl.step, warm=0)
+    for _ in range(args.warmup + args.steps):
+        g.replay()
+    torch.cuda.synchronize()
+    st = gsg.get_device_status()
+    print(json.dumps({"profile_steps": args.warmup + args.steps, "config": cfg.name,
+                      "kernels_per_step": wl.launches_per_step(), "status": st}), flush=True)
+    if st != 0:
+        raise RuntimeError(f"device status {st}")
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -543,6 +567,8 @@ def main():
     ap.add_argument("--quick", action="store_true", help="skip e2e, dense control and CPU baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-experts", type=int, default=24)
+    ap.add_argument("--profile-steps", action="store_true",
+                    help="for profiler launch lists: only replay the step graph (warmup + steps), print no bench line")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -550,6 +576,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif args.profile_steps:
+            run_profile_steps(args, local)
         else:
             run_ours(args, world, rank, local)
     finally:

@@ -7,7 +7,7 @@
 // §D.2 (p.19) -- a dense control that differs from the sparse kernel only in sparsity.
 //
 // One CTA per SM, 352 threads (11 warps), warp-specialised around one shared-memory ring whose
-// stages hold 256 or 512 logical K of one tile (weights, activation codes and both scales):
+// stages hold 256 to 768 logical K of one tile (weights, activation codes and both scales):
 //   warp 0      weight producer: one bulk copy per stage of the interleaved packed weight blocks.
 //   warp 2      activation producer: tensor-map TMA boxes (128B swizzle) of only the token rows the
 //               tile holds, and one 3-D TMA box of the activation scale atoms.
@@ -255,7 +255,8 @@ template <bool kSparse, int kBN>
 struct Geo {
   static constexpr int kKbLogical = kSparse ? 128 : 64;            // logical K per MMA
   static constexpr int kKbPerChunk = kChunkK / kKbLogical;         // 2 sparse, 4 dense
-  static constexpr int kCPS = (kSparse || kBN <= 32) ? 2 : 1;     // 256-wide chunks per stage
+  // 256-wide K chunks per stage: short token tiles take longer stages (fewer waits per weight byte)
+  static constexpr int kCPS = kSparse ? (kBN <= 32 ? 3 : 2) : (kBN <= 32 ? 2 : 1);
   static constexpr int kKbps = kCPS * kKbPerChunk;                 // MMAs per stage
   static constexpr int kCB = kSparse ? kSparseChunkBytes : kDenseChunkBytes;   // packed chunk block
   static constexpr int kCBMeta = 8192;                             // metadata offset in a chunk block
@@ -610,7 +611,7 @@ static GemmPlan make_plan(bool sparse, int BN, int E, int tcap) {
   GemmPlan g;
   g.BN = BN;
   g.tcap = tcap;
-  g.cps = (sparse || BN <= 32) ? 2 : 1;
+  g.cps = sparse ? (BN <= 32 ? 3 : 2) : (BN <= 32 ? 2 : 1);
   const int kbps = g.cps * (sparse ? 2 : 4);
   const int body = g.cps * BN * 128 + g.cps * (sparse ? kSparseChunkBytes : kDenseChunkBytes) + kbps * 512;
   g.stage = (body + 1023) / 1024 * 1024;

@@ -69,6 +69,28 @@ __device__ __forceinline__ uint32_t e2m1_encode(float v) {
   return c | ((__float_as_uint(v) >> 28) & 8u);
 }
 
+// The same two encoders on the hardware converters (PTX cvt.rn.satfinite to e2m1x2 / e4m3x2):
+// round to nearest, ties to even, saturating at the largest finite value, sign kept.  For a
+// non-negative finite x the E4M3 code equals the UE4M3 code (sign bit 0).  Eight values -> eight
+// E2M1 codes, v[i] in bits 4i..4i+3.
+__device__ __forceinline__ uint32_t e2m1_encode8_cvt(const float v[8]) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+  return r;
+}
+__device__ __forceinline__ uint32_t ue4m3_encode_cvt(float x) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x));
+  return r & 0xFFu;
+}
+
 // Block rule shared by weights and activations (s = tensor scale, b = block amax):
 //   sc = UE4M3(b / (6 s)),  d = dec(sc) * s,  inv = d == 0 ? 0 : 1/d,  code = E2M1(v * inv)
 struct BlockScale {
@@ -78,6 +100,13 @@ struct BlockScale {
 __device__ __forceinline__ BlockScale block_scale(float blk_amax, float six_s, float s) {
   BlockScale r;
   r.sc = ue4m3_encode(__fdiv_rn(blk_amax, six_s));
+  float d = __fmul_rn(ue4m3_decode(r.sc), s);
+  r.inv = (d == 0.0f) ? 0.0f : __frcp_rn(d);
+  return r;
+}
+__device__ __forceinline__ BlockScale block_scale_cvt(float blk_amax, float six_s, float s) {
+  BlockScale r;
+  r.sc = ue4m3_encode_cvt(__fdiv_rn(blk_amax, six_s));
   float d = __fmul_rn(ue4m3_decode(r.sc), s);
   r.inv = (d == 0.0f) ? 0.0f : __frcp_rn(d);
   return r;

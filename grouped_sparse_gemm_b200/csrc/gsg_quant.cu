@@ -18,6 +18,7 @@
 namespace gsg {
 
 constexpr int kQuantThreads = 256;
+constexpr int kQuantMainThreads = 128;   // the quantize launch: more, smaller blocks balance the SMs
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
 
@@ -87,9 +88,9 @@ __device__ __forceinline__ void quant_fetch(const QuantParams& p, long long base
   q.myrow = lane < p.k ? (p.inv_perm != nullptr ? __ldg(p.inv_perm + (size_t)t * p.k + lane) : t) : -1;
 }
 
-__global__ void __launch_bounds__(kQuantThreads)
+__global__ void __launch_bounds__(kQuantMainThreads)
 act_quant_kernel(QuantParams p) {
-  __shared__ float red[kQuantThreads / 32];
+  __shared__ float red[kQuantMainThreads / 32];
   __shared__ float s_sh;
   const int lane = threadIdx.x & 31;
   const int units_per_row = p.K / 8;
@@ -112,7 +113,7 @@ act_quant_kernel(QuantParams p) {
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
     __syncthreads();
     if (threadIdx.x < 32) {
-      float w = threadIdx.x < kQuantThreads / 32 ? red[threadIdx.x] : 0.0f;
+      float w = threadIdx.x < kQuantMainThreads / 32 ? red[threadIdx.x] : 0.0f;
       w = warp_max(w);
       if (threadIdx.x == 0) s_sh = tensor_scale_from_amax(w);
     }
@@ -126,6 +127,7 @@ act_quant_kernel(QuantParams p) {
   // sit in 16 lanes (8), so a slice holds nkb = 2 (4) k-blocks
   const int step = p.sf == 32 ? 4 : 2;
   const int nkb = 8 / step;
+  const int lg_ent = p.sf == 32 ? 3 : 4;   // log2(4 * nkb): scale entries per routed row and slice
   uint32_t* sw = reinterpret_cast<uint32_t*>(p.scales);
   for (; base < U; base += wstep) {
     const QuantSlice q = cur;
@@ -145,10 +147,11 @@ act_quant_kernel(QuantParams p) {
     for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(x[j]));
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
     if (p.sf == 32) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-    const BlockScale bs = block_scale(amax, six_s, s);
-    uint32_t codes = 0;
+    const BlockScale bs = block_scale_cvt(amax, six_s, s);
+    float xs[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) codes |= e2m1_encode(__fmul_rn(x[j], bs.inv)) << (4 * j);
+    for (int j = 0; j < 8; ++j) xs[j] = __fmul_rn(x[j], bs.inv);
+    const uint32_t codes = e2m1_encode8_cvt(xs);
     // four scales of one MMA k-block -> one 32-bit word, held by the k-block's first lane
     const int g = lane & ~(4 * step - 1);
     const uint32_t word = __shfl_sync(0xffffffffu, bs.sc, g) | (__shfl_sync(0xffffffffu, bs.sc, g + step) << 8) |
@@ -172,7 +175,7 @@ act_quant_kernel(QuantParams p) {
       const int ng = jn * 4 * nkb;
       for (int e0 = 0; e0 < ng; e0 += 32) {
         const int e = e0 + lane;
-        const int jj = e / (4 * nkb), rem = e % (4 * nkb);
+        const int jj = e >> lg_ent, rem = e & (4 * nkb - 1);
         const int c = rem & 3, kbw = rem >> 2;
         const int row = __shfl_sync(0xffffffffu, myrow, jj & 31);
         const uint32_t wd = __shfl_sync(0xffffffffu, word, (kbw * 4 * step) & 31);
@@ -223,10 +226,10 @@ cudaError_t launch_quant(const uint16_t* X, int T, int K, int sf, const int32_t*
   p.codes = codes; p.scales = scales; p.s_out = s_out; p.status = status;
   const long long units = (long long)T * (K / 8);
   const long long pad = (long long)(K / (4 * sf)) * (T * k + kActScalePadRows - (T * k > 96 ? T * k - 96 : 0)) * 4;
-  long long blocks = ((units > pad ? units : pad) + kQuantThreads - 1) / kQuantThreads;
+  long long blocks = ((units > pad ? units : pad) + kQuantMainThreads - 1) / kQuantMainThreads;
   if (blocks < 1) blocks = 1;
-  if (blocks > (long long)num_sms * 8) blocks = (long long)num_sms * 8;
-  act_quant_kernel<<<(unsigned)blocks, kQuantThreads, 0, stream>>>(p);
+  if (blocks > (long long)num_sms * 16) blocks = (long long)num_sms * 16;
+  act_quant_kernel<<<(unsigned)blocks, kQuantMainThreads, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

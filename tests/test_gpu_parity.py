@@ -128,6 +128,35 @@ def test_quantize_many_routed_rows(gsg, T, k, E, K, sf):
     _status_ok(gsg)
 
 
+def _rounding_rows():
+    """bf16 rows whose 32-element blocks put values exactly on E2M1 rounding midpoints and block
+    maxima exactly on UE4M3 midpoints, subnormals and the saturation limit (with s_x = 1)."""
+    mids = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]
+    grid = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    blocks = []
+    for j in (-6, -2, 0, 3):                      # scale 2^j: block max 6 * 2^j
+        v = [6.0] + mids + [-m for m in mids] + grid + [-g for g in grid[1:]] + [0.1, -0.1, -0.0]
+        blocks.append([x * 2.0 ** j for x in v[:32]])
+    # block maxima / 6 on UE4M3 ties (1.0625 -> 1.0, 1.1875 -> 1.25), a subnormal tie
+    # (1.5 * 2^-9 -> 2^-8) and one far above 6 * 448 (saturates)
+    for amax in (6.375, 7.125, 9.0 * 2.0 ** -9, 4096.0):
+        blocks.append([amax] + [amax * f for f in (0.5, -0.25, 0.125, 0.9, -0.7, 0.33)] + [0.0] * 25)
+    rows = [sum(blocks[i:i + 8], []) for i in range(0, len(blocks), 8)]
+    return torch.tensor(rows, dtype=torch.float32).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("sf", [32, 16])
+def test_quantize_rounding_midpoints(gsg, sf):
+    X = _rounding_rows()
+    assert X.float().abs().max().item() == 4096.0     # 4096 / 6 > 448: the saturating block
+    one = torch.tensor([1.0], dtype=torch.float32)
+    qa = gsg.quantize_act_nvfp4(X.to(DEV), sf_block=sf, x_scale_in=one.to(DEV))
+    codes, quad, s, _, _ = tl.oracle_act(X.float().numpy(), sf, None, 1, np.float32(1.0))
+    np.testing.assert_array_equal(qa.codes.cpu().numpy(), codes)
+    np.testing.assert_array_equal(qa.scales.cpu().numpy(), quad)
+    _status_ok(gsg)
+
+
 def test_quantize_identity_and_given_scale(gsg):
     cfg = inputs.custom_config("q", E=1, K=512, N=128, T=37, top_k=1, outlier_frac=0.01, outlier_scale=50.0)
     X = inputs.activations(cfg)
