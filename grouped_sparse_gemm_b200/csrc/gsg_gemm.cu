@@ -306,7 +306,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
   auto acce_bar = [&](int a) { return bar0 + 8u * (2 * S + kNSets + NACC + a); };
   const uint32_t drain_bar = bar0 + 8u * (2 * S + kNSets + 2 * NACC);
 
-  // ---- set-up: barriers, TMEM, tile schedule, tensor scales
+  // ---- set-up: barriers, TMEM, tile schedule, tensor scales (global memory only after pdl_wait)
+  pdl_launch_dependents();
+  if (warp == 2 && lane == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_b)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_sfb)) : "memory");
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) { mbar_init(full_bar(s), 2); mbar_init(empty_bar(s), 1); }
     for (int s = 0; s < kNSets; ++s) mbar_init(tfull_bar(s), 4);
@@ -322,6 +327,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
+  pdl_wait();
   // expert offsets, clamped to [0, R] so a corrupt array can never send a copy or a store out
   // of bounds (a decreasing pair makes that expert empty, see below)
   bool bad = false;
@@ -683,13 +689,13 @@ cudaError_t gemm_set_smem_attrs() {
 }
 
 template <bool kSparse>
-static void launch_bn(int BN, int grid, size_t smem, cudaStream_t stream, const CUtensorMap& tb,
-                      const CUtensorMap& ts, const GemmParams& p) {
+static cudaError_t launch_bn(int BN, int grid, size_t smem, cudaStream_t stream, const CUtensorMap& tb,
+                             const CUtensorMap& ts, const GemmParams& p) {
   switch (BN) {
-    case 16: grouped_gemm_kernel<kSparse, 16><<<grid, kGemmThreads, smem, stream>>>(tb, ts, p); break;
-    case 32: grouped_gemm_kernel<kSparse, 32><<<grid, kGemmThreads, smem, stream>>>(tb, ts, p); break;
-    case 64: grouped_gemm_kernel<kSparse, 64><<<grid, kGemmThreads, smem, stream>>>(tb, ts, p); break;
-    default: grouped_gemm_kernel<kSparse, 128><<<grid, kGemmThreads, smem, stream>>>(tb, ts, p); break;
+    case 16: return launch_pdl(grouped_gemm_kernel<kSparse, 16>, grid, kGemmThreads, smem, stream, tb, ts, p);
+    case 32: return launch_pdl(grouped_gemm_kernel<kSparse, 32>, grid, kGemmThreads, smem, stream, tb, ts, p);
+    case 64: return launch_pdl(grouped_gemm_kernel<kSparse, 64>, grid, kGemmThreads, smem, stream, tb, ts, p);
+    default: return launch_pdl(grouped_gemm_kernel<kSparse, 128>, grid, kGemmThreads, smem, stream, tb, ts, p);
   }
 }
 
@@ -736,11 +742,9 @@ int launch_gemm(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, co
   p.w_scale = w_scale; p.off = off; p.Y = Y; p.status = status;
   p.E = E; p.N = N; p.K = K; p.R = R; p.y_f32 = y_f32; p.rcap = rcap;
   p.stages = g.stages; p.nacc = g.nacc; p.tcap = g.tcap;
-  if (sparse)
-    launch_bn<true>(g.BN, num_sms, g.smem, stream, tb, ts, p);
-  else
-    launch_bn<false>(g.BN, num_sms, g.smem, stream, tb, ts, p);
-  return cudaGetLastError() == cudaSuccess ? 0 : 1;
+  const cudaError_t e = sparse ? launch_bn<true>(g.BN, num_sms, g.smem, stream, tb, ts, p)
+                               : launch_bn<false>(g.BN, num_sms, g.smem, stream, tb, ts, p);
+  return e == cudaSuccess ? 0 : 1;
 }
 
 }  // namespace gsg

@@ -7,6 +7,7 @@
 #pragma once
 
 #include <cstdint>
+#include <utility>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -114,6 +115,33 @@ __device__ __forceinline__ BlockScale block_scale_cvt(float blk_amax, float six_
 
 __device__ __forceinline__ float tensor_scale_from_amax(float amax) {
   return amax == 0.0f ? 1.0f : __fdiv_rn(amax, kTensorScaleDen);
+}
+
+// ------------------------------------------------------------------ programmatic dependent launch
+// The step's kernels are launched with programmatic stream serialization: a kernel may be
+// scheduled while the previous kernel in the stream is still running, does only set-up that
+// touches no global memory (shared memory, barriers, TMEM, tensor-map prefetch), then waits in
+// pdl_wait() until the previous grid has completed and its writes are visible.  Every global
+// read and write comes after pdl_wait(), so stream order is kept exactly; each kernel lets its
+// own successor launch early with pdl_launch_dependents().  Without a programmatic predecessor
+// (first kernel, other work before it) the wait returns at once.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 // ------------------------------------------------------------------ small utilities

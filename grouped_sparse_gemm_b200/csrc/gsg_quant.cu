@@ -25,6 +25,8 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as
 __global__ void __launch_bounds__(kQuantThreads)
 act_amax_kernel(const uint16_t* __restrict__ X, long long n8, float* __restrict__ partial, int* status) {
   __shared__ float red[kQuantThreads / 32];
+  pdl_launch_dependents();
+  pdl_wait();
   float mx = 0.0f;
   bool finite = true;
   const uint4* X4 = reinterpret_cast<const uint4*>(X);
@@ -92,6 +94,8 @@ __global__ void __launch_bounds__(kQuantMainThreads)
 act_quant_kernel(QuantParams p) {
   __shared__ float red[kQuantMainThreads / 32];
   __shared__ float s_sh;
+  pdl_launch_dependents();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int units_per_row = p.K / 8;
   const long long U = (long long)p.T * units_per_row;   // a multiple of 32
@@ -215,8 +219,7 @@ cudaError_t launch_quant(const uint16_t* X, int T, int K, int sf, const int32_t*
   const long long n = (long long)T * K;
   int P = quant_partials(n);
   if (s_in == nullptr && n > 0) {
-    act_amax_kernel<<<P, kQuantThreads, 0, stream>>>(X, n / 8, partial, status);
-    cudaError_t err = cudaGetLastError();
+    cudaError_t err = launch_pdl(act_amax_kernel, P, kQuantThreads, 0, stream, X, n / 8, partial, status);
     if (err != cudaSuccess) return err;
   }
   if (n == 0) P = 0;  // no data: the quant kernel folds zero partials -> amax 0 -> s_x = 1
@@ -229,8 +232,7 @@ cudaError_t launch_quant(const uint16_t* X, int T, int K, int sf, const int32_t*
   long long blocks = ((units > pad ? units : pad) + kQuantMainThreads - 1) / kQuantMainThreads;
   if (blocks < 1) blocks = 1;
   if (blocks > (long long)num_sms * 16) blocks = (long long)num_sms * 16;
-  act_quant_kernel<<<(unsigned)blocks, kQuantMainThreads, 0, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(act_quant_kernel, (unsigned)blocks, kQuantMainThreads, 0, stream, p);
 }
 
 }  // namespace gsg

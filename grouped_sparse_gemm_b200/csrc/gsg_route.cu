@@ -136,10 +136,12 @@ route_single_kernel(const int32_t* __restrict__ ids, int R, int E, int32_t* off,
   extern __shared__ int hist[];  // [32][E]
   __shared__ int warp_sums[32];
   __shared__ int total;
+  pdl_launch_dependents();
   for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) hist[i] = 0;
   const int warp = threadIdx.x >> 5;
   int f0, f1;
   warp_run<1>(0, R, f0, f1);
+  pdl_wait();
   int x[1];
   unsigned m[1];
   warp_load_ids<1>(ids, f0, f1, E, x, status);
@@ -170,7 +172,9 @@ template <int kPer>
 __global__ void __launch_bounds__(kRouteThreads)
 route_hist_kernel(const int32_t* __restrict__ ids, int R, int E, int* ws_hist, int* status) {
   extern __shared__ int hist[];
+  pdl_launch_dependents();
   for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) hist[i] = 0;
+  pdl_wait();
   const int c0 = blockIdx.x * 1024 * kPer, c1 = min(c0 + 1024 * kPer, R);
   int f0, f1;
   warp_run<kPer>(c0, c1, f0, f1);
@@ -192,6 +196,8 @@ __global__ void __launch_bounds__(kRouteThreads)
 route_scan_kernel(const int* ws_hist, int nchunks, int E, int32_t* off, int* ws_base) {
   __shared__ int warp_sums[32];
   __shared__ int total;
+  pdl_launch_dependents();
+  pdl_wait();
   const int e = threadIdx.x;
   int tot = 0;
   if (e < E)
@@ -219,6 +225,8 @@ route_scatter_kernel(const int32_t* __restrict__ ids, int R, int E, const int* w
   extern __shared__ int hist[];
   __shared__ int warp_sums[32];
   __shared__ int total;
+  pdl_launch_dependents();
+  pdl_wait();
   int chunk_base = 0;
   if (kSelfScan) {
     // expert e's first row in this chunk: rows of experts < e, then of earlier chunks
@@ -291,22 +299,26 @@ cudaError_t launch_route(const int32_t* ids, int R, int E, int32_t* off, int32_t
   const size_t smem = (size_t)32 * E * sizeof(int);
   const int nc = route_chunks(R, E);
   if (nc <= 1) {
-    route_single_kernel<<<1, kRouteThreads, smem, stream>>>(ids, R, E, off, perm_src, inv_perm, status);
-    return cudaGetLastError();
+    return launch_pdl(route_single_kernel, 1, kRouteThreads, smem, stream, ids, R, E, off, perm_src, inv_perm,
+                      status);
   }
   int* ws_hist = static_cast<int*>(ws);
   int* ws_base = ws_hist + (size_t)nc * E;
+  cudaError_t e;
   if (route_chunk_size(R, E) == 1024) {
-    route_hist_kernel<1><<<nc, kRouteThreads, smem, stream>>>(ids, R, E, ws_hist, status);
-    route_scatter_kernel<1, true><<<nc, kRouteThreads, smem, stream>>>(ids, R, E, ws_hist, nc, off, perm_src,
-                                                                       inv_perm);
+    e = launch_pdl(route_hist_kernel<1>, nc, kRouteThreads, smem, stream, ids, R, E, ws_hist, status);
+    if (e == cudaSuccess)
+      e = launch_pdl(route_scatter_kernel<1, true>, nc, kRouteThreads, smem, stream, ids, R, E,
+                     (const int*)ws_hist, nc, off, perm_src, inv_perm);
   } else {
-    route_hist_kernel<8><<<nc, kRouteThreads, smem, stream>>>(ids, R, E, ws_hist, status);
-    route_scan_kernel<<<1, kRouteThreads, 0, stream>>>(ws_hist, nc, E, off, ws_base);
-    route_scatter_kernel<8, false><<<nc, kRouteThreads, smem, stream>>>(ids, R, E, ws_base, nc, off, perm_src,
-                                                                        inv_perm);
+    e = launch_pdl(route_hist_kernel<8>, nc, kRouteThreads, smem, stream, ids, R, E, ws_hist, status);
+    if (e == cudaSuccess)
+      e = launch_pdl(route_scan_kernel, 1, kRouteThreads, 0, stream, (const int*)ws_hist, nc, E, off, ws_base);
+    if (e == cudaSuccess)
+      e = launch_pdl(route_scatter_kernel<8, false>, nc, kRouteThreads, smem, stream, ids, R, E,
+                     (const int*)ws_base, nc, off, perm_src, inv_perm);
   }
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace gsg

@@ -16,6 +16,8 @@ __global__ void __launch_bounds__(kUnpermThreads)
 unpermute_kernel(const uint16_t* __restrict__ Y, const int32_t* __restrict__ inv_perm,
                  const float* __restrict__ gates, int T, int k, int N, int R, uint16_t* __restrict__ out,
                  int* status) {
+  pdl_launch_dependents();
+  pdl_wait();
   const unsigned n8 = (unsigned)N / 8u;
   const unsigned total = (unsigned)T * n8;   // T * N / 8 < 2^31 is checked on the host
   for (unsigned i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
@@ -68,9 +70,8 @@ cudaError_t launch_unpermute(const uint16_t* Y, const int32_t* inv_perm, const f
   if (total == 0) return cudaSuccess;
   long long blocks = (total + kUnpermThreads - 1) / kUnpermThreads;
   if (blocks > (long long)num_sms * 16) blocks = (long long)num_sms * 16;
-  unpermute_kernel<<<(unsigned)blocks, kUnpermThreads, 0, stream>>>(Y, inv_perm, gates, T, k, N, T * k,
-                                                                    out, status);
-  return cudaGetLastError();
+  return launch_pdl(unpermute_kernel, (unsigned)blocks, kUnpermThreads, 0, stream, Y, inv_perm, gates, T, k, N,
+                    T * k, out, status);
 }
 
 }  // namespace gsg
