@@ -8,9 +8,10 @@
 //
 // One CTA per SM, 352 threads (11 warps), warp-specialised around one shared-memory ring whose
 // stages hold 256 to 768 logical K of one tile (weights, activation codes and both scales):
-//   warp 0      weight producer: one bulk copy per stage of the interleaved packed weight blocks.
-//   warp 2      activation producer: tensor-map TMA boxes (128B swizzle) of only the token rows the
-//               tile holds, and one 3-D TMA box of the activation scale atoms.
+//   warp 0      weight producer: one bulk copy per stage of the interleaved packed weight blocks and
+//               one 3-D TMA box of the activation scale atoms.
+//   warp 2      activation producer: tensor-map TMA boxes (128B swizzle, 64 or 32 rows) of only the
+//               token rows the tile holds.
 //   warps 7..10 scale/metadata loaders, one per TMEM lane quadrant: read the stage's metadata and
 //               scale atoms from shared memory and tcgen05.st them into one of three TMEM sets.
 //   warp 1      TMEM owner and MMA issuer: per stage only tcgen05.mma(.sp) kind::mxf4nvf4
@@ -277,7 +278,8 @@ struct Geo {
 
 template <bool kSparse, int kBN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ CUtensorMap tmap_sfb,
+grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ CUtensorMap tmap_b64,
+                    const __grid_constant__ CUtensorMap tmap_sfb,
                     const GemmParams p) {
   using G = Geo<kSparse, kBN>;
   extern __shared__ uint8_t smem_raw[];
@@ -310,6 +312,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
   pdl_launch_dependents();
   if (warp == 2 && lane == 0) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_b)) : "memory");
+    if (kBN >= 64) asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_b64)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_sfb)) : "memory");
   }
   if (threadIdx.x == 0) {
@@ -391,7 +394,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
       const TileDesc c = my_tile(j, ttab, p.tcap, pref, offs, E, kBN);
       const uint8_t* wsrc = p.w_packed + ((size_t)c.e * NT + c.nt) * KC * G::kCB;
       const int r0 = c.r0;
-      const int nbox = (c.valid + G::kBoxH - 1) / G::kBoxH;
+      // token rows to fetch: whole 32-row boxes (BN <= 32: one box of BN rows), as few 64-row
+      // boxes as possible for the larger tiles -- every TMA instruction costs the issuing warp
+      const int rows = (c.valid + G::kBoxH - 1) / G::kBoxH * G::kBoxH;
+      const int n64 = kBN >= 64 ? rows / 64 : 0;
+      const int n32 = (rows - 64 * n64) / G::kBoxH;
       bool ok = true;
       for (int kc = 0; kc < KC; kc += G::kCPS) {
         const int nch = KC - kc >= G::kCPS ? G::kCPS : KC - kc;
@@ -399,14 +406,20 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
         const uint32_t st = sbase + (uint32_t)s * G::kStage;
         const uint32_t fb = full_bar(s);
         if (wprod) {
-          mbar_arrive_expect_tx(fb, (uint32_t)(nch * G::kCB));
+          // weights (+ metadata + weight scales) and the activation scale atoms: the activation
+          // producer issues one TMA per box already
+          mbar_arrive_expect_tx(fb, (uint32_t)(nch * G::kCB + G::kKbps * 512));
           bulk_g2s(st + G::kOffW, wsrc + (size_t)kc * G::kCB, nch * G::kCB, fb);
-        } else {
-          mbar_arrive_expect_tx(fb, (uint32_t)(nch * nbox * G::kBoxH * 128 + G::kKbps * 512));
-          for (int ch = 0; ch < nch; ++ch)
-            for (int b = 0; b < nbox; ++b)
-              tma_load_2d(st + ch * G::kBChunk + b * G::kBoxH * 128, &tmap_b, (kc + ch) * 128, r0 + b * G::kBoxH, fb);
           tma_load_3d(st + G::kOffSFB, &tmap_sfb, 0, r0, kc * G::kKbPerChunk, fb);
+        } else {
+          mbar_arrive_expect_tx(fb, (uint32_t)(nch * rows * 128));
+          for (int ch = 0; ch < nch; ++ch) {
+            for (int b = 0; b < n64; ++b)
+              tma_load_2d(st + ch * G::kBChunk + b * 64 * 128, &tmap_b64, (kc + ch) * 128, r0 + b * 64, fb);
+            for (int b = 0; b < n32; ++b)
+              tma_load_2d(st + ch * G::kBChunk + (64 * n64 + b * G::kBoxH) * 128, &tmap_b, (kc + ch) * 128,
+                          r0 + 64 * n64 + b * G::kBoxH, fb);
+          }
         }
         ++issued;
         if (++s == S) { s = 0; ph ^= 1u; }
@@ -690,12 +703,12 @@ cudaError_t gemm_set_smem_attrs() {
 
 template <bool kSparse>
 static cudaError_t launch_bn(int BN, int grid, size_t smem, cudaStream_t stream, const CUtensorMap& tb,
-                             const CUtensorMap& ts, const GemmParams& p) {
+                             const CUtensorMap& tb64, const CUtensorMap& ts, const GemmParams& p) {
   switch (BN) {
-    case 16: return launch_pdl(grouped_gemm_kernel<kSparse, 16>, grid, kGemmThreads, smem, stream, tb, ts, p);
-    case 32: return launch_pdl(grouped_gemm_kernel<kSparse, 32>, grid, kGemmThreads, smem, stream, tb, ts, p);
-    case 64: return launch_pdl(grouped_gemm_kernel<kSparse, 64>, grid, kGemmThreads, smem, stream, tb, ts, p);
-    default: return launch_pdl(grouped_gemm_kernel<kSparse, 128>, grid, kGemmThreads, smem, stream, tb, ts, p);
+    case 16: return launch_pdl(grouped_gemm_kernel<kSparse, 16>, grid, kGemmThreads, smem, stream, tb, tb64, ts, p);
+    case 32: return launch_pdl(grouped_gemm_kernel<kSparse, 32>, grid, kGemmThreads, smem, stream, tb, tb64, ts, p);
+    case 64: return launch_pdl(grouped_gemm_kernel<kSparse, 64>, grid, kGemmThreads, smem, stream, tb, tb64, ts, p);
+    default: return launch_pdl(grouped_gemm_kernel<kSparse, 128>, grid, kGemmThreads, smem, stream, tb, tb64, ts, p);
   }
 }
 
@@ -715,14 +728,16 @@ int launch_gemm(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, co
   const int kbps = g.cps * (sparse ? 2 : 4);
   const int rcap = R + kActScalePadRows;
   const int KBa = K / (sparse ? 128 : 64);
-  CUtensorMap tb, ts;
-  {
+  CUtensorMap tb, tb64, ts;
+  // activation codes [R][K/2]: boxes of 128 bytes x box_h rows, and (token tiles >= 64) x 64 rows
+  for (int m = 0; m < 2; ++m) {
+    if (m == 1 && g.BN < 64) { tb64 = tb; break; }
     cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)R};
     cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
-    cuuint32_t box[2] = {128u, (cuuint32_t)box_h};
+    cuuint32_t box[2] = {128u, (cuuint32_t)(m == 0 ? box_h : 64)};
     cuuint32_t estr[2] = {1u, 1u};
-    if (enc(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a_codes), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    if (enc(m == 0 ? &tb : &tb64, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(a_codes), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return 2;
   }
@@ -742,8 +757,8 @@ int launch_gemm(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, co
   p.w_scale = w_scale; p.off = off; p.Y = Y; p.status = status;
   p.E = E; p.N = N; p.K = K; p.R = R; p.y_f32 = y_f32; p.rcap = rcap;
   p.stages = g.stages; p.nacc = g.nacc; p.tcap = g.tcap;
-  const cudaError_t e = sparse ? launch_bn<true>(g.BN, num_sms, g.smem, stream, tb, ts, p)
-                               : launch_bn<false>(g.BN, num_sms, g.smem, stream, tb, ts, p);
+  const cudaError_t e = sparse ? launch_bn<true>(g.BN, num_sms, g.smem, stream, tb, tb64, ts, p)
+                               : launch_bn<false>(g.BN, num_sms, g.smem, stream, tb, tb64, ts, p);
   return e == cudaSuccess ? 0 : 1;
 }
 
