@@ -547,6 +547,103 @@ def gsg_token_tile(max_rows: int, R: int, E: int) -> int:
     return 128 if R >= 64 * E else 64
 
 
+# ------------------------------------------------------------------ G x N sweep
+SWEEP_SHAPES = {            # expert projection shapes: (K, N)
+    "30b_up": (2048, 1536), "30b_down": (768, 2048), "1t_up": (7168, 4096), "1t_down": (2048, 7168)}
+
+
+class Energy:
+    """Board energy counter through NVML (read only); None when NVML is not available."""
+
+    def __init__(self, index: int):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv, self.h = pynvml, pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.nv.nvmlDeviceGetTotalEnergyConsumption(self.h)
+        except Exception:
+            self.nv = None
+
+    def mj(self):
+        return None if self.nv is None else float(self.nv.nvmlDeviceGetTotalEnergyConsumption(self.h))
+
+
+def run_sweep(args, local):
+    """Sparse GEMM vs the dense-NVFP4 control over expert-group count G x tokens per expert, for
+    the 30B-A3B and 1T expert shapes (weights N(0, 0.02), activations N(0, 1), every expert with
+    the same token count).  Per point: in-graph time after an L2 flush, and energy per call from
+    the board's energy counter over ~0.2 s of back-to-back replays.  One JSON line per point."""
+    dev = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(dev)
+    gsg.load_library()
+    L = gsg.lib()
+    u8 = dict(dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, **u8)
+    energy = Energy(local)
+    Gs = [int(x) for x in args.sweep_g.split(",")]
+    Ns = [int(x) for x in args.sweep_n.split(",")]
+    shapes = args.sweep_shapes.split(",")
+    reps = max(10, min(args.steps, 200))
+    for shape in shapes:
+        K, N = SWEEP_SHAPES[shape]
+        Gmax = max(Gs)
+        pw = gsg.PackedSparseWeights(packed=torch.empty(L.gsg_sparse_packed_bytes(Gmax, N, K), **u8),
+                                     w_scale=torch.empty(Gmax, dtype=torch.float32, device=dev), E=Gmax, N=N, K=K)
+        pd = gsg.PackedDenseWeights(packed=torch.empty(L.gsg_dense_packed_bytes(Gmax, N, K), **u8),
+                                    w_scale=torch.empty(Gmax, dtype=torch.float32, device=dev), E=Gmax, N=N, K=K)
+        ws = torch.empty(max(gsg.workspace_size(gsg.OP_PACK_SPARSE, 1, N, K), 16), **u8)
+        cfg_w = inputs.custom_config("sweep", E=Gmax, K=K, N=N, T=1, top_k=1, w_sigma=0.02)
+        for e in range(Gmax):
+            We = inputs.expert_weight(cfg_w, e, str(dev))[None]
+            gsg.pack_sparse_nvfp4(We, out=pw.expert(e), workspace=ws)
+            gsg.pack_dense_nvfp4(We, out=pd.expert(e), workspace=ws)
+            del We
+        sp_per, dn_per = pw.packed.numel() // Gmax, pd.packed.numel() // Gmax
+        for G in Gs:
+            pwG = gsg.PackedSparseWeights(pw.packed[:G * sp_per], pw.w_scale[:G], G, N, K)
+            pdG = gsg.PackedDenseWeights(pd.packed[:G * dn_per], pd.w_scale[:G], G, N, K)
+            for nt in Ns:
+                R = G * nt
+                X = inputs.random_bf16((R, K), seed=7, device=str(dev))
+                off = torch.arange(0, R + 1, nt, dtype=torch.int32, device=dev)
+                qa32 = gsg.quantize_act_nvfp4(X, 32)
+                qa16 = gsg.quantize_act_nvfp4(X, 16)
+                Ys = torch.empty(R, N, dtype=torch.bfloat16, device=dev)
+                Yd = torch.empty(R, N, dtype=torch.bfloat16, device=dev)
+                run_s = lambda: gsg.grouped_sparse_gemm(qa32, pwG, off, nt, out=Ys)
+                run_d = lambda: gsg.grouped_dense_gemm(qa16, pdG, off, nt, out=Yd)
+                line = {"sweep": shape, "K": K, "N": N, "G": G, "tokens_per_expert": nt, "R": R}
+                for tag, fn, wbytes in (("sparse", run_s, G * sp_per), ("dense", run_d, G * dn_per)):
+                    gt = capture_timed(fn)
+                    for _ in range(3):
+                        flush.fill_(1)
+                        gt[0].replay()
+                    ms, _ = timed_graph_ms(gt, reps, flush, 1)
+                    e_call = None
+                    e0 = energy.mj()
+                    if e0 is not None:
+                        n = max(20, int(0.2 / max(ms * 1e-3, 1e-6)))
+                        torch.cuda.synchronize()
+                        e0 = energy.mj()
+                        for _ in range(n):
+                            gt[0].replay()
+                        torch.cuda.synchronize()
+                        e_call = (energy.mj() - e0) / n
+                    act = R * K // 2 + R * K // (32 if tag == "sparse" else 16)
+                    line[tag] = {"us": ms * 1e3, "tflops": 2.0 * R * N * K / (ms * 1e-3) / 1e12,
+                                 "hbm_gbs": (wbytes + act + R * N * 2) / (ms * 1e-3) / 1e9,
+                                 "mj_per_call": e_call}
+                    del gt
+                line["sparse_speedup"] = line["dense"]["us"] / line["sparse"]["us"]
+                st = gsg.get_device_status()
+                if st != 0:
+                    raise RuntimeError(f"device status {st} in the sweep")
+                print(json.dumps(line), flush=True)
+                del X, qa32, qa16, Ys, Yd
+        del pw, pd
+        torch.cuda.empty_cache()
+
+
 def run_profile_steps(args, local):
     """The step graph replayed warmup + steps times and nothing else, so that a profiler's launch
     list holds only the step's kernels in step order."""
@@ -578,6 +675,11 @@ def main():
     ap.add_argument("--quick", action="store_true", help="skip e2e, dense control and CPU baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-experts", type=int, default=24)
+    ap.add_argument("--sweep", action="store_true",
+                    help="G x N sweep of the sparse GEMM against the dense control (one JSON line per point)")
+    ap.add_argument("--sweep-shapes", default="30b_up,30b_down,1t_up,1t_down")
+    ap.add_argument("--sweep-g", default="1,8,32,128")
+    ap.add_argument("--sweep-n", default="1,8,32,128,512")
     ap.add_argument("--profile-steps", action="store_true",
                     help="for profiler launch lists: only replay the step graph (warmup + steps), print no bench line")
     args = ap.parse_args()
@@ -589,6 +691,8 @@ def main():
             run_reference(args, world, rank)
         elif args.profile_steps:
             run_profile_steps(args, local)
+        elif args.sweep:
+            run_sweep(args, local)
         else:
             run_ours(args, world, rank, local)
     finally:

@@ -25,7 +25,8 @@ __all__ = [
     "PackedSparseWeights", "PackedDenseWeights", "Routing", "QuantizedActivations",
     "pack_sparse_nvfp4", "pack_dense_nvfp4", "moe_route_permute", "moe_route_permute_noalloc",
     "quantize_act_nvfp4",
-    "grouped_sparse_gemm", "grouped_dense_gemm", "unpermute_scale", "get_device_status",
+    "grouped_sparse_gemm", "grouped_sparse_gemm_swiglu", "grouped_dense_gemm", "unpermute_scale",
+    "get_device_status",
     "act_scales_bytes", "workspace_size", "OP_PACK_SPARSE", "OP_PACK_DENSE", "OP_ROUTE",
     "OP_QUANTIZE", "OP_GEMM", "EXPORTED_SYMBOLS",
 ]
@@ -40,7 +41,7 @@ EXPORTED_SYMBOLS = [
     "gsg_pack_sparse_nvfp4", "gsg_pack_dense_nvfp4", "gsg_moe_route_permute",
     "gsg_quantize_act_nvfp4", "gsg_grouped_sparse_gemm", "gsg_grouped_dense_gemm",
     "gsg_unpermute_scale", "gsg_get_device_status", "gsg_status_string", "gsg_version",
-    "gsg_moe_route_permute_noalloc",
+    "gsg_moe_route_permute_noalloc", "gsg_grouped_sparse_gemm_swiglu",
 ]
 
 _STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported shape", -3: "CUDA error",
@@ -89,6 +90,7 @@ def load_library(build_if_missing: bool = False) -> ctypes.CDLL:
         "gsg_status_string": (ctypes.c_char_p, [i]),
         "gsg_version": (i, []),
         "gsg_moe_route_permute_noalloc": (i, [vp, i, i, i, vp, vp, vp, vp]),
+        "gsg_grouped_sparse_gemm_swiglu": (i, [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -302,6 +304,27 @@ def grouped_sparse_gemm(act: QuantizedActivations, w: PackedSparseWeights, offse
     _check("gsg_grouped_sparse_gemm", lib().gsg_grouped_sparse_gemm(
         _ptr(act.codes), _ptr(act.scales), _ptr(act.x_scale), _ptr(w.packed), _ptr(w.w_scale),
         _ptr(offsets), w.E, w.N, w.K, act.R, max_rows_per_expert, _ptr(out), ydt, _stream(stream)))
+    return out
+
+
+def grouped_sparse_gemm_swiglu(act: QuantizedActivations, w: PackedSparseWeights, offsets: torch.Tensor,
+                               h_scale: torch.Tensor, max_rows_per_expert: int = -1,
+                               out: Optional[QuantizedActivations] = None, stream=None) -> QuantizedActivations:
+    """Up-projection (fused gate|up weights [2I, K]) with SwiGLU and NVFP4 quantization of
+    h = silu(gate) * up in the epilogue (gsg_grouped_sparse_gemm_swiglu): returns h's codes and
+    scales, ready as the down-projection's activations (tensor scale h_scale, fp32 [1])."""
+    assert act.sf_block == 32 and act.K == w.K and w.N % 256 == 0
+    _need_cuda(act.codes, act.scales, offsets, h_scale)
+    I = w.N // 2
+    dev = act.codes.device
+    if out is None:
+        out = QuantizedActivations(codes=torch.empty(max(act.R, 1), I // 2, dtype=torch.uint8, device=dev),
+                                   scales=torch.empty(act_scales_bytes(act.R, I, 32), dtype=torch.uint8, device=dev),
+                                   x_scale=h_scale, R=act.R, K=I, sf_block=32)
+    _check("gsg_grouped_sparse_gemm_swiglu", lib().gsg_grouped_sparse_gemm_swiglu(
+        _ptr(act.codes), _ptr(act.scales), _ptr(act.x_scale), _ptr(w.packed), _ptr(w.w_scale),
+        _ptr(offsets), w.E, w.N, w.K, act.R, max_rows_per_expert, _ptr(h_scale), _ptr(out.codes),
+        _ptr(out.scales), _stream(stream)))
     return out
 
 

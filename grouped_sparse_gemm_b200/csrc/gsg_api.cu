@@ -198,6 +198,33 @@ gsg_status_t gsg_grouped_dense_gemm(const uint8_t* a_codes, const uint8_t* a_sca
                      max_rows_per_expert, Y, y_dtype, stream);
 }
 
+gsg_status_t gsg_grouped_sparse_gemm_swiglu(const uint8_t* a_codes, const uint8_t* a_scales,
+                                            const float* x_tensor_scale, const uint8_t* w_packed,
+                                            const float* w_tensor_scale, const int32_t* expert_offsets, int E,
+                                            int N2, int K, int R, int max_rows_per_expert,
+                                            const float* h_tensor_scale, uint8_t* h_codes, uint8_t* h_scales,
+                                            void* stream) {
+  if (R < 0) return GSG_ERR_INVALID_ARG;
+  if (!weight_shape_ok(E, N2, K) || N2 % 256 != 0 || !gsg::gemm_supported(E)) return GSG_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)R > (1ll << 30)) return GSG_ERR_UNSUPPORTED_SHAPE;
+  if (!expert_offsets || !w_packed || !w_tensor_scale || !x_tensor_scale || !h_tensor_scale || !h_scales)
+    return GSG_ERR_INVALID_ARG;
+  if (!aligned16(h_scales) || !aligned16(w_packed)) return GSG_ERR_INVALID_ARG;
+  DeviceState* d = nullptr;
+  gsg_status_t st = device_state(&d);
+  if (st != GSG_OK) return st;
+  if (R == 0) {   // nothing routed: only the (all padding) scale entries to clear
+    const size_t n = gsg_act_scales_bytes(0, N2 / 2, 32);
+    return from_cuda(cudaMemsetAsync(h_scales, 0, n, as_stream(stream)));
+  }
+  if (!a_codes || !a_scales || !h_codes) return GSG_ERR_INVALID_ARG;
+  if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(h_codes)) return GSG_ERR_INVALID_ARG;
+  const int rc = gsg::launch_gemm(true, a_codes, a_scales, x_tensor_scale, w_packed, w_tensor_scale, expert_offsets,
+                                  E, N2, K, R, max_rows_per_expert, h_codes, 0, d->status, d->num_sms,
+                                  as_stream(stream), h_scales, h_tensor_scale);
+  return rc == 0 ? GSG_OK : GSG_ERR_CUDA;
+}
+
 gsg_status_t gsg_unpermute_scale(const uint16_t* Y, const int32_t* inv_perm, const float* gates, int T, int k, int N,
                                  uint16_t* out, void* stream) {
   if (T < 0 || k < 1 || N < 8 || N % 8 != 0) return GSG_ERR_INVALID_ARG;

@@ -46,10 +46,12 @@ struct GemmParams {
   const uint8_t* w_packed;
   const float* w_scale;
   const int32_t* off;
-  void* Y;
+  void* Y;                 // Y [R][N] (bf16 or fp32); with the SwiGLU epilogue: h codes [R][N/4]
   int* status;
   int E, N, K, R, y_f32, rcap;
   int stages, nacc, tcap;
+  uint8_t* h_scales;       // SwiGLU epilogue: h scales, quad layout [N/256][R+256][4][4]
+  const float* h_scale;    // SwiGLU epilogue: tensor scale of h
 };
 
 // ------------------------------------------------------------------ PTX wrappers
@@ -251,39 +253,43 @@ __device__ __forceinline__ TileDesc my_tile(int j, const int4* table, int tcap, 
   return decode_tile(blockIdx.x + j * (int)gridDim.x, pref, offs, E, BN);
 }
 
-// Compile-time stage geometry of one (sparse/dense, token tile) instantiation.
-template <bool kSparse, int kBN>
+// Compile-time stage geometry of one (sparse/dense, token tile, SwiGLU) instantiation.  With the
+// SwiGLU epilogue a tile holds two weight n-tiles (gate rows nt*128.., up rows N/2 + nt*128..) that
+// share the activation tile: two MMAs per k-block into two accumulators side by side.
+template <bool kSparse, int kBN, bool kGLU = false>
 struct Geo {
+  static constexpr int kNT = kGLU ? 2 : 1;                         // weight n-tiles per tile
   static constexpr int kKbLogical = kSparse ? 128 : 64;            // logical K per MMA
   static constexpr int kKbPerChunk = kChunkK / kKbLogical;         // 2 sparse, 4 dense
   // 256-wide K chunks per stage: short token tiles take longer stages (fewer waits per weight byte)
-  static constexpr int kCPS = kSparse ? (kBN <= 32 ? 3 : 2) : (kBN <= 32 ? 2 : 1);
-  static constexpr int kKbps = kCPS * kKbPerChunk;                 // MMAs per stage
+  static constexpr int kCPS = kGLU ? 2 : kSparse ? (kBN <= 32 ? 3 : 2) : (kBN <= 32 ? 2 : 1);
+  static constexpr int kKbps = kCPS * kKbPerChunk;                 // k-blocks per stage
   static constexpr int kCB = kSparse ? kSparseChunkBytes : kDenseChunkBytes;   // packed chunk block
   static constexpr int kCBMeta = 8192;                             // metadata offset in a chunk block
   static constexpr int kCBScale = kSparse ? 10240 : 16384;         // scale atoms offset in a chunk block
   static constexpr int kBChunk = kBN * 128;                        // activation codes per chunk
   static constexpr int kOffW = kCPS * kBChunk;                     // stage layout: B chunks | W blocks | SFB
-  static constexpr int kOffSFB = kOffW + kCPS * kCB;
+  static constexpr int kOffSFB = kOffW + kNT * kCPS * kCB;
   static constexpr int kStage = (kOffSFB + kKbps * 512 + 1023) / 1024 * 1024;
-  static constexpr int kMetaCols = kSparse ? 4 * kCPS : 0;         // TMEM set: meta | SFA | SFB
+  static constexpr int kMetaCols = kSparse ? 4 * kCPS * kNT : 0;   // TMEM set: meta | SFA | SFB
   static constexpr int kColSFA = kMetaCols;
-  static constexpr int kColSFB = kMetaCols + 4 * kKbps;
-  static constexpr int kSetUsed = kMetaCols + 8 * kKbps;
+  static constexpr int kColSFB = kMetaCols + 4 * kKbps * kNT;
+  static constexpr int kSetUsed = kColSFB + 4 * kKbps;
   static constexpr uint32_t kBStep = kSparse ? 64 : 32;            // B bytes per row per MMA
   static constexpr int kBoxH = kBN < 32 ? kBN : 32;                // token rows per TMA box
   static constexpr int kAccStride = kBN < 32 ? 32 : kBN;
   static_assert(kSetUsed <= (int)kSetCols, "TMEM set too small");
 };
 
-template <bool kSparse, int kBN>
+template <bool kSparse, int kBN, bool kGLU>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ CUtensorMap tmap_b64,
                     const __grid_constant__ CUtensorMap tmap_sfb,
                     const GemmParams p) {
-  using G = Geo<kSparse, kBN>;
+  using G = Geo<kSparse, kBN, kGLU>;
   extern __shared__ uint8_t smem_raw[];
-  const int E = p.E, NT = p.N / kTileN, KC = p.K / kChunkK;
+  // NT: weight n-tiles; tiles run over NT / kNT columns (the gate n-tiles with the SwiGLU epilogue)
+  const int E = p.E, NT = p.N / kTileN, NTt = NT / G::kNT, KC = p.K / kChunkK;
   const int S = p.stages, NACC = p.nacc;
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + (size_t)S * G::kStage);
@@ -340,16 +346,24 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
     offs[i] = v;
     if (i < E) wsc[i] = __ldg(p.w_scale + i);
   }
+  if (kGLU) {
+    // h scale entries that refer to rows >= R (no tile writes them): zero, shared by the CTAs
+    const int r_lo = p.R > 96 ? p.R - 96 : 0, span = p.rcap - r_lo, kbh = p.N / 256;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < kbh * span * 4; i += gridDim.x * blockDim.x) {
+      const int cc = i & 3, rest = i >> 2, rr = r_lo + rest % span, kb = rest / span;
+      if (rr + 32 * cc >= p.R) *reinterpret_cast<uint32_t*>(p.h_scales + ((size_t)kb * p.rcap + rr) * 16 + cc * 4) = 0u;
+    }
+  }
   __syncthreads();
   {
-    // chunked exclusive scan of tiles_e = ceil(rows_e / BN) * NT over E experts
+    // chunked exclusive scan of tiles_e = ceil(rows_e / BN) * NTt over E experts
     const int per = (E + kGemmThreads - 1) / kGemmThreads;
     const int e0 = threadIdx.x * per, e1 = min(e0 + per, E);
     int local = 0;
     for (int e = e0; e < e1; ++e) {
       int rows = offs[e + 1] - offs[e];
       if (rows < 0) { bad = true; rows = 0; }
-      local += ((rows + kBN - 1) / kBN) * NT;
+      local += ((rows + kBN - 1) / kBN) * NTt;
     }
     int incl = local;
 #pragma unroll
@@ -367,7 +381,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
       pref[e] = run;
       int rows = offs[e + 1] - offs[e];
       if (rows < 0) rows = 0;
-      run += ((rows + kBN - 1) / kBN) * NT;
+      run += ((rows + kBN - 1) / kBN) * NTt;
     }
     if (threadIdx.x == kGemmThreads - 1) pref[E] = before + incl;
   }
@@ -393,6 +407,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
     for (int j = 0; j < n_my && !*abort_flag; ++j) {
       const TileDesc c = my_tile(j, ttab, p.tcap, pref, offs, E, kBN);
       const uint8_t* wsrc = p.w_packed + ((size_t)c.e * NT + c.nt) * KC * G::kCB;
+      const uint8_t* wsrc_up = wsrc + (size_t)(NT / 2) * KC * G::kCB;   // SwiGLU: the matching up n-tile
       const int r0 = c.r0;
       // token rows to fetch: whole 32-row boxes (BN <= 32: one box of BN rows), as few 64-row
       // boxes as possible for the larger tiles -- every TMA instruction costs the issuing warp
@@ -408,8 +423,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
         if (wprod) {
           // weights (+ metadata + weight scales) and the activation scale atoms: the activation
           // producer issues one TMA per box already
-          mbar_arrive_expect_tx(fb, (uint32_t)(nch * G::kCB + G::kKbps * 512));
+          mbar_arrive_expect_tx(fb, (uint32_t)(G::kNT * nch * G::kCB + G::kKbps * 512));
           bulk_g2s(st + G::kOffW, wsrc + (size_t)kc * G::kCB, nch * G::kCB, fb);
+          if (kGLU) bulk_g2s(st + G::kOffW + G::kCPS * G::kCB, wsrc_up + (size_t)kc * G::kCB, nch * G::kCB, fb);
           tma_load_3d(st + G::kOffSFB, &tmap_sfb, 0, r0, kc * G::kKbPerChunk, fb);
         } else {
           mbar_arrive_expect_tx(fb, (uint32_t)(nch * rows * 128));
@@ -456,17 +472,25 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
         uint32_t r[G::kSetUsed];
         if (kSparse) {
 #pragma unroll
-          for (int ch = 0; ch < G::kCPS; ++ch)
-            if (ch < nch)
-              lds128(st + G::kOffW + ch * G::kCB + G::kCBMeta + row * 16, r[4 * ch], r[4 * ch + 1], r[4 * ch + 2],
-                     r[4 * ch + 3]);
+          for (int t = 0; t < G::kNT; ++t)
+#pragma unroll
+            for (int ch = 0; ch < G::kCPS; ++ch)
+              if (ch < nch) {
+                const int m = 4 * (t * G::kCPS + ch);
+                lds128(st + G::kOffW + (t * G::kCPS + ch) * G::kCB + G::kCBMeta + row * 16, r[m], r[m + 1], r[m + 2],
+                       r[m + 3]);
+              }
         }
 #pragma unroll
         for (int kb = 0; kb < G::kKbps; ++kb) {
           if (kb < nch * G::kKbPerChunk) {
-            const uint32_t sfa = st + G::kOffW + (kb / G::kKbPerChunk) * G::kCB + G::kCBScale + (kb % G::kKbPerChunk) * 512;
-            lds128(sfa + lane * 16, r[G::kColSFA + 4 * kb], r[G::kColSFA + 4 * kb + 1],
-                   r[G::kColSFA + 4 * kb + 2], r[G::kColSFA + 4 * kb + 3]);
+#pragma unroll
+            for (int t = 0; t < G::kNT; ++t) {
+              const uint32_t sfa = st + G::kOffW + (t * G::kCPS + kb / G::kKbPerChunk) * G::kCB + G::kCBScale +
+                                   (kb % G::kKbPerChunk) * 512;
+              const int m = G::kColSFA + 4 * (t * G::kKbps + kb);
+              lds128(sfa + lane * 16, r[m], r[m + 1], r[m + 2], r[m + 3]);
+            }
             lds128(st + G::kOffSFB + kb * 512 + lane * 16, r[G::kColSFB + 4 * kb], r[G::kColSFB + 4 * kb + 1],
                    r[G::kColSFB + 4 * kb + 2], r[G::kColSFB + 4 * kb + 3]);
           }
@@ -492,7 +516,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
       const uint32_t idesc = make_idesc(kSparse, (c.valid + 15) & ~15);
       if (!wait_warp(acce_bar(acc), aph ^ 1u, abort_flag, p.status)) break;
       tc_fence_after();
-      const uint32_t d_tmem = tmem + kColAcc + (uint32_t)(acc * G::kAccStride);
+      const uint32_t d_tmem = tmem + kColAcc + (uint32_t)(acc * G::kNT * G::kAccStride);
       bool ok = true;
       for (int kc = 0; kc < KC; kc += G::kCPS) {
         const int nch = KC - kc >= G::kCPS ? G::kCPS : KC - kc;
@@ -510,15 +534,21 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
 #pragma unroll
             for (int h = 0; h < G::kKbPerChunk; ++h) {
               const int kbi = ch * G::kKbPerChunk + h;
-              const uint64_t adesc = smem_desc(st + G::kOffW + ch * G::kCB + 4096u * h, 128, 256, 0);
               const uint64_t bdesc = smem_desc(st + ch * G::kBChunk + G::kBStep * h, 16, 1024, 2);
               const uint32_t accum = (kc | ch | h) != 0 ? 1u : 0u;
-              if (kSparse)
-                tc_mma_sparse(d_tmem, adesc, bdesc, idesc, accum, tset + G::kColSFA + 4 * kbi,
-                              tset + G::kColSFB + 4 * kbi, tset + 2 * kbi);
-              else
-                tc_mma_dense(d_tmem, adesc, bdesc, idesc, accum, tset + G::kColSFA + 4 * kbi,
-                             tset + G::kColSFB + 4 * kbi);
+#pragma unroll
+              for (int t = 0; t < G::kNT; ++t) {
+                const uint64_t adesc =
+                    smem_desc(st + G::kOffW + (t * G::kCPS + ch) * G::kCB + 4096u * h, 128, 256, 0);
+                const uint32_t d = d_tmem + (uint32_t)(t * G::kAccStride);
+                const int kt = t * G::kKbps + kbi;
+                if (kSparse)
+                  tc_mma_sparse(d, adesc, bdesc, idesc, accum, tset + G::kColSFA + 4 * kt,
+                                tset + G::kColSFB + 4 * kbi, tset + 2 * kt);
+                else
+                  tc_mma_dense(d, adesc, bdesc, idesc, accum, tset + G::kColSFA + 4 * kt,
+                               tset + G::kColSFB + 4 * kbi);
+              }
             }
           }
         }
@@ -552,7 +582,49 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
       if (!wait_warp(accf_bar(acc), aph, abort_flag, p.status)) break;
       tc_fence_after();
       const float scale = __fmul_rn(sx, wsc[c.e]);
-      const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + kColAcc + (uint32_t)(acc * G::kAccStride);
+      const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + kColAcc + (uint32_t)(acc * G::kNT * G::kAccStride);
+      if constexpr (kGLU) {
+        // SwiGLU output preparation: lane = feature f of this warp's 32-feature block (the block
+        // the next GEMM's scales cover), h = silu(gate) * up in fp32, one NVFP4 block per token
+        // (block max over the warp), codes packed 8 lanes to a 32-bit word, scales into the quad
+        // layout (k-block nt, position q).
+        const float sh = __ldg(p.h_scale);
+        const float six_sh = __fmul_rn(6.0f, sh);
+        const int f0 = c.nt * kTileN + 32 * q;
+        const int hrow = p.N / 4;                 // bytes of h codes per row (N/2 features)
+        uint8_t* hc = static_cast<uint8_t*>(p.Y);
+        for (int c0 = 0; c0 < valid; c0 += 16) {
+          float g[16], u[16];
+          tc_ld_16(taddr + c0, g);
+          tc_ld_16(taddr + G::kAccStride + c0, u);
+          uint32_t scs[16];
+#pragma unroll
+          for (int t = 0; t < 16; ++t) {
+            const float gs = __fmul_rn(g[t], scale), us = __fmul_rn(u[t], scale);
+            const float hv = __fmul_rn(__fdiv_rn(gs, __fadd_rn(1.0f, expf(-gs))), us);
+            const float am = warp_max(fabsf(hv));
+            const BlockScale bs = block_scale_cvt(am, six_sh, sh);
+            scs[t] = bs.sc;
+            uint32_t w = e2m1_encode(__fmul_rn(hv, bs.inv)) << (4 * (lane & 7));
+            w |= __shfl_xor_sync(0xffffffffu, w, 1);
+            w |= __shfl_xor_sync(0xffffffffu, w, 2);
+            w |= __shfl_xor_sync(0xffffffffu, w, 4);
+            if ((lane & 7) == 0 && c0 + t < valid)
+              *reinterpret_cast<uint32_t*>(hc + (size_t)(r0 + c0 + t) * hrow + f0 / 2 + (lane >> 3) * 4) = w;
+          }
+          // quad scale entries (nt, row - 32c, c, q) of the 16 tokens: 64 single bytes, two per lane
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int idx = lane + 32 * k, t = idx >> 2, cc = idx & 3;
+            uint32_t sc = 0;
+#pragma unroll
+            for (int tt = 0; tt < 16; ++tt) sc = tt == t ? scs[tt] : sc;
+            const int row = r0 + c0 + t, rr = row - 32 * cc;
+            if (c0 + t < valid && rr >= 0)
+              p.h_scales[((size_t)c.nt * p.rcap + rr) * 16 + cc * 4 + q] = (uint8_t)sc;
+          }
+        }
+      } else {
       // Each 16-token chunk: TMEM lane (= output feature) -> registers, scale, transpose through
       // the warp's shared buffer into [token][32 features], then 16-byte stores of whole row
       // segments (64 B bf16 / 128 B fp32 per token).
@@ -597,6 +669,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
         }
         __syncwarp();
       }
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acce_bar(acc));
@@ -626,13 +699,14 @@ static int g_smem_limit = 232448 - 1024;
 
 // tcap: capacity of the per-CTA tile table (tiles beyond it are decoded on the fly); an upper
 // bound on a CTA's tiles is ceil((ceil(R/BN) + E) * NT / grid).
-static GemmPlan make_plan(bool sparse, int BN, int E, int tcap) {
+static GemmPlan make_plan(bool sparse, int BN, int E, int tcap, bool glu = false) {
   GemmPlan g;
   g.BN = BN;
   g.tcap = tcap;
-  g.cps = sparse ? (BN <= 32 ? 3 : 2) : (BN <= 32 ? 2 : 1);
+  const int nt = glu ? 2 : 1;   // weight n-tiles per tile (gate + up with the SwiGLU epilogue)
+  g.cps = glu ? 2 : sparse ? (BN <= 32 ? 3 : 2) : (BN <= 32 ? 2 : 1);
   const int kbps = g.cps * (sparse ? 2 : 4);
-  const int body = g.cps * BN * 128 + g.cps * (sparse ? kSparseChunkBytes : kDenseChunkBytes) + kbps * 512;
+  const int body = g.cps * BN * 128 + nt * g.cps * (sparse ? kSparseChunkBytes : kDenseChunkBytes) + kbps * 512;
   g.stage = (body + 1023) / 1024 * 1024;
   // everything but the stage ring and the tile table, at its largest
   const int fixed = 1024 + (2 * kMaxStages + kNSets + 2 * kMaxAcc + 1) * 8 + (int)sizeof(Ctl) + (3 * E + 2) * 4 +
@@ -641,7 +715,7 @@ static GemmPlan make_plan(bool sparse, int BN, int E, int tcap) {
   if (BN == 128 && budget > kStageBudget128) budget = kStageBudget128;
   g.stages = (budget - tcap * 16) / g.stage;
   if (g.stages > kMaxStages) g.stages = kMaxStages;
-  const int acc_stride = BN < 32 ? 32 : BN;
+  const int acc_stride = (BN < 32 ? 32 : BN) * nt;
   g.nacc = (int)((kTmemCols - kColAcc) / acc_stride);
   if (g.nacc > kMaxAcc) g.nacc = kMaxAcc;
   const int nbars = 2 * g.stages + kNSets + 2 * g.nacc + 1;
@@ -680,9 +754,10 @@ static EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-template <bool kSparse, int kBN>
+template <bool kSparse, int kBN, bool kGLU = false>
 static cudaError_t set_attr_one(int bytes) {
-  return cudaFuncSetAttribute(grouped_gemm_kernel<kSparse, kBN>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  return cudaFuncSetAttribute(grouped_gemm_kernel<kSparse, kBN, kGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              bytes);
 }
 
 cudaError_t gemm_set_smem_attrs() {
@@ -693,36 +768,51 @@ cudaError_t gemm_set_smem_attrs() {
   if (e != cudaSuccess) return e;
   maxb -= 1024;   // room for the kernels' static shared memory
   g_smem_limit = maxb;
-  cudaError_t errs[8] = {set_attr_one<true, 16>(maxb),  set_attr_one<true, 32>(maxb),  set_attr_one<true, 64>(maxb),
-                         set_attr_one<true, 128>(maxb), set_attr_one<false, 16>(maxb), set_attr_one<false, 32>(maxb),
-                         set_attr_one<false, 64>(maxb), set_attr_one<false, 128>(maxb)};
+  cudaError_t errs[11] = {set_attr_one<true, 16>(maxb),       set_attr_one<true, 32>(maxb),
+                          set_attr_one<true, 64>(maxb),       set_attr_one<true, 128>(maxb),
+                          set_attr_one<false, 16>(maxb),      set_attr_one<false, 32>(maxb),
+                          set_attr_one<false, 64>(maxb),      set_attr_one<false, 128>(maxb),
+                          set_attr_one<true, 16, true>(maxb), set_attr_one<true, 32, true>(maxb),
+                          set_attr_one<true, 64, true>(maxb)};
   for (cudaError_t x : errs)
     if (x != cudaSuccess) return x;
   return cudaSuccess;
 }
 
-template <bool kSparse>
+template <bool kSparse, bool kGLU = false>
 static cudaError_t launch_bn(int BN, int grid, size_t smem, cudaStream_t stream, const CUtensorMap& tb,
                              const CUtensorMap& tb64, const CUtensorMap& ts, const GemmParams& p) {
   switch (BN) {
-    case 16: return launch_pdl(grouped_gemm_kernel<kSparse, 16>, grid, kGemmThreads, smem, stream, tb, tb64, ts, p);
-    case 32: return launch_pdl(grouped_gemm_kernel<kSparse, 32>, grid, kGemmThreads, smem, stream, tb, tb64, ts, p);
-    case 64: return launch_pdl(grouped_gemm_kernel<kSparse, 64>, grid, kGemmThreads, smem, stream, tb, tb64, ts, p);
-    default: return launch_pdl(grouped_gemm_kernel<kSparse, 128>, grid, kGemmThreads, smem, stream, tb, tb64, ts, p);
+    case 16: return launch_pdl(grouped_gemm_kernel<kSparse, 16, kGLU>, grid, kGemmThreads, smem, stream, tb, tb64, ts, p);
+    case 32: return launch_pdl(grouped_gemm_kernel<kSparse, 32, kGLU>, grid, kGemmThreads, smem, stream, tb, tb64, ts, p);
+    default: return launch_pdl(grouped_gemm_kernel<kSparse, 64, kGLU>, grid, kGemmThreads, smem, stream, tb, tb64, ts, p);
   }
 }
 
-// returns 0 ok, 1 cuda error, 2 tensor map failure
+template <bool kSparse>
+static cudaError_t launch_bn(int BN, int grid, size_t smem, cudaStream_t stream, const CUtensorMap& tb,
+                             const CUtensorMap& tb64, const CUtensorMap& ts, const GemmParams& p, bool glu) {
+  if (glu) return launch_bn<true, true>(BN, grid, smem, stream, tb, tb64, ts, p);
+  if (BN == 128)
+    return launch_pdl(grouped_gemm_kernel<kSparse, 128, false>, grid, kGemmThreads, smem, stream, tb, tb64, ts, p);
+  return launch_bn<kSparse, false>(BN, grid, smem, stream, tb, tb64, ts, p);
+}
+
+// returns 0 ok, 1 cuda error, 2 tensor map failure.  h_scales / h_scale non-null: the SwiGLU
+// epilogue (sparse only; Y receives the h codes).
 int launch_gemm(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, const float* x_scale,
                 const uint8_t* w_packed, const float* w_scale, const int32_t* off, int E, int N, int K, int R,
-                int max_rows, void* Y, int y_f32, int* status, int num_sms, cudaStream_t stream) {
+                int max_rows, void* Y, int y_f32, int* status, int num_sms, cudaStream_t stream,
+                uint8_t* h_scales, const float* h_scale) {
   EncodeTiledFn enc = get_encode_fn();
   if (enc == nullptr) return 2;
-  const int BN = gemm_pick_bn(max_rows, R, E);
-  const long long bound = (((long long)R + BN - 1) / BN + E) * (N / kTileN);
+  const bool glu = h_scales != nullptr;
+  int BN = gemm_pick_bn(max_rows, R, E);
+  if (glu && BN > 64) BN = 64;   // two accumulators per tile: 64-token tiles at most
+  const long long bound = (((long long)R + BN - 1) / BN + E) * (N / kTileN / (glu ? 2 : 1));
   long long tcap = (bound + num_sms - 1) / num_sms;
   if (tcap > kMaxTableTiles) tcap = kMaxTableTiles;
-  const GemmPlan g = make_plan(sparse, BN, E, (int)tcap);
+  const GemmPlan g = make_plan(sparse, BN, E, (int)tcap, glu);
   if (g.stages < kNSets || g.smem > (size_t)g_smem_limit) return 1;   // ring too shallow: refuse, launch nothing
   const int box_h = g.BN < 32 ? g.BN : 32;
   const int kbps = g.cps * (sparse ? 2 : 4);
@@ -757,8 +847,9 @@ int launch_gemm(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, co
   p.w_scale = w_scale; p.off = off; p.Y = Y; p.status = status;
   p.E = E; p.N = N; p.K = K; p.R = R; p.y_f32 = y_f32; p.rcap = rcap;
   p.stages = g.stages; p.nacc = g.nacc; p.tcap = g.tcap;
-  const cudaError_t e = sparse ? launch_bn<true>(g.BN, num_sms, g.smem, stream, tb, tb64, ts, p)
-                               : launch_bn<false>(g.BN, num_sms, g.smem, stream, tb, tb64, ts, p);
+  p.h_scales = h_scales; p.h_scale = h_scale;
+  const cudaError_t e = sparse ? launch_bn<true>(g.BN, num_sms, g.smem, stream, tb, tb64, ts, p, glu)
+                               : launch_bn<false>(g.BN, num_sms, g.smem, stream, tb, tb64, ts, p, false);
   return e == cudaSuccess ? 0 : 1;
 }
 

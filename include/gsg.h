@@ -163,6 +163,32 @@ gsg_status_t gsg_grouped_dense_gemm(const uint8_t* a_codes, const uint8_t* a_sca
                                     const int32_t* expert_offsets, int E, int N, int K, int R,
                                     int max_rows_per_expert, void* Y, int y_dtype, void* stream);
 
+/* gsg_grouped_sparse_gemm_swiglu -- the up-projection with SwiGLU output preparation fused into
+ * the epilogue, producing the down-projection's NVFP4 input directly.
+ * Paper: §D.1 (p.19): the serving integration fuses SwiGLU output preparation for the second
+ * expert GEMM; §3.4 (pp.5-6) and App. A: the NVFP4 block rule.
+ * The weights are one fused [N2][K] matrix per expert, gate rows [0, I) then up rows [I, 2I)
+ * (I = N2/2), packed with gsg_pack_sparse_nvfp4 as usual (one s_w[e] for both halves).  With
+ * y[r][n] = s_x * s_w[e] * sum_k a[r][k] * w[e][n][k] (fp32, never rounded to bf16):
+ *     h[r][f] = silu(y[r][f]) * y[r][I + f],  silu(x) = x / (1 + exp(-x)),   f < I
+ * then h is quantized like the activations (32-element blocks along f, UE4M3 scale, E2M1 codes)
+ * with the caller's tensor scale *h_tensor_scale (a calibrated value; the dynamic amax of h
+ * would need a pass over all of h before any block could be encoded):
+ *     h_codes  [R][I/2]  (low nibble = even f)
+ *     h_scales the quad layout above for K = I (gsg_act_scales_bytes(R, I, 32) bytes)
+ * i.e. exactly what gsg_grouped_sparse_gemm takes as a_codes / a_scales for the down-projection
+ * over the same expert_offsets (with x_tensor_scale = h_tensor_scale).  N2 % 256 == 0; rows >=
+ * off[E] are not written (their scale entries are zero).  The fp32 h is not reproducible bit
+ * for bit by a CPU (exp); parity is checked against the exact h within the GEMM tolerance plus
+ * one quantization step.  No workspace.
+ */
+gsg_status_t gsg_grouped_sparse_gemm_swiglu(const uint8_t* a_codes, const uint8_t* a_scales,
+                                            const float* x_tensor_scale,
+                                            const uint8_t* w_packed, const float* w_tensor_scale,
+                                            const int32_t* expert_offsets, int E, int N2, int K, int R,
+                                            int max_rows_per_expert, const float* h_tensor_scale,
+                                            uint8_t* h_codes, uint8_t* h_scales, void* stream);
+
 /* ----------------------------------------------------------------------------------------
  * gsg_unpermute_scale -- gate-weighted scatter back to tokens.
  * Paper: §D.1 (p.19): scatter after the expert GEMM.

@@ -360,3 +360,57 @@ def test_gemm_full_size_sampled_30b_up(gsg):
             rows += sorted({lo, hi - 1, (lo + hi) // 2, min(lo + 128, hi - 1), min(lo + 129, hi - 1)})
     y_ref, bound = tl.reference_rows(np.array(rows), off, q, sc, 32, canon, s_x, sws)
     tl.assert_gemm_close(Y[torch.tensor(rows, device=DEV)], y_ref, bound, "30b_up_prefill sampled")
+
+
+# ---------------------------------------------------------------- up-projection with the SwiGLU epilogue
+def _unquad(quad: np.ndarray, R: int, K: int) -> np.ndarray:
+    """Quad activation-scale bytes -> scales [R, K/32] (entry (kb, r, 0, j) is row r, block 4 kb + j)."""
+    q = np.asarray(quad, dtype=np.uint8).reshape(K // 128, R + olayout.ACT_SCALE_PAD_ROWS, 4, 4)
+    return q[:, :R, 0, :].transpose(1, 0, 2).reshape(R, K // 32)
+
+
+SWIGLU_CASES = [
+    ([16], 128, 256),                        # one tile, I = 128
+    ([40, 0, 77], 256, 512),                 # ragged with an empty expert
+    ([0, 1, 7, 9, 33, 64], 128, 768),        # the small-tile ladder
+    ([300, 5], 384, 256),                    # tiles above 64 rows (64-token tiles), I = 384
+]
+
+
+@pytest.mark.parametrize("counts,I,K", SWIGLU_CASES)
+def test_swiglu_gemm_matches_oracle(gsg, counts, I, K):
+    from oracle import codecs as ocodecs
+    from oracle import quant as oquant
+    from oracle import swiglu as oswiglu
+    c = _gemm_case(counts, 2 * I, K, sparse=True)
+    R = c["R"]
+    y_ref, b = tl.reference_rows(np.arange(R), c["off"], c["q"], c["sc"], 32, c["canon"], c["s_x"], c["sws"])
+    h_ref = oswiglu.swiglu_rows(y_ref)
+    s_h = np.float32(np.abs(h_ref).max() / 2688.0)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+    act = gsg.QuantizedActivations(codes=t(c["a_codes"]), scales=t(c["a_quad"]),
+                                   x_scale=torch.tensor([c["s_x"]], dtype=torch.float32, device=DEV), R=R, K=K,
+                                   sf_block=32)
+    w = gsg.PackedSparseWeights(packed=t(c["w"]["packed"]), w_scale=t(c["w"]["w_scale"]), E=c["E"], N=2 * I, K=K)
+    hq = gsg.grouped_sparse_gemm_swiglu(act, w, t(c["off"]), torch.tensor([s_h], device=DEV),
+                                        max_rows_per_expert=max(counts))
+    _status_ok(gsg)
+    codes = olayout.unpack_act_codes(hq.codes.cpu().numpy()[:R])
+    quad = hq.scales.cpu().numpy()
+    scales = _unquad(quad, R, I)
+    hd = oquant.decode_rows(codes, scales, 32) * float(s_h)
+    # one quantization step of the block (|v - dec(q(v))| <= d for the E2M1 grid, saturation
+    # included) + the exact propagation of the GEMM tolerance through silu(g) * u + fp32 rounding
+    d_blk = np.repeat(ocodecs.ue4m3_decode(scales).astype(np.float64) * float(s_h), 32, axis=1)
+    tau = 2.0 ** -10 * b + 1e-6
+    bound = d_blk + oswiglu.swiglu_error_bound(y_ref, tau) + 2.0 ** -18 * np.abs(h_ref)
+    err = np.abs(hd - h_ref)
+    assert np.all(err <= bound), (np.max(err - bound), np.argmax(err - bound))
+    # almost every code equals the oracle's quantization of the exact h
+    qr, scr = oquant.quantize_rows(h_ref.astype(np.float32), 32, s_h)
+    assert np.mean(codes == qr) > 0.95 and np.mean(scales == scr) > 0.95
+    # scale entries that refer to rows >= R are zero
+    q5 = quad.reshape(I // 128, R + olayout.ACT_SCALE_PAD_ROWS, 4, 4)
+    for cc in range(4):
+        rr = np.arange(R + olayout.ACT_SCALE_PAD_ROWS)
+        assert not q5[:, rr + 32 * cc >= R, cc, :].any()

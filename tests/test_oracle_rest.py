@@ -190,3 +190,27 @@ def test_golden_act_block():
     q, sc = quant.quantize_rows(x, 32, np.float32(g["s_x"]))
     assert sc[0].tolist() == g["scales"]
     assert q[0].tolist() == g["codes"]
+
+
+def test_swiglu_oracle_pins():
+    """silu against its closed forms and an independent float64 implementation (torch), the slope
+    bound against a dense grid, and the h error bound against brute-force perturbations."""
+    import torch
+    from oracle import swiglu as osw
+    assert osw.silu(np.array([0.0]))[0] == 0.0
+    x = np.linspace(-30, 30, 20001)
+    s = osw.silu(x)
+    np.testing.assert_allclose(osw.silu(-x), s - x, rtol=0, atol=1e-12)          # silu(-x) = silu(x) - x
+    np.testing.assert_allclose(s, torch.nn.functional.silu(torch.from_numpy(x)).numpy(), rtol=1e-15, atol=1e-300)
+    assert np.abs(osw.silu(np.array([40.0, -40.0])) - np.array([40.0, 0.0])).max() < 1e-15
+    slope = np.abs(np.diff(s) / np.diff(x)).max()
+    assert 1.09 < slope <= osw.SILU_SLOPE_MAX
+    rng = np.random.default_rng(11)
+    y = rng.normal(size=(6, 8)) * 3
+    h = osw.swiglu_rows(y)
+    np.testing.assert_allclose(h, osw.silu(y[:, :4]) * y[:, 4:], rtol=0, atol=0)
+    tau = np.abs(rng.normal(size=y.shape)) * 0.05
+    bound = osw.swiglu_error_bound(y, tau)
+    for _ in range(200):                                   # no perturbation within tau escapes the bound
+        yp = y + tau * rng.uniform(-1, 1, size=y.shape)
+        assert np.all(np.abs(osw.swiglu_rows(yp) - h) <= bound + 1e-12)
