@@ -547,6 +547,110 @@ def gsg_token_tile(max_rows: int, R: int, E: int) -> int:
     return 128 if R >= 64 * E else 64
 
 
+# ------------------------------------------------------------------ a whole MoE layer
+class LayerWorkload:
+    """route -> quantize -> up-projection with the SwiGLU epilogue -> down-projection -> unpermute,
+    all buffers resident.  The tensor scale of h (the down-projection's input) is calibrated once
+    beforehand, like the packing: the amax of h from an unfused fp32 pass over the same batch."""
+
+    def __init__(self, L: inputs.MoELayer, dev: torch.device):
+        self.L, self.dev = L, dev
+        up, dn = L.up(), L.down()
+        E, H, I, T, k, R = L.E, L.H, L.I, L.T, L.top_k, L.R
+        u8 = dict(dtype=torch.uint8, device=dev)
+        lib = gsg.lib()
+        self.wu = gsg.PackedSparseWeights(packed=torch.empty(lib.gsg_sparse_packed_bytes(E, 2 * I, H), **u8),
+                                          w_scale=torch.empty(E, dtype=torch.float32, device=dev), E=E, N=2 * I, K=H)
+        self.wd = gsg.PackedSparseWeights(packed=torch.empty(lib.gsg_sparse_packed_bytes(E, H, I), **u8),
+                                          w_scale=torch.empty(E, dtype=torch.float32, device=dev), E=E, N=H, K=I)
+        ws = torch.empty(max(gsg.workspace_size(gsg.OP_PACK_SPARSE, 1, 2 * I, H),
+                             gsg.workspace_size(gsg.OP_PACK_SPARSE, 1, H, I), 16), **u8)
+        for e in range(E):
+            gsg.pack_sparse_nvfp4(inputs.expert_weight(up, e, str(dev))[None], out=self.wu.expert(e), workspace=ws)
+            gsg.pack_sparse_nvfp4(inputs.down_weight(L, e, str(dev))[None], out=self.wd.expert(e), workspace=ws)
+        self.X = inputs.activations(up).to(dev)
+        ids_h = inputs.routing(up)
+        self.ids = ids_h.to(dev)
+        self.gates = inputs.gates(up).to(dev)
+        counts = torch.bincount(ids_h.reshape(-1).long(), minlength=E)
+        self.max_rows = int(counts.max())
+        self.touched = int((counts > 0).sum())
+        self.route = gsg.Routing(offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+                                 perm_src=torch.empty(R, dtype=torch.int32, device=dev),
+                                 inv_perm=torch.empty(R, dtype=torch.int32, device=dev), T=T, k=k, E=E)
+        self.ws_route = torch.empty(max(gsg.workspace_size(gsg.OP_ROUTE, E, 0, 0, T, k), 16), **u8)
+        self.ws_quant = torch.empty(max(gsg.workspace_size(gsg.OP_QUANTIZE, 0, 0, H, T, k), 16), **u8)
+        self.qa = gsg.QuantizedActivations(codes=torch.empty(R, H // 2, **u8),
+                                           scales=torch.empty(gsg.act_scales_bytes(R, H, 32), **u8),
+                                           x_scale=torch.empty(1, dtype=torch.float32, device=dev), R=R, K=H,
+                                           sf_block=32)
+        self.h_scale = torch.ones(1, dtype=torch.float32, device=dev)
+        self.hq = gsg.QuantizedActivations(codes=torch.empty(R, I // 2, **u8),
+                                           scales=torch.empty(gsg.act_scales_bytes(R, I, 32), **u8),
+                                           x_scale=self.h_scale, R=R, K=I, sf_block=32)
+        self.Y2 = torch.empty(R, H, dtype=torch.bfloat16, device=dev)
+        self.out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+        # calibration of h's tensor scale (offline, like the packing)
+        gsg.moe_route_permute(self.ids, E, out=self.route, workspace=self.ws_route)
+        gsg.quantize_act_nvfp4(self.X, 32, self.route.inv_perm, k, out=self.qa, workspace=self.ws_quant)
+        y = gsg.grouped_sparse_gemm(self.qa, self.wu, self.route.offsets, self.max_rows, out_dtype=torch.float32)
+        h = torch.nn.functional.silu(y[:R, :I]) * y[:R, I:]
+        amax = float(h.abs().max())
+        self.h_scale.fill_(amax / 2688.0 if amax > 0 else 1.0)
+        del y, h
+        torch.cuda.synchronize()
+
+    def step(self):
+        L = self.L
+        gsg.moe_route_permute(self.ids, L.E, out=self.route, workspace=self.ws_route)
+        gsg.quantize_act_nvfp4(self.X, 32, self.route.inv_perm, L.top_k, out=self.qa, workspace=self.ws_quant)
+        gsg.grouped_sparse_gemm_swiglu(self.qa, self.wu, self.route.offsets, self.h_scale, self.max_rows,
+                                       out=self.hq)
+        gsg.grouped_sparse_gemm(self.hq, self.wd, self.route.offsets, self.max_rows, out=self.Y2)
+        gsg.unpermute_scale(self.Y2, self.route.inv_perm, self.gates, L.top_k, out=self.out)
+
+    def flops(self) -> float:
+        L = self.L
+        return 2.0 * L.R * (2 * L.I * L.H + L.H * L.I)
+
+    def weight_bytes(self) -> int:
+        L = self.L
+        return self.touched * (2 * L.I * L.H + L.H * L.I) * 11 // 32
+
+
+def run_layer(args, local):
+    """One MoE layer per step (see LayerWorkload), timed in-graph after an L2 flush: latency per
+    token batch, tokens/s, dense-equivalent TFLOP/s of the two GEMMs, weight GB/s."""
+    dev = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(dev)
+    gsg.load_library()
+    L = inputs.LAYERS[args.layer]
+    wl = LayerWorkload(L, dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    wl.step()
+    torch.cuda.synchronize()
+    st = gsg.get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after the first layer step")
+    gt = capture_timed(wl.step)
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        gt[0].replay()
+    ms, _ = timed_graph_ms(gt, args.steps, flush, 1)
+    st = gsg.get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after timing")
+    print(json.dumps({
+        "layer": L.name, "E": L.E, "hidden": L.H, "expert_ffn": L.I, "tokens": L.T, "top_k": L.top_k,
+        "routed_rows": L.R, "routing": L.routing, "steps": args.steps, "warmup": args.warmup,
+        "us_per_layer": ms * 1e3, "tokens_per_s": L.T / (ms * 1e-3),
+        "tflops_dense_equivalent": wl.flops() / (ms * 1e-3) / 1e12,
+        "weight_gbs": wl.weight_bytes() / (ms * 1e-3) / 1e9, "h_tensor_scale": float(wl.h_scale.item()),
+        "kernels": "route, amax + quantize, up-projection + SwiGLU + NVFP4 of h, down-projection, unpermute",
+        "timing": "in-graph CUDA events around the layer, L2 flushed (256 MB write) before every replay"}),
+          flush=True)
+
+
 # ------------------------------------------------------------------ G x N sweep
 SWEEP_SHAPES = {            # expert projection shapes: (K, N)
     "30b_up": (2048, 1536), "30b_down": (768, 2048), "1t_up": (7168, 4096), "1t_down": (2048, 7168)}
@@ -675,6 +779,8 @@ def main():
     ap.add_argument("--quick", action="store_true", help="skip e2e, dense control and CPU baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-experts", type=int, default=24)
+    ap.add_argument("--layer", default=None, choices=sorted(inputs.LAYERS),
+                    help="time a whole MoE layer (up + SwiGLU + down) instead of the headline step")
     ap.add_argument("--sweep", action="store_true",
                     help="G x N sweep of the sparse GEMM against the dense control (one JSON line per point)")
     ap.add_argument("--sweep-shapes", default="30b_up,30b_down,1t_up,1t_down")
@@ -693,6 +799,8 @@ def main():
             run_profile_steps(args, local)
         elif args.sweep:
             run_sweep(args, local)
+        elif args.layer:
+            run_layer(args, local)
         else:
             run_ours(args, world, rank, local)
     finally:

@@ -39,6 +39,7 @@ constexpr uint64_t kWaitTimeoutNs = 2000000000ull;   // 2 s
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColAcc = kNSets * kSetCols;       // first accumulator (192)
 constexpr int kOutStageBytes = 16 * 32 * 4;           // epilogue transpose buffer per warp
+constexpr int kGluStageBytes = 32 * 36 * 4;           // SwiGLU epilogue: 32 tokens x 32 features (+4 pad)
 
 struct GemmParams {
   const uint8_t* a_scales;
@@ -300,8 +301,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
   int* pref = offs + (E + 1);                    // [E+1]
   float* wsc = reinterpret_cast<float*>(pref + (E + 1));   // [E]
   int4* ttab = reinterpret_cast<int4*>((reinterpret_cast<uintptr_t>(wsc + E) + 15) & ~uintptr_t(15));   // [tcap]
-  // per-epilogue-warp staging buffer for 16 tokens x 32 output features (fp32 worst case)
-  uint8_t* ostage = reinterpret_cast<uint8_t*>(ttab + p.tcap);   // [4][kOutStageBytes]
+  // per-epilogue-warp staging buffer: 16 tokens x 32 output features (fp32 worst case), or the
+  // SwiGLU epilogue's 32 x 36 fp32
+  uint8_t* ostage = reinterpret_cast<uint8_t*>(ttab + p.tcap);   // [4][kOutStageBytes or kGluStageBytes]
   volatile int* abort_flag = &ctl->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -584,44 +586,61 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
       const float scale = __fmul_rn(sx, wsc[c.e]);
       const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + kColAcc + (uint32_t)(acc * G::kNT * G::kAccStride);
       if constexpr (kGLU) {
-        // SwiGLU output preparation: lane = feature f of this warp's 32-feature block (the block
-        // the next GEMM's scales cover), h = silu(gate) * up in fp32, one NVFP4 block per token
-        // (block max over the warp), codes packed 8 lanes to a 32-bit word, scales into the quad
-        // layout (k-block nt, position q).
+        // SwiGLU output preparation, 32 tokens at a time: lane = feature f of this warp's
+        // 32-feature block (one NVFP4 block of the down-projection's K), h = silu(gate) * up in
+        // fp32; the block is transposed through shared memory so that each lane then owns one
+        // token's 32 values: block max, UE4M3 scale and E2M1 codes once per token, 16-byte code
+        // stores, scale bytes into the quad layout (k-block nt, position q).
         const float sh = __ldg(p.h_scale);
         const float six_sh = __fmul_rn(6.0f, sh);
         const int f0 = c.nt * kTileN + 32 * q;
         const int hrow = p.N / 4;                 // bytes of h codes per row (N/2 features)
         uint8_t* hc = static_cast<uint8_t*>(p.Y);
-        for (int c0 = 0; c0 < valid; c0 += 16) {
-          float g[16], u[16];
+        const uint32_t tb = smem_u32(ostage + (size_t)(warp - 3) * kGluStageBytes);   // [32][36] fp32
+        for (int c0 = 0; c0 < valid; c0 += 32) {
+          float g[32], u[32];
           tc_ld_16(taddr + c0, g);
+          tc_ld_16(taddr + c0 + 16, g + 16);
           tc_ld_16(taddr + G::kAccStride + c0, u);
-          uint32_t scs[16];
+          tc_ld_16(taddr + G::kAccStride + c0 + 16, u + 16);
 #pragma unroll
-          for (int t = 0; t < 16; ++t) {
+          for (int t = 0; t < 32; ++t) {
             const float gs = __fmul_rn(g[t], scale), us = __fmul_rn(u[t], scale);
-            const float hv = __fmul_rn(__fdiv_rn(gs, __fadd_rn(1.0f, expf(-gs))), us);
-            const float am = warp_max(fabsf(hv));
-            const BlockScale bs = block_scale_cvt(am, six_sh, sh);
-            scs[t] = bs.sc;
-            uint32_t w = e2m1_encode(__fmul_rn(hv, bs.inv)) << (4 * (lane & 7));
-            w |= __shfl_xor_sync(0xffffffffu, w, 1);
-            w |= __shfl_xor_sync(0xffffffffu, w, 2);
-            w |= __shfl_xor_sync(0xffffffffu, w, 4);
-            if ((lane & 7) == 0 && c0 + t < valid)
-              *reinterpret_cast<uint32_t*>(hc + (size_t)(r0 + c0 + t) * hrow + f0 / 2 + (lane >> 3) * 4) = w;
+            const float hv = __fmul_rn(__fdividef(gs, __fadd_rn(1.0f, __expf(-gs))), us);
+            asm volatile("st.shared.f32 [%0], %1;" ::"r"(tb + (uint32_t)(t * 36 + lane) * 4u), "f"(hv) : "memory");
           }
-          // quad scale entries (nt, row - 32c, c, q) of the 16 tokens: 64 single bytes, two per lane
+          __syncwarp();
+          float v[32];
 #pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            const int idx = lane + 32 * k, t = idx >> 2, cc = idx & 3;
-            uint32_t sc = 0;
+          for (int k4 = 0; k4 < 8; ++k4) {
+            uint32_t a, b, cc, d;
+            lds128(tb + (uint32_t)(lane * 36 + 4 * k4) * 4u, a, b, cc, d);
+            v[4 * k4] = __uint_as_float(a);
+            v[4 * k4 + 1] = __uint_as_float(b);
+            v[4 * k4 + 2] = __uint_as_float(cc);
+            v[4 * k4 + 3] = __uint_as_float(d);
+          }
+          __syncwarp();
+          float am = 0.0f;
 #pragma unroll
-            for (int tt = 0; tt < 16; ++tt) sc = tt == t ? scs[tt] : sc;
-            const int row = r0 + c0 + t, rr = row - 32 * cc;
-            if (c0 + t < valid && rr >= 0)
-              p.h_scales[((size_t)c.nt * p.rcap + rr) * 16 + cc * 4 + q] = (uint8_t)sc;
+          for (int k = 0; k < 32; ++k) am = fmaxf(am, fabsf(v[k]));
+          const BlockScale bs = block_scale_cvt(am, six_sh, sh);
+          uint32_t wd[4];
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            float xs[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) xs[i] = __fmul_rn(v[8 * w + i], bs.inv);
+            wd[w] = e2m1_encode8_cvt(xs);
+          }
+          const int row = r0 + c0 + lane;
+          if (c0 + lane < valid) {
+            *reinterpret_cast<uint4*>(hc + (size_t)row * hrow + f0 / 2) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+              const int rr = row - 32 * cc;
+              if (rr >= 0) p.h_scales[((size_t)c.nt * p.rcap + rr) * 16 + cc * 4 + q] = (uint8_t)bs.sc;
+            }
           }
         }
       } else {
@@ -709,8 +728,9 @@ static GemmPlan make_plan(bool sparse, int BN, int E, int tcap, bool glu = false
   const int body = g.cps * BN * 128 + nt * g.cps * (sparse ? kSparseChunkBytes : kDenseChunkBytes) + kbps * 512;
   g.stage = (body + 1023) / 1024 * 1024;
   // everything but the stage ring and the tile table, at its largest
+  const int ostage = 4 * (glu ? kGluStageBytes : kOutStageBytes);
   const int fixed = 1024 + (2 * kMaxStages + kNSets + 2 * kMaxAcc + 1) * 8 + (int)sizeof(Ctl) + (3 * E + 2) * 4 +
-                    16 + 4 * kOutStageBytes;
+                    16 + ostage;
   int budget = g_smem_limit - fixed;
   if (BN == 128 && budget > kStageBudget128) budget = kStageBudget128;
   g.stages = (budget - tcap * 16) / g.stage;
@@ -720,7 +740,7 @@ static GemmPlan make_plan(bool sparse, int BN, int E, int tcap, bool glu = false
   if (g.nacc > kMaxAcc) g.nacc = kMaxAcc;
   const int nbars = 2 * g.stages + kNSets + 2 * g.nacc + 1;
   g.smem = 1024 + (size_t)g.stages * g.stage + nbars * 8 + sizeof(Ctl) + (size_t)(3 * E + 2) * 4 + 16 +
-           (size_t)tcap * 16 + 4 * kOutStageBytes;
+           (size_t)tcap * 16 + ostage;
   return g;
 }
 

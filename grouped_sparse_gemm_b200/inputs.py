@@ -12,8 +12,8 @@ model (hidden 2048, expert FFN 768, 128 experts, top-8) and a 1T-shaped model
 datasets are used: weights are N(0, sigma) in fp32, activations N(0, 1) in
 bf16 with a few scaled outlier channels, routing is uniform or Zipf.
 
-Seed streams (base seed 0): expert e's weight -> 1000 + e, activations -> 1,
-routing -> 2, gate logits -> 3, outlier channels -> 4.
+Seed streams (base seed 0): expert e's weight -> 1000 + e (a layer's down-projection:
+3000 + e), activations -> 1, routing -> 2, gate logits -> 3, outlier channels -> 4.
 """
 from __future__ import annotations
 
@@ -65,6 +65,55 @@ for _b in (1, 32, 128, 256):
     CONFIGS[f"1t_down_decode_b{_b}"] = MoEConfig(
         f"1t_down_decode_b{_b}", E=384, K=2048, N=7168, T=_b, top_k=8,
         routing="uniform", w_sigma=0.015)
+
+
+@dataclasses.dataclass(frozen=True)
+class MoELayer:
+    """A routed MoE FFN layer: up-projection with fused gate|up weights [2I, H], SwiGLU, then the
+    down-projection [H, I], over the same routed tokens.  Shapes of the expert FFNs of the
+    30B-A3B-shaped and 1T-shaped models (see the module docstring)."""
+    name: str
+    E: int
+    H: int                 # hidden size: K of the up-projection, N of the down-projection
+    I: int                 # expert FFN size: N/2 of the up-projection, K of the down-projection
+    T: int
+    top_k: int
+    routing: str
+    zipf_s: float = 0.0
+    w_sigma: float = 0.02
+    outlier_frac: float = 0.0
+    outlier_scale: float = 1.0
+
+    @property
+    def R(self) -> int:
+        return self.T * self.top_k
+
+    def up(self) -> MoEConfig:
+        """The up-projection (its activations, routing and gates are the layer's)."""
+        return MoEConfig(self.name + "_up", E=self.E, K=self.H, N=2 * self.I, T=self.T, top_k=self.top_k,
+                         routing=self.routing, zipf_s=self.zipf_s, w_sigma=self.w_sigma,
+                         outlier_frac=self.outlier_frac, outlier_scale=self.outlier_scale)
+
+    def down(self) -> MoEConfig:
+        return MoEConfig(self.name + "_down", E=self.E, K=self.I, N=self.H, T=self.T, top_k=self.top_k,
+                         routing=self.routing, zipf_s=self.zipf_s, w_sigma=self.w_sigma)
+
+
+LAYERS = {
+    "tiny_layer": MoELayer("tiny_layer", E=4, H=256, I=256, T=32, top_k=2, routing="uniform"),
+    "30b_layer": MoELayer("30b_layer", E=128, H=2048, I=768, T=512, top_k=8, routing="zipf", zipf_s=1.0,
+                          w_sigma=0.02, outlier_frac=0.01, outlier_scale=20.0),
+    "1t_layer": MoELayer("1t_layer", E=384, H=7168, I=2048, T=1024, top_k=8, routing="zipf", zipf_s=1.1,
+                         w_sigma=0.015, outlier_frac=0.005, outlier_scale=30.0),
+}
+SEED_W_DOWN_BASE = 3000
+
+
+def down_weight(layer: MoELayer, e: int, device: str = "cpu") -> torch.Tensor:
+    """Expert e's down-projection weight fp32 [H, I] ~ N(0, w_sigma) (its own seed stream)."""
+    g = _gen(SEED_W_DOWN_BASE + e, device)
+    w = torch.randn(layer.H, layer.I, generator=g, device=device, dtype=torch.float32)
+    return w.mul_(layer.w_sigma)
 
 
 def _gen(seed: int, device: str) -> torch.Generator:

@@ -178,9 +178,10 @@ gsg_status_t gsg_grouped_dense_gemm(const uint8_t* a_codes, const uint8_t* a_sca
  *     h_scales the quad layout above for K = I (gsg_act_scales_bytes(R, I, 32) bytes)
  * i.e. exactly what gsg_grouped_sparse_gemm takes as a_codes / a_scales for the down-projection
  * over the same expert_offsets (with x_tensor_scale = h_tensor_scale).  N2 % 256 == 0; rows >=
- * off[E] are not written (their scale entries are zero).  The fp32 h is not reproducible bit
- * for bit by a CPU (exp); parity is checked against the exact h within the GEMM tolerance plus
- * one quantization step.  No workspace.
+ * off[E] are not written (their scale entries are zero).  silu is evaluated in fp32 with the
+ * fast exponential and division (a few ulp), so h is not reproducible bit for bit by a CPU;
+ * parity is checked against the exact h within the GEMM tolerance plus one quantization step.
+ * Token tiles are at most 64 rows (two accumulators per tile).  No workspace.
  */
 gsg_status_t gsg_grouped_sparse_gemm_swiglu(const uint8_t* a_codes, const uint8_t* a_scales,
                                             const float* x_tensor_scale,
