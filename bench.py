@@ -547,6 +547,53 @@ def gsg_token_tile(max_rows: int, R: int, E: int) -> int:
     return 128 if R >= 64 * E else 64
 
 
+# ------------------------------------------------------------------ every configuration
+def run_all_configs(args, local):
+    """Per configuration (the tiny case, the 30B and 1T prefill and decode shapes, the 1T decode
+    batch sweep): the GEMM alone and the whole step, in-graph after an L2 flush, the dense-NVFP4
+    control on the same routed rows, algorithmic GB/s and the fraction of the measured HBM copy
+    bandwidth.  One JSON line per configuration."""
+    dev = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(dev)
+    gsg.load_library()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    peaks, kind = measured_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    names = args.configs.split(",") if args.configs else list(inputs.CONFIGS)
+    reps = max(10, min(args.steps, 500))
+    for name in names:
+        cfg = inputs.CONFIGS[name]
+        wl = Workload(cfg, dev, with_dense=True)
+        wl.step()
+        wl.prepare_dense()
+        torch.cuda.synchronize()
+        res = {"config": name, "E": cfg.E, "K": cfg.K, "N": cfg.N, "tokens": cfg.T, "top_k": cfg.top_k,
+               "routed_rows": cfg.R, "touched_experts": wl.touched, "max_rows_per_expert": wl.max_rows}
+        for tag, fn in (("gemm", wl.gemm), ("step", wl.step), ("dense_gemm", wl.dense_gemm)):
+            gt = capture_timed(fn)
+            for _ in range(3):
+                flush.fill_(1)
+                gt[0].replay()
+            ms, _ = timed_graph_ms(gt, reps, flush, 1)
+            res[tag + "_us"] = ms * 1e3
+            del gt
+        st = gsg.get_device_status()
+        if st != 0:
+            raise RuntimeError(f"device status {st} on {name}")
+        w, a, y = wl.gemm_bytes()
+        flops = 2.0 * cfg.R * cfg.N * cfg.K
+        g_s = res["gemm_us"] * 1e-6
+        res.update({"gemm_tflops": flops / g_s / 1e12, "gemm_weight_gbs": w / g_s / 1e9,
+                    "gemm_total_gbs": (w + a + y) / g_s / 1e9, "gemm_hbm_frac": (w + a + y) / g_s / 1e9 / hbm,
+                    "dense_gemm_gbs": wl.dense_gemm_bytes() / (res["dense_gemm_us"] * 1e-6) / 1e9,
+                    "sparse_speedup": res["dense_gemm_us"] / res["gemm_us"],
+                    "hbm_peak_gbs": hbm, "peak_source": kind, "reps": reps,
+                    "timing": "in-graph CUDA events, L2 flushed (256 MB write) before every replay"})
+        print(json.dumps(res), flush=True)
+        del wl
+        torch.cuda.empty_cache()
+
+
 # ------------------------------------------------------------------ a whole MoE layer
 class LayerWorkload:
     """route -> quantize -> up-projection with the SwiGLU epilogue -> down-projection -> unpermute,
@@ -779,6 +826,9 @@ def main():
     ap.add_argument("--quick", action="store_true", help="skip e2e, dense control and CPU baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-experts", type=int, default=24)
+    ap.add_argument("--all-configs", action="store_true",
+                    help="GEMM, step and dense control for every configuration (one JSON line each)")
+    ap.add_argument("--configs", default=None, help="comma-separated subset for --all-configs")
     ap.add_argument("--layer", default=None, choices=sorted(inputs.LAYERS),
                     help="time a whole MoE layer (up + SwiGLU + down) instead of the headline step")
     ap.add_argument("--sweep", action="store_true",
@@ -801,6 +851,8 @@ def main():
             run_sweep(args, local)
         elif args.layer:
             run_layer(args, local)
+        elif args.all_configs:
+            run_all_configs(args, local)
         else:
             run_ours(args, world, rank, local)
     finally:

@@ -25,13 +25,14 @@ __all__ = [
     "PackedSparseWeights", "PackedDenseWeights", "Routing", "QuantizedActivations",
     "pack_sparse_nvfp4", "pack_dense_nvfp4", "moe_route_permute", "moe_route_permute_noalloc",
     "quantize_act_nvfp4",
-    "grouped_sparse_gemm", "grouped_sparse_gemm_swiglu", "grouped_dense_gemm", "unpermute_scale",
+    "grouped_sparse_gemm", "grouped_sparse_gemm_swiglu", "grouped_sparse_gemm_combine", "combine_workspace",
+    "grouped_dense_gemm", "unpermute_scale", "OP_COMBINE",
     "get_device_status",
     "act_scales_bytes", "workspace_size", "OP_PACK_SPARSE", "OP_PACK_DENSE", "OP_ROUTE",
     "OP_QUANTIZE", "OP_GEMM", "EXPORTED_SYMBOLS",
 ]
 
-OP_PACK_SPARSE, OP_PACK_DENSE, OP_ROUTE, OP_QUANTIZE, OP_GEMM = 1, 2, 3, 4, 5
+OP_PACK_SPARSE, OP_PACK_DENSE, OP_ROUTE, OP_QUANTIZE, OP_GEMM, OP_COMBINE = 1, 2, 3, 4, 5, 6
 OUT_BF16, OUT_F32 = 0, 1
 ACT_SCALE_PAD_ROWS = 256
 
@@ -41,7 +42,7 @@ EXPORTED_SYMBOLS = [
     "gsg_pack_sparse_nvfp4", "gsg_pack_dense_nvfp4", "gsg_moe_route_permute",
     "gsg_quantize_act_nvfp4", "gsg_grouped_sparse_gemm", "gsg_grouped_dense_gemm",
     "gsg_unpermute_scale", "gsg_get_device_status", "gsg_status_string", "gsg_version",
-    "gsg_moe_route_permute_noalloc", "gsg_grouped_sparse_gemm_swiglu",
+    "gsg_moe_route_permute_noalloc", "gsg_grouped_sparse_gemm_swiglu", "gsg_grouped_sparse_gemm_combine",
 ]
 
 _STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported shape", -3: "CUDA error",
@@ -91,6 +92,7 @@ def load_library(build_if_missing: bool = False) -> ctypes.CDLL:
         "gsg_version": (i, []),
         "gsg_moe_route_permute_noalloc": (i, [vp, i, i, i, vp, vp, vp, vp]),
         "gsg_grouped_sparse_gemm_swiglu": (i, [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, vp, vp, vp]),
+        "gsg_grouped_sparse_gemm_combine": (i, [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, vp, vp, sz, vp, vp]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -325,6 +327,29 @@ def grouped_sparse_gemm_swiglu(act: QuantizedActivations, w: PackedSparseWeights
         _ptr(act.codes), _ptr(act.scales), _ptr(act.x_scale), _ptr(w.packed), _ptr(w.w_scale),
         _ptr(offsets), w.E, w.N, w.K, act.R, max_rows_per_expert, _ptr(h_scale), _ptr(out.codes),
         _ptr(out.scales), _stream(stream)))
+    return out
+
+
+def combine_workspace(E: int, N: int, K: int, T: int, k: int, device) -> torch.Tensor:
+    """A zeroed workspace for grouped_sparse_gemm_combine (reusable call after call)."""
+    return torch.zeros(max(workspace_size(OP_COMBINE, E, N, K, T, k), 16), dtype=torch.uint8, device=device)
+
+
+def grouped_sparse_gemm_combine(act: QuantizedActivations, w: PackedSparseWeights, routing: "Routing",
+                                gates: torch.Tensor, workspace: torch.Tensor, max_rows_per_expert: int = -1,
+                                out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Down-projection with the gate-weighted combine fused into the epilogue
+    (gsg_grouped_sparse_gemm_combine): out [T, N] bf16, bit for bit grouped_sparse_gemm followed by
+    unpermute_scale.  workspace from combine_workspace (zero before the first call, left zero)."""
+    assert act.sf_block == 32 and act.K == w.K and act.R == routing.T * routing.k
+    _need_cuda(act.codes, act.scales, routing.offsets, routing.perm_src, gates, workspace)
+    T, k = routing.T, routing.k
+    if out is None:
+        out = torch.empty(max(T, 1), w.N, dtype=torch.bfloat16, device=act.codes.device)
+    _check("gsg_grouped_sparse_gemm_combine", lib().gsg_grouped_sparse_gemm_combine(
+        _ptr(act.codes), _ptr(act.scales), _ptr(act.x_scale), _ptr(w.packed), _ptr(w.w_scale),
+        _ptr(routing.offsets), w.E, w.N, w.K, T, k, max_rows_per_expert, _ptr(routing.perm_src), _ptr(gates),
+        _ptr(workspace), workspace.numel(), _ptr(out), _stream(stream)))
     return out
 
 

@@ -49,6 +49,8 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 inline gsg_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? GSG_OK : GSG_ERR_CUDA; }
 
+size_t combine_slot_bytes(int T, int k, int N) { return ((size_t)T * k * N * 2 + 255) / 256 * 256; }
+
 bool weight_shape_ok(int E, int N, int K) {
   return E >= 1 && N >= 128 && K >= 256 && N % 128 == 0 && K % 256 == 0;
 }
@@ -93,6 +95,9 @@ size_t gsg_workspace_size(int op, int E, int N, int K, int T, int k) {
     case GSG_OP_QUANTIZE:
       if (T < 0 || K < 1) return 0;
       return (size_t)gsg::quant_partials((long long)T * K) * sizeof(float);
+    case GSG_OP_COMBINE:   // slots bf16 [T*k][N], then counters int32 [T][N/32]
+      if (T < 0 || k < 1 || N < 32) return 0;
+      return combine_slot_bytes(T, k, N) + (size_t)T * (N / 32) * sizeof(int);
     default:
       return 0;
   }
@@ -222,6 +227,40 @@ gsg_status_t gsg_grouped_sparse_gemm_swiglu(const uint8_t* a_codes, const uint8_
   const int rc = gsg::launch_gemm(true, a_codes, a_scales, x_tensor_scale, w_packed, w_tensor_scale, expert_offsets,
                                   E, N2, K, R, max_rows_per_expert, h_codes, 0, d->status, d->num_sms,
                                   as_stream(stream), h_scales, h_tensor_scale);
+  return rc == 0 ? GSG_OK : GSG_ERR_CUDA;
+}
+
+gsg_status_t gsg_grouped_sparse_gemm_combine(const uint8_t* a_codes, const uint8_t* a_scales,
+                                             const float* x_tensor_scale, const uint8_t* w_packed,
+                                             const float* w_tensor_scale, const int32_t* expert_offsets, int E,
+                                             int N, int K, int T, int k, int max_rows_per_expert,
+                                             const int32_t* perm_src, const float* gates, void* workspace,
+                                             size_t workspace_bytes, uint16_t* out, void* stream) {
+  if (T < 0 || k < 1) return GSG_ERR_INVALID_ARG;
+  if (!weight_shape_ok(E, N, K) || !gsg::gemm_supported(E)) return GSG_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)T * k > (1ll << 30)) return GSG_ERR_UNSUPPORTED_SHAPE;
+  if (T == 0) return GSG_OK;
+  const int R = T * k;
+  if (!a_codes || !a_scales || !x_tensor_scale || !w_packed || !w_tensor_scale || !expert_offsets || !perm_src ||
+      !gates || !out)
+    return GSG_ERR_INVALID_ARG;
+  if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(w_packed) || !aligned16(out))
+    return GSG_ERR_INVALID_ARG;
+  if (workspace == nullptr || !aligned16(workspace) ||
+      workspace_bytes < gsg_workspace_size(GSG_OP_COMBINE, E, N, K, T, k))
+    return GSG_ERR_WORKSPACE;
+  DeviceState* d = nullptr;
+  gsg_status_t st = device_state(&d);
+  if (st != GSG_OK) return st;
+  gsg::CombineArgs ca;
+  ca.perm_src = perm_src;
+  ca.gates = gates;
+  ca.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + combine_slot_bytes(T, k, N));
+  ca.out = out;
+  ca.k = k;
+  const int rc = gsg::launch_gemm(true, a_codes, a_scales, x_tensor_scale, w_packed, w_tensor_scale, expert_offsets,
+                                  E, N, K, R, max_rows_per_expert, workspace, 0, d->status, d->num_sms,
+                                  as_stream(stream), nullptr, nullptr, &ca);
   return rc == 0 ? GSG_OK : GSG_ERR_CUDA;
 }
 

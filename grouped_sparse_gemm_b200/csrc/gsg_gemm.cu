@@ -27,6 +27,7 @@
 #include <cuda.h>
 
 #include "gsg_internal.cuh"
+#include "gsg_launch.h"
 
 namespace gsg {
 
@@ -53,6 +54,13 @@ struct GemmParams {
   int stages, nacc, tcap;
   uint8_t* h_scales;       // SwiGLU epilogue: h scales, quad layout [N/256][R+256][4][4]
   const float* h_scale;    // SwiGLU epilogue: tensor scale of h
+  // combine epilogue (perm_src non-null): Y is the slot buffer [T*k][N] bf16 (row = flat index
+  // t*k + j of the routed pair), counters [T][N/32] (zero on entry, left zero), out [T][N] bf16
+  const int32_t* perm_src;
+  const float* gates;
+  int* counters;
+  uint16_t* out;
+  int k;
 };
 
 // ------------------------------------------------------------------ PTX wrappers
@@ -676,13 +684,48 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
           }
           __syncwarp();
           __nv_bfloat16* Y = static_cast<__nv_bfloat16*>(p.Y);
+          // combine: lane j < 16 holds the flat index f = t*k + j of chunk row j; the row goes to
+          // slot f instead of row r
+          const bool comb = p.perm_src != nullptr;
+          const int myf = (comb && lane < 16 && c0 + lane < valid) ? __ldg(p.perm_src + r0 + c0 + lane) : 0;
 #pragma unroll
           for (int k = 0; k < 2; ++k) {          // 16 tokens x 4 chunks of 16 B
             const int ci = lane + 32 * k, tok = ci >> 2, part = ci & 3;
+            const int f = __shfl_sync(0xffffffffu, myf, tok);
             if (c0 + tok < valid) {
               uint32_t a, b, cc, d;
               lds128(obuf_s + (uint32_t)(tok * 64 + part * 16), a, b, cc, d);
-              *reinterpret_cast<uint4*>(Y + (size_t)(r0 + c0 + tok) * p.N + col0 + part * 8) = make_uint4(a, b, cc, d);
+              const size_t dst = comb ? (size_t)f : (size_t)(r0 + c0 + tok);
+              *reinterpret_cast<uint4*>(Y + dst * p.N + col0 + part * 8) = make_uint4(a, b, cc, d);
+            }
+          }
+          if (comb) {
+            // count this warp's 32 features of each chunk row towards its token; the warp that
+            // brings a token's count to k reduces the token's k slots in j order (the scatter's
+            // arithmetic: fp32 products and sum, j ascending, one bf16 rounding)
+            __threadfence();
+            __syncwarp();
+            const int g32 = (int)(col0 >> 5), ng32 = p.N >> 5;
+            bool last = false;
+            if (lane < 16 && c0 + lane < valid) {
+              const int t = myf / p.k;
+              last = atomicAdd(p.counters + (size_t)t * ng32 + g32, 1) == p.k - 1;
+            }
+            unsigned todo = __ballot_sync(0xffffffffu, last);
+            if (todo) __threadfence();
+            while (todo) {
+              const int j = __ffs(todo) - 1;
+              todo &= todo - 1;
+              const int t = __shfl_sync(0xffffffffu, myf, j) / p.k;
+              float accum = 0.0f;
+              for (int jj = 0; jj < p.k; ++jj) {
+                const float gt = __ldg(p.gates + (size_t)t * p.k + jj);
+                const unsigned short yb = __ldcg(reinterpret_cast<const unsigned short*>(Y) +
+                                                 ((size_t)t * p.k + jj) * p.N + col0 + lane);
+                accum = __fadd_rn(accum, __fmul_rn(gt, __uint_as_float((uint32_t)yb << 16)));
+              }
+              p.out[(size_t)t * p.N + col0 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(accum));
+              if (lane == 0) p.counters[(size_t)t * ng32 + g32] = 0;
             }
           }
         }
@@ -819,11 +862,12 @@ static cudaError_t launch_bn(int BN, int grid, size_t smem, cudaStream_t stream,
 }
 
 // returns 0 ok, 1 cuda error, 2 tensor map failure.  h_scales / h_scale non-null: the SwiGLU
-// epilogue (sparse only; Y receives the h codes).
+// epilogue (sparse only; Y receives the h codes).  comb non-null: the combine epilogue (Y is the
+// slot buffer, bf16 output only).
 int launch_gemm(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, const float* x_scale,
                 const uint8_t* w_packed, const float* w_scale, const int32_t* off, int E, int N, int K, int R,
                 int max_rows, void* Y, int y_f32, int* status, int num_sms, cudaStream_t stream,
-                uint8_t* h_scales, const float* h_scale) {
+                uint8_t* h_scales, const float* h_scale, const CombineArgs* comb) {
   EncodeTiledFn enc = get_encode_fn();
   if (enc == nullptr) return 2;
   const bool glu = h_scales != nullptr;
@@ -868,6 +912,11 @@ int launch_gemm(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, co
   p.E = E; p.N = N; p.K = K; p.R = R; p.y_f32 = y_f32; p.rcap = rcap;
   p.stages = g.stages; p.nacc = g.nacc; p.tcap = g.tcap;
   p.h_scales = h_scales; p.h_scale = h_scale;
+  p.perm_src = comb ? comb->perm_src : nullptr;
+  p.gates = comb ? comb->gates : nullptr;
+  p.counters = comb ? comb->counters : nullptr;
+  p.out = comb ? comb->out : nullptr;
+  p.k = comb ? comb->k : 1;
   const cudaError_t e = sparse ? launch_bn<true>(g.BN, num_sms, g.smem, stream, tb, tb64, ts, p, glu)
                                : launch_bn<false>(g.BN, num_sms, g.smem, stream, tb, tb64, ts, p, false);
   return e == cudaSuccess ? 0 : 1;

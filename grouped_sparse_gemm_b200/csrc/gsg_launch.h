@@ -36,12 +36,19 @@ cudaError_t launch_unpermute(const uint16_t* Y, const int32_t* inv_perm, const f
                              uint16_t* out, int* status, int num_sms, cudaStream_t stream);
 
 // gsg_gemm.cu
+struct CombineArgs {          // the combine epilogue of the down-projection
+  const int32_t* perm_src;    // routed row -> flat index t*k + j
+  const float* gates;         // [T][k]
+  int* counters;              // [T][N/32], zero on entry, left zero
+  uint16_t* out;              // [T][N] bf16
+  int k;
+};
 bool gemm_supported(int E);
 int gemm_pick_bn(int max_rows, int R, int E);
 cudaError_t gemm_set_smem_attrs();
 int launch_gemm(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, const float* x_scale,
                 const uint8_t* w_packed, const float* w_scale, const int32_t* off, int E, int N, int K, int R,
                 int max_rows, void* Y, int y_f32, int* status, int num_sms, cudaStream_t stream,
-                uint8_t* h_scales = nullptr, const float* h_scale = nullptr);
+                uint8_t* h_scales = nullptr, const float* h_scale = nullptr, const CombineArgs* comb = nullptr);
 
 }  // namespace gsg

@@ -68,7 +68,8 @@ enum {
   GSG_OP_PACK_DENSE = 2,
   GSG_OP_ROUTE = 3,
   GSG_OP_QUANTIZE = 4,
-  GSG_OP_GEMM = 5
+  GSG_OP_GEMM = 5,
+  GSG_OP_COMBINE = 6    /* gsg_grouped_sparse_gemm_combine: token slots + completion counters */
 };
 
 /* Output element types of the grouped GEMMs. */
@@ -189,6 +190,32 @@ gsg_status_t gsg_grouped_sparse_gemm_swiglu(const uint8_t* a_codes, const uint8_
                                             const int32_t* expert_offsets, int E, int N2, int K, int R,
                                             int max_rows_per_expert, const float* h_tensor_scale,
                                             uint8_t* h_codes, uint8_t* h_scales, void* stream);
+
+/* gsg_grouped_sparse_gemm_combine -- the down-projection with the gate-weighted combine fused
+ * into the epilogue: gsg_grouped_sparse_gemm (bf16 Y) followed by gsg_unpermute_scale, in one
+ * launch, with the same result bit for bit.
+ * Paper: §D.1 (p.19): the serving integration fuses dispatch and scatter into the expert GEMMs.
+ * Every routed row is written (bf16, as Y would hold it) to its token slot f = t*k + j of the
+ * workspace instead of row r; each epilogue warp then counts its 32 features of the row towards
+ * token t, and the warp that completes a token's k contributions computes
+ *     out[t][n] = bf16_rne( sum_{j<k} fp32(gates[t][j] * slot[t*k + j][n]) )   (j ascending, from 0)
+ * -- the scatter's arithmetic and order, so the result does not depend on which warp finishes
+ * last.  R = T*k routed rows; perm_src int32 [R] and expert_offsets from gsg_moe_route_permute;
+ * gates fp32 [T][k]; out bf16 [T][N].
+ * workspace: gsg_workspace_size(GSG_OP_COMBINE, E, N, K, T, k) bytes, 16-byte aligned: the slots
+ * bf16 [T*k][N] and then int32 completion counters [T][N/32].  The counters must be zero before
+ * the first call (e.g. allocate the workspace zeroed); every call that completes leaves them zero
+ * again, so a workspace can be reused call after call.  After a device error the outputs and the
+ * counters are unspecified: zero the workspace again.  Calls that share a workspace must not run
+ * concurrently.
+ */
+gsg_status_t gsg_grouped_sparse_gemm_combine(const uint8_t* a_codes, const uint8_t* a_scales,
+                                             const float* x_tensor_scale,
+                                             const uint8_t* w_packed, const float* w_tensor_scale,
+                                             const int32_t* expert_offsets, int E, int N, int K, int T, int k,
+                                             int max_rows_per_expert, const int32_t* perm_src,
+                                             const float* gates, void* workspace, size_t workspace_bytes,
+                                             uint16_t* out, void* stream);
 
 /* ----------------------------------------------------------------------------------------
  * gsg_unpermute_scale -- gate-weighted scatter back to tokens.

@@ -465,3 +465,39 @@ def test_moe_layer_pipeline(gsg, name):
     # scatter
     ref = ounperm.unpermute_scale(Y2.cpu().view(torch.uint16).numpy(), ip, g.numpy(), L.top_k)
     np.testing.assert_array_equal(out.cpu().view(torch.uint16).numpy(), ref)
+
+
+# ---------------------------------------------------------------- down-projection with the combine epilogue
+@pytest.mark.parametrize("name", ["tiny", "30b_down_decode", "1t_down_decode_b1", "dup"])
+def test_combine_gemm_equals_gemm_then_unpermute(gsg, name):
+    """The fused combine is the unfused GEMM (bf16 Y) + scatter bit for bit, on every token, and
+    it leaves its completion counters at zero so the workspace can be reused."""
+    if name == "dup":     # a token that picks the same expert twice, and uneven expert loads
+        cfg = inputs.custom_config("dup", E=5, K=512, N=256, T=40, top_k=3, routing="zipf", zipf_s=1.5)
+        ids = inputs.routing(cfg)
+        ids[3] = torch.tensor([2, 2, 4], dtype=torch.int32)
+    else:
+        cfg = inputs.CONFIGS[name]
+        ids = inputs.routing(cfg)
+    X, g = inputs.activations(cfg).to(DEV), inputs.gates(cfg).to(DEV)
+    L = gsg.lib()
+    w = gsg.PackedSparseWeights(packed=torch.empty(L.gsg_sparse_packed_bytes(cfg.E, cfg.N, cfg.K), dtype=torch.uint8,
+                                                   device=DEV),
+                                w_scale=torch.empty(cfg.E, dtype=torch.float32, device=DEV), E=cfg.E, N=cfg.N, K=cfg.K)
+    for e in range(cfg.E):    # one expert at a time (the 1T weights are 22 GB in fp32)
+        gsg.pack_sparse_nvfp4(inputs.expert_weight(cfg, e, DEV)[None], out=w.expert(e))
+    r = gsg.moe_route_permute(ids.to(DEV), cfg.E)
+    qa = gsg.quantize_act_nvfp4(X, 32, r.inv_perm, cfg.top_k)
+    Y = gsg.grouped_sparse_gemm(qa, w, r.offsets)
+    ref = gsg.unpermute_scale(Y, r.inv_perm, g, cfg.top_k)
+    ws = gsg.combine_workspace(cfg.E, cfg.N, cfg.K, cfg.T, cfg.top_k, DEV)
+    for _ in range(2):
+        out = gsg.grouped_sparse_gemm_combine(qa, w, r, g, ws)
+        _status_ok(gsg)
+        np.testing.assert_array_equal(out.cpu().view(torch.uint16).numpy(), ref.cpu().view(torch.uint16).numpy())
+        slots = cfg.T * cfg.top_k * cfg.N * 2
+        assert not ws[(slots + 255) // 256 * 256:].any()          # counters back at zero
+    # and against the oracle scatter of the GPU's own Y
+    oref = ounperm.unpermute_scale(Y.cpu().view(torch.uint16).numpy(), r.inv_perm.cpu().numpy(), g.cpu().numpy(),
+                                   cfg.top_k)
+    np.testing.assert_array_equal(out.cpu().view(torch.uint16).numpy(), oref)
