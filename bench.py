@@ -458,6 +458,14 @@ def run_ours(args, world, rank, local):
     achieved_gbs = gemm_bytes / (gemm_ms * 1e-3) / 1e9
     gemm_tflops = flops / (gemm_ms * 1e-3) / 1e12
 
+    # the same number of bytes read by a plain library reduction (torch int64 sum) on the same
+    # harness (flush, in-graph events): what a bare read of the GEMM's traffic achieves at this size
+    rbuf = torch.empty(((w_b + a_b + y_b) + 7) // 8, dtype=torch.int64, device=dev)
+    rout = torch.empty((), dtype=torch.int64, device=dev)
+    gt_read = capture_timed(lambda: torch.sum(rbuf, dim=0, out=rout))
+    read_ms = timed_graph_ms(gt_read, max(10, args.steps // 10), flush, world)[0] if gt_read is not None else None
+    del rbuf, gt_read
+
     # end to end through the Python API: pinned host inputs -> device, step, result -> pinned host
     e2e = None
     if not args.quick:
@@ -530,6 +538,10 @@ def run_ours(args, world, rank, local):
                          "kernel": "grouped_gemm_kernel<sparse>",
                          "algorithmic_bytes_per_launch": int(gemm_bytes),
                          "peak_source": f"{peak_kind} hbm_gbs (burst copy)"},
+            "read_ceiling": None if read_ms is None else {
+                "gbs": (w_b + a_b + y_b) / (read_ms * 1e-3) / 1e9, "us": read_ms * 1e3,
+                "gemm_frac_of_it": achieved_gbs / ((w_b + a_b + y_b) / (read_ms * 1e-3) / 1e9),
+                "how": "torch int64 sum over the GEMM's algorithmic byte count, same flush and in-graph timing"},
             "e2e": e2e,
             "cpu_baseline": cpu,
             "control": control,
