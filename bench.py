@@ -205,6 +205,16 @@ class Workload:
         gsg.grouped_sparse_gemm(self.qa, self.pw, self.route.offsets, self.max_rows, out=self.Y)
         gsg.unpermute_scale(self.Y, self.route.inv_perm, self.gates, c.top_k, out=self.out)
 
+    def step_fused(self):
+        """The same step with the scatter fused into the GEMM's epilogue (bit-identical out)."""
+        c = self.cfg
+        if getattr(self, "ws_comb", None) is None:
+            self.ws_comb = gsg.combine_workspace(c.E, c.N, c.K, c.T, c.top_k, self.dev)
+        gsg.moe_route_permute(self.ids, c.E, out=self.route, workspace=self.ws_route)
+        gsg.quantize_act_nvfp4(self.X, 32, self.route.inv_perm, c.top_k, out=self.qa, workspace=self.ws_quant)
+        gsg.grouped_sparse_gemm_combine(self.qa, self.pw, self.route, self.gates, self.ws_comb, self.max_rows,
+                                        out=self.out)
+
     def launches_per_step(self) -> int:
         """Library kernels one step launches (the library's routing rule: one launch up to 1024
         rows, histogram + scatter while ceil(R/1024)*E <= 16384, else histogram + scan + scatter)."""

@@ -703,7 +703,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
             // count this warp's 32 features of each chunk row towards its token; the warp that
             // brings a token's count to k reduces the token's k slots in j order (the scatter's
             // arithmetic: fp32 products and sum, j ascending, one bf16 rounding)
-            __threadfence();
+            asm volatile("fence.acq_rel.gpu;" ::: "memory");   // this lane's slot stores before the count
             __syncwarp();
             const int g32 = (int)(col0 >> 5), ng32 = p.N >> 5;
             bool last = false;
@@ -712,17 +712,26 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
               last = atomicAdd(p.counters + (size_t)t * ng32 + g32, 1) == p.k - 1;
             }
             unsigned todo = __ballot_sync(0xffffffffu, last);
-            if (todo) __threadfence();
+            if (todo) asm volatile("fence.acq_rel.gpu;" ::: "memory");   // the other slots' stores
             while (todo) {
               const int j = __ffs(todo) - 1;
               todo &= todo - 1;
               const int t = __shfl_sync(0xffffffffu, myf, j) / p.k;
               float accum = 0.0f;
-              for (int jj = 0; jj < p.k; ++jj) {
-                const float gt = __ldg(p.gates + (size_t)t * p.k + jj);
-                const unsigned short yb = __ldcg(reinterpret_cast<const unsigned short*>(Y) +
-                                                 ((size_t)t * p.k + jj) * p.N + col0 + lane);
-                accum = __fadd_rn(accum, __fmul_rn(gt, __uint_as_float((uint32_t)yb << 16)));
+              for (int j0 = 0; j0 < p.k; j0 += 8) {   // eight slots' loads in flight, then the sum in order
+                float gt[8];
+                unsigned short yb[8];
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                  const bool in = j0 + jj < p.k;
+                  gt[jj] = in ? __ldg(p.gates + (size_t)t * p.k + j0 + jj) : 0.0f;
+                  yb[jj] = in ? __ldcg(reinterpret_cast<const unsigned short*>(Y) + ((size_t)t * p.k + j0 + jj) * p.N +
+                                       col0 + lane)
+                              : (unsigned short)0;
+                }
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj)
+                  if (j0 + jj < p.k) accum = __fadd_rn(accum, __fmul_rn(gt[jj], __uint_as_float((uint32_t)yb[jj] << 16)));
               }
               p.out[(size_t)t * p.N + col0 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(accum));
               if (lane == 0) p.counters[(size_t)t * ng32 + g32] = 0;
