@@ -6,7 +6,9 @@
 // activations are packed in corresponding scale blocks.
 //
 // Launch 1 (skipped when the caller supplies s_x): partial max|X| per block, 128-bit loads,
-// warp-shuffle reductions.  Launch 2: every block folds the partials into s_x = amax/2688,
+// warp-shuffle reductions.  Launch 2, 32-element blocks (the sparse path): one lane per block
+// (act_quant32_kernel, below).  Launch 2, 16-element blocks (the dense control): every block
+// folds the partials into s_x = amax/2688,
 // then each warp quantizes 256 consecutive elements of one token row at a time (8 per lane, one
 // 128-bit load), groups of 4 lanes (2 for 16-element blocks) combine their maxima into the
 // block amax, the four scales of one MMA k-block are gathered into a 32-bit word, and the
@@ -74,6 +76,135 @@ struct QuantParams {
   int* status;
 };
 
+// The tensor scale: the caller's value, or max|X| folded from the partial maxima (block-wide;
+// every thread of the block must call it).
+__device__ __forceinline__ float quant_tensor_scale(const QuantParams& p, float* red, float* s_sh) {
+  if (p.s_in != nullptr) {
+    if (threadIdx.x == 0) *s_sh = __ldg(p.s_in);
+  } else {
+    float v = 0.0f;
+    for (int i = threadIdx.x; i < p.nparts; i += blockDim.x) v = fmaxf(v, p.partial[i]);
+    v = warp_max(v);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      float w = threadIdx.x < (int)(blockDim.x >> 5) ? red[threadIdx.x] : 0.0f;
+      w = warp_max(w);
+      if (threadIdx.x == 0) *s_sh = tensor_scale_from_amax(w);
+    }
+  }
+  __syncthreads();
+  const float s = *s_sh;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *p.s_out = s;
+  return s;
+}
+
+// Zero the quad scale entries that refer to rows >= R (no routed row writes them).
+__device__ __forceinline__ void quant_zero_padding(const QuantParams& p) {
+  uint32_t* sw = reinterpret_cast<uint32_t*>(p.scales);
+  const int KBa = p.K / (4 * p.sf);
+  const int r_lo = p.R > 96 ? p.R - 96 : 0;
+  const int span = p.rcap - r_lo;                 // at most 352 rows
+  const int npad = KBa * span * 4;                // K / 64 * 352 * 4 < 2^31
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < npad; i += gridDim.x * blockDim.x) {
+    const int c = i & 3;
+    const int rest = i >> 2;
+    const int rr = r_lo + rest % span;
+    const int kb = rest / span;
+    if (rr + 32 * c >= p.R) sw[((size_t)kb * p.rcap + rr) * 4 + c] = 0u;
+  }
+}
+
+// 32-element blocks: one lane quantizes one whole block (four 128-bit loads, the block max, one
+// scale, 16 bytes of codes), so the per-block work is not repeated across lanes.  Four
+// consecutive lanes hold the four blocks of one MMA k-block (K % 128 == 0) and assemble its scale
+// word; lane c of the four writes quad entry c of each routed row.  Lanes load their token's
+// routed rows themselves (lanes of one token read the same addresses).
+constexpr int kQ32Rows = 8;   // routed rows loaded ahead with the block (the rest on demand)
+
+struct Quant32Unit {
+  uint4 x[4];
+  int rows[kQ32Rows];
+  int t, b;
+  bool valid;
+};
+
+__device__ __forceinline__ void quant32_fetch(const QuantParams& p, long long u, long long U, int bpr, Quant32Unit& q) {
+  q.valid = u < U;
+  const unsigned u32 = (unsigned)(q.valid ? u : 0);   // U = T*K/32 < 2^31 (checked on the host)
+  q.t = int(u32 / (unsigned)bpr);
+  q.b = int(u32 % (unsigned)bpr);
+  const uint4* src = reinterpret_cast<const uint4*>(p.X + (size_t)q.t * p.K + (size_t)q.b * 32);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) q.x[i] = q.valid ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+  for (int j = 0; j < kQ32Rows; ++j)
+    q.rows[j] = (q.valid && j < p.k) ? (p.inv_perm != nullptr ? __ldg(p.inv_perm + (size_t)q.t * p.k + j) : q.t) : -1;
+}
+
+__global__ void __launch_bounds__(128)
+act_quant32_kernel(QuantParams p) {
+  __shared__ float red[4];
+  __shared__ float s_sh;
+  pdl_launch_dependents();
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int bpr = p.K / 32;                                    // blocks per row
+  const long long U = (long long)p.T * bpr;
+  const int gwarp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  const long long wstep = (long long)nwarps * 32;
+  long long base = (long long)gwarp * 32;
+  Quant32Unit cur;
+  quant32_fetch(p, base + lane, U, bpr, cur);                  // before the tensor scale is known
+  const float s = quant_tensor_scale(p, red, &s_sh);
+  const float six_s = __fmul_rn(6.0f, s);
+  uint32_t* sw = reinterpret_cast<uint32_t*>(p.scales);
+  for (; base < U; base += wstep) {
+    const Quant32Unit q = cur;
+    if (base + wstep < U) quant32_fetch(p, base + wstep + lane, U, bpr, cur);
+    float x[32];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t w[4] = {q.x[i].x, q.x[i].y, q.x[i].z, q.x[i].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        x[8 * i + 2 * j] = bf16_bits_to_f32(w[j] & 0xFFFFu);
+        x[8 * i + 2 * j + 1] = bf16_bits_to_f32(w[j] >> 16);
+      }
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(x[i]));
+    const BlockScale bs = block_scale_cvt(amax, six_s, s);
+    uint32_t cw[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float xs[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) xs[j] = __fmul_rn(x[8 * i + j], bs.inv);
+      cw[i] = e2m1_encode8_cvt(xs);
+    }
+    const int g = lane & ~3;
+    const uint32_t word = __shfl_sync(0xffffffffu, bs.sc, g) | (__shfl_sync(0xffffffffu, bs.sc, g + 1) << 8) |
+                          (__shfl_sync(0xffffffffu, bs.sc, g + 2) << 16) | (__shfl_sync(0xffffffffu, bs.sc, g + 3) << 24);
+    if (!q.valid) continue;
+    const int kb = q.b >> 2, cq = lane & 3;
+    auto dispatch = [&](int row) {
+      if (row < 0 || row >= p.R) { set_status(p.status, GSG_ERR_BAD_ROUTING); return; }
+      *reinterpret_cast<uint4*>(p.codes + (size_t)row * (p.K / 2) + (size_t)q.b * 16) =
+          make_uint4(cw[0], cw[1], cw[2], cw[3]);
+      const int rr = row - 32 * cq;
+      if (rr >= 0) sw[((size_t)kb * p.rcap + rr) * 4 + cq] = word;
+    };
+#pragma unroll
+    for (int j = 0; j < kQ32Rows; ++j)
+      if (j < p.k) dispatch(q.rows[j]);
+    for (int j = kQ32Rows; j < p.k; ++j) dispatch(__ldg(p.inv_perm + (size_t)q.t * p.k + j));
+  }
+  quant_zero_padding(p);
+}
+
 // One warp-iteration covers 256 consecutive elements of one token row (K % 256 == 0): lane L
 // holds elements 8L..8L+7 of them, and lane j < k also holds the token's j-th routed row.
 struct QuantSlice {
@@ -108,23 +239,7 @@ act_quant_kernel(QuantParams p) {
   if (base < U) quant_fetch(p, base, units_per_row, lane, cur);
 
   // ---- tensor scale
-  if (p.s_in != nullptr) {
-    if (threadIdx.x == 0) s_sh = __ldg(p.s_in);
-  } else {
-    float v = 0.0f;
-    for (int i = threadIdx.x; i < p.nparts; i += blockDim.x) v = fmaxf(v, p.partial[i]);
-    v = warp_max(v);
-    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
-    __syncthreads();
-    if (threadIdx.x < 32) {
-      float w = threadIdx.x < kQuantMainThreads / 32 ? red[threadIdx.x] : 0.0f;
-      w = warp_max(w);
-      if (threadIdx.x == 0) s_sh = tensor_scale_from_amax(w);
-    }
-  }
-  __syncthreads();
-  const float s = s_sh;
-  if (blockIdx.x == 0 && threadIdx.x == 0) *p.s_out = s;
+  const float s = quant_tensor_scale(p, red, &s_sh);
   const float six_s = __fmul_rn(6.0f, s);
 
   // a 32-element block is 4 lanes (16-element block: 2 lanes); one MMA k-block's four scales
@@ -191,18 +306,7 @@ act_quant_kernel(QuantParams p) {
       }
     }
   }
-  // ---- zero the quad entries that refer to rows >= R
-  const int KBa = p.K / (4 * p.sf);
-  const int r_lo = p.R > 96 ? p.R - 96 : 0;
-  const int span = p.rcap - r_lo;                 // at most 352 rows
-  const int npad = KBa * span * 4;                // K / 128 * 352 * 4 < 2^31
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < npad; i += gridDim.x * blockDim.x) {
-    const int c = i & 3;
-    const int rest = i >> 2;
-    const int rr = r_lo + rest % span;
-    const int kb = rest / span;
-    if (rr + 32 * c >= p.R) sw[((size_t)kb * p.rcap + rr) * 4 + c] = 0u;
-  }
+  quant_zero_padding(p);
 }
 
 int quant_partials(long long n_elems) {
@@ -227,11 +331,12 @@ cudaError_t launch_quant(const uint16_t* X, int T, int K, int sf, const int32_t*
   p.X = X; p.inv_perm = inv_perm; p.s_in = s_in; p.partial = partial; p.nparts = P;
   p.T = T; p.K = K; p.sf = sf; p.k = k; p.R = T * k; p.rcap = T * k + kActScalePadRows;
   p.codes = codes; p.scales = scales; p.s_out = s_out; p.status = status;
-  const long long units = (long long)T * (K / 8);
+  const long long units = (long long)T * (K / (sf == 32 ? 32 : 8));   // lanes of work
   const long long pad = (long long)(K / (4 * sf)) * (T * k + kActScalePadRows - (T * k > 96 ? T * k - 96 : 0)) * 4;
   long long blocks = ((units > pad ? units : pad) + kQuantMainThreads - 1) / kQuantMainThreads;
   if (blocks < 1) blocks = 1;
   if (blocks > (long long)num_sms * 16) blocks = (long long)num_sms * 16;
+  if (sf == 32) return launch_pdl(act_quant32_kernel, (unsigned)blocks, kQuantMainThreads, 0, stream, p);
   return launch_pdl(act_quant_kernel, (unsigned)blocks, kQuantMainThreads, 0, stream, p);
 }
 
