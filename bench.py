@@ -4,14 +4,18 @@
 One step = one pass of the hot path over one batch of routed tokens, inputs resident in HBM:
 moe_route_permute -> quantize_act_nvfp4 (fused dispatch) -> grouped_sparse_gemm ->
 unpermute_scale, replayed as one CUDA graph (the weights are packed once, offline, as in
-serving).  The L2 cache is flushed (a 256 MB write) before every timed step; each step is timed
-with CUDA events on the launching stream and the flush is left outside the events.
+serving).  The L2 cache is flushed before every timed step (a 256 MB write, then a 256 MB read
+of another buffer, so that L2 holds neither the step's inputs nor dirty lines whose write-back
+would land in the step); each step is timed with CUDA events on the launching stream and the
+flush is left outside the events.
 
 Reported (rank 0, one JSON line):
   value     dense-equivalent TFLOP/s of the whole step (2*R*N*K per step, the unit the sparse
             NVFP4 tensor peak is quoted in), summed over ranks / max time over ranks
   e2e       the same metric through the Python API with host (pinned) inputs and outputs,
-            host<->device copies inside the timed region
+            host<->device copies inside the timed region: a double-buffered serving loop
+            (uploads, compute and downloads of neighbouring steps overlap on three streams);
+            e2e.serial is the same calls one step at a time
   roofline  the grouped GEMM kernel alone: algorithmic bytes per launch / its event time
             against the measured HBM copy bandwidth
   cpu_baseline  the CPU oracle timed on a bounded sample of the same workload (N=1, rank 0)
@@ -48,6 +52,24 @@ METRIC = "grouped sparse-NVFP4 GEMM TFLOP/s + weight GB/s, as % of B200 roofline
 SPARSE_NVFP4_PEAK_TFLOPS_NOMINAL = 18000.0     # the pages' sparse NVFP4 figure (dense-equivalent)
 HBM_NOMINAL_GBS = 8000.0
 L2_FLUSH_BYTES = 256 << 20
+
+
+class L2Flush:
+    """Flush of the 126 MB L2 before a timed step: a 256 MB write, then a 256 MB read of a
+    second buffer (the read writes back the dirty lines the write left, outside the timing, and
+    leaves L2 full of clean lines that no step touches), then a random 0-4 µs spin.  The spin
+    spreads the step's start over the event timer's tick (about 2 µs on B200), so that the mean
+    of many event intervals is not biased by the tick."""
+
+    def __init__(self, dev):
+        self.w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        self.r = torch.ones(L2_FLUSH_BYTES // 8, dtype=torch.int64, device=dev)
+        self.rng = np.random.default_rng(1234)
+
+    def fill_(self, v: int):
+        self.w.fill_(v)
+        self.r.sum()
+        torch.cuda._sleep(int(self.rng.integers(0, 8192)))
 
 
 # ------------------------------------------------------------------ distributed plumbing
@@ -216,10 +238,10 @@ class Workload:
                                         out=self.out)
 
     def launches_per_step(self) -> int:
-        """Library kernels one step launches (the library's routing rule: one launch up to 1024
+        """Library kernels one step launches (the library's routing rule: one launch up to 2048
         rows, histogram + scatter while ceil(R/1024)*E <= 16384, else histogram + scan + scatter)."""
         R, E = self.cfg.R, self.cfg.E
-        route = 1 if R <= 1024 else (2 if -(-R // 1024) * E <= 16384 else 3)
+        route = 1 if R <= 2048 else (2 if -(-R // 1024) * E <= 16384 else 3)
         return route + 2 + 1 + 1        # route, amax + quantize, GEMM, scatter
 
     def gemm(self):
@@ -276,7 +298,7 @@ def capture_timed(fn):
         return None
 
 
-def timed_graph_ms(gt, steps: int, flush_buf: torch.Tensor, world: int):
+def timed_graph_ms(gt, steps: int, flush_buf: "L2Flush", world: int):
     """Mean of the in-graph event interval over `steps` replays, L2 flushed before each."""
     g, (e0, e1) = gt
     barrier(world)
@@ -292,7 +314,7 @@ def timed_graph_ms(gt, steps: int, flush_buf: torch.Tensor, world: int):
     return sum(ts) / steps, ts
 
 
-def timed_ms(fn, steps: int, flush_buf: torch.Tensor, world: int):
+def timed_ms(fn, steps: int, flush_buf: "L2Flush", world: int):
     """Mean device time of fn over `steps` runs, L2 flushed before each (outside the events)."""
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
@@ -307,6 +329,99 @@ def timed_ms(fn, steps: int, flush_buf: torch.Tensor, world: int):
     barrier(world)
     ts = [a.elapsed_time(b) for a, b in zip(starts, ends)]
     return sum(ts) / steps, ts
+
+
+class E2EPipeline:
+    """End to end through the public API as a serving loop runs it: every step copies its inputs
+    (X, top-k ids, gates) from pinned host memory to the device on an upload stream, runs route ->
+    quantize -> GEMM -> scatter on the compute stream, and copies its result to pinned host memory
+    on a download stream.  Inputs and results are double-buffered, so step i's upload and step
+    i-1's download overlap step i-1's and step i's compute.  The packed weights rotate over three
+    replicas (3 x 138 MB at the 30B prefill shape, against a 126 MB L2): a step never finds the
+    weights of the step before it in L2, so no flush is needed between steps.  Timed: K steps
+    between an event on the upload stream before the first upload and one on the download
+    stream after the last download."""
+
+    NW = 3
+
+    def __init__(self, wl: "Workload"):
+        self.wl, c = wl, wl.cfg
+        self.X_p, self.ids_p, self.g_p = wl.X_h.pin_memory(), wl.ids_h.pin_memory(), wl.gates_h.pin_memory()
+        self.out_p = [torch.empty(c.T, c.N, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        self.X = [wl.X, torch.empty_like(wl.X)]
+        self.ids = [wl.ids, torch.empty_like(wl.ids)]
+        self.gates = [wl.gates, torch.empty_like(wl.gates)]
+        self.out = [wl.out, torch.empty_like(wl.out)]
+        self.pw = [wl.pw] + [gsg.PackedSparseWeights(packed=wl.pw.packed.clone(), w_scale=wl.pw.w_scale.clone(),
+                                                     E=c.E, N=c.N, K=c.K) for _ in range(self.NW - 1)]
+        self.up, self.comp, self.down = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+        self.uploaded = [torch.cuda.Event() for _ in range(2)]
+        self.computed = [torch.cuda.Event() for _ in range(2)]
+        self.downloaded = [torch.cuda.Event() for _ in range(2)]
+
+    def h2d_bytes(self) -> int:
+        return self.X_p.numel() * 2 + self.ids_p.numel() * 4 + self.g_p.numel() * 4
+
+    def d2h_bytes(self) -> int:
+        return self.out_p[0].numel() * 2
+
+    def step(self, i: int, first: bool):
+        wl, c, b = self.wl, self.wl.cfg, i & 1
+        with torch.cuda.stream(self.up):
+            if not first:
+                self.up.wait_event(self.computed[b])          # step i-2 is done reading set b
+            self.X[b].copy_(self.X_p, non_blocking=True)
+            self.ids[b].copy_(self.ids_p, non_blocking=True)
+            self.gates[b].copy_(self.g_p, non_blocking=True)
+            self.uploaded[b].record(self.up)
+        s = self.comp
+        s.wait_event(self.uploaded[b])
+        if not first:
+            s.wait_event(self.downloaded[b])                  # step i-2's result has left out[b]
+        gsg.moe_route_permute(self.ids[b], c.E, out=wl.route, workspace=wl.ws_route, stream=s)
+        gsg.quantize_act_nvfp4(self.X[b], 32, wl.route.inv_perm, c.top_k, out=wl.qa, workspace=wl.ws_quant,
+                               stream=s)
+        gsg.grouped_sparse_gemm(wl.qa, self.pw[i % self.NW], wl.route.offsets, wl.max_rows, out=wl.Y, stream=s)
+        gsg.unpermute_scale(wl.Y, wl.route.inv_perm, self.gates[b], c.top_k, out=self.out[b], stream=s)
+        self.computed[b].record(s)
+        with torch.cuda.stream(self.down):
+            self.down.wait_event(self.computed[b])
+            self.out_p[b].copy_(self.out[b], non_blocking=True)
+            self.downloaded[b].record(self.down)
+
+    def run(self, steps: int) -> float:
+        """Mean ms per step over `steps` pipelined steps (after a synchronised start)."""
+        torch.cuda.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(self.up)
+        self.comp.wait_stream(self.up)
+        self.down.wait_stream(self.up)
+        h0 = time.perf_counter()
+        for i in range(steps):
+            self.step(i, first=i < 2)
+        self.host_ms = (time.perf_counter() - h0) * 1e3 / steps     # host time to issue one step
+        self.down.wait_stream(self.comp)
+        self.down.wait_stream(self.up)
+        t1.record(self.down)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1) / steps
+
+    def copy_ms(self, reps: int = 20):
+        """Device time of one step's uploads alone and of its download alone."""
+        res = []
+        for fn in (lambda: (self.X[0].copy_(self.X_p, non_blocking=True),
+                            self.ids[0].copy_(self.ids_p, non_blocking=True),
+                            self.gates[0].copy_(self.g_p, non_blocking=True)),
+                   lambda: self.out_p[0].copy_(self.out[0], non_blocking=True)):
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(reps):
+                fn()
+            b.record()
+            torch.cuda.synchronize()
+            res.append(a.elapsed_time(b) / reps)
+        return res
 
 
 # ------------------------------------------------------------------ CPU oracle (baseline / reference arm)
@@ -365,7 +480,8 @@ def blas_threads() -> int:
     return os.cpu_count() or 1
 
 
-def workload_config(cfg, l2="flushed before every timed step (256 MB write, outside the events)"):
+def workload_config(cfg, l2="flushed before every timed step (256 MB write + 256 MB read of another buffer, "
+                              "outside the events)"):
     return {"workload": f"{cfg.name}: E={cfg.E} K={cfg.K} N={cfg.N}, {cfg.T} tokens top-{cfg.top_k} "
                         f"(R={cfg.R}), routing {cfg.routing}"
                         + (f" s={cfg.zipf_s}" if cfg.routing == "zipf" else ""),
@@ -426,7 +542,7 @@ def run_ours(args, world, rank, local):
     gsg.load_library()
     cfg = inputs.CONFIGS[args.config]
     wl = Workload(cfg, dev, with_dense=not args.quick)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     wl.step()
     torch.cuda.synchronize()
     st = gsg.get_device_status()
@@ -479,23 +595,33 @@ def run_ours(args, world, rank, local):
     # end to end through the Python API: pinned host inputs -> device, step, result -> pinned host
     e2e = None
     if not args.quick:
-        X_p, ids_p, g_p = wl.X_h.pin_memory(), wl.ids_h.pin_memory(), wl.gates_h.pin_memory()
-        out_p = torch.empty(cfg.T, cfg.N, dtype=torch.bfloat16).pin_memory()
+        pipe = E2EPipeline(wl)
+        pipe.run(max(3, args.warmup))
+        barrier(world)
+        e2e_ms = max_over_ranks(pipe.run(max(10, args.steps // 10)), world, dev)
+        host_ms = pipe.host_ms
+        h2d_ms, d2h_ms = pipe.copy_ms()
 
+        # the same calls one step at a time (copies, step, copy back), L2 flushed before each
         def e2e_step():
-            wl.X.copy_(X_p, non_blocking=True)
-            wl.ids.copy_(ids_p, non_blocking=True)
-            wl.gates.copy_(g_p, non_blocking=True)
-            wl.step()
-            out_p.copy_(wl.out, non_blocking=True)
-        for _ in range(3):
-            e2e_step()
-        e2e_ms, _ = timed_ms(e2e_step, max(10, args.steps // 10), flush, world)
-        e2e_ms = max_over_ranks(e2e_ms, world, dev)
-        h2d = X_p.numel() * 2 + ids_p.numel() * 4 + g_p.numel() * 4
+            cur = torch.cuda.current_stream()
+            for st in (pipe.up, pipe.comp, pipe.down):
+                st.wait_stream(cur)
+            pipe.step(0, first=True)
+            cur.wait_stream(pipe.down)
+        serial_ms = max_over_ranks(timed_ms(e2e_step, max(10, args.steps // 10), flush, world)[0], world, dev)
         e2e = {"value": job_value(flops, world, e2e_ms), "unit": "TFLOP/s", "ms_per_step": e2e_ms,
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(out_p.numel() * 2),
-               "path": "pinned host -> device copies, 4 library calls via the Python binding, result -> pinned host"}
+               "h2d_bytes_per_step": int(pipe.h2d_bytes()), "d2h_bytes_per_step": int(pipe.d2h_bytes()),
+               "path": "per step: pinned host -> device copies (upload stream), 4 library calls via the Python "
+                       "binding (compute stream), result -> pinned host (download stream); double-buffered so "
+                       "uploads and downloads overlap neighbouring steps' compute; weights rotate over 3 "
+                       "replicas, no L2 flush",
+               "parts_us": {"host_issue_per_step": host_ms * 1e3, "h2d_alone": h2d_ms * 1e3,
+                            "d2h_alone": d2h_ms * 1e3},
+               "serial": {"value": job_value(flops, world, serial_ms), "ms_per_step": serial_ms,
+                          "how": "one step at a time, every stream joined before the end event, L2 flushed "
+                                 "before each step"}}
+        del pipe
 
     control = None
     if not args.quick:
@@ -578,7 +704,7 @@ def run_all_configs(args, local):
     dev = torch.device(f"cuda:{local}")
     torch.cuda.set_device(dev)
     gsg.load_library()
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     peaks, kind = measured_peaks()
     hbm = float(peaks["hbm_gbs"])
     names = args.configs.split(",") if args.configs else list(inputs.CONFIGS)
@@ -620,7 +746,8 @@ def run_all_configs(args, local):
                     "sparse_speedup": res["dense_gemm_us"] / res["gemm_us"],
                     "gemm_frac_of_read": res["read_same_bytes_us"] / res["gemm_us"],
                     "hbm_peak_gbs": hbm, "peak_source": kind, "reps": reps,
-                    "timing": "in-graph CUDA events, L2 flushed (256 MB write) before every replay"})
+                    "timing": "in-graph CUDA events, L2 flushed (256 MB write + 256 MB read of another buffer) "
+                              "before every replay"})
         print(json.dumps(res), flush=True)
         del wl
         torch.cuda.empty_cache()
@@ -705,7 +832,7 @@ def run_layer(args, local):
     gsg.load_library()
     L = inputs.LAYERS[args.layer]
     wl = LayerWorkload(L, dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     wl.step()
     torch.cuda.synchronize()
     st = gsg.get_device_status()
@@ -726,7 +853,8 @@ def run_layer(args, local):
         "tflops_dense_equivalent": wl.flops() / (ms * 1e-3) / 1e12,
         "weight_gbs": wl.weight_bytes() / (ms * 1e-3) / 1e9, "h_tensor_scale": float(wl.h_scale.item()),
         "kernels": "route, amax + quantize, up-projection + SwiGLU + NVFP4 of h, down-projection, unpermute",
-        "timing": "in-graph CUDA events around the layer, L2 flushed (256 MB write) before every replay"}),
+        "timing": "in-graph CUDA events around the layer, L2 flushed (256 MB write + 256 MB read of another "
+                  "buffer) before every replay"}),
           flush=True)
 
 
@@ -761,7 +889,7 @@ def run_sweep(args, local):
     gsg.load_library()
     L = gsg.lib()
     u8 = dict(dtype=torch.uint8, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, **u8)
+    flush = L2Flush(dev)
     energy = Energy(local)
     Gs = [int(x) for x in args.sweep_g.split(",")]
     Ns = [int(x) for x in args.sweep_n.split(",")]

@@ -15,7 +15,7 @@
 // device address comes from cudaGetSymbolAddress, taken once per device (with that device
 // current) by the entry point's first call on that device.
 //
-// Limits: R <= 1024 uses no scratch.  Above that the routing needs the workspace that
+// Limits: R <= 2048 uses no scratch.  Above that the routing needs the workspace that
 // gsg_workspace_size(GSG_OP_ROUTE, ...) reports: at most 128 KiB while it cuts R into 1024-row
 // chunks, else 2 * ceil(R / 8192) * E int32.  So a call is accepted when ceil(R / 8192) * E <=
 // 32768 (E = 384: R up to 696,320 rows; E = 128: R up to 2,097,152); larger requests return

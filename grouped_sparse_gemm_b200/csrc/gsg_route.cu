@@ -9,9 +9,12 @@
 // indices (one per thread) while ceil(R/1024) * E <= 16384 (a workspace of at most 128 KiB),
 // else 8192 (eight per thread).  Each warp owns a contiguous run of its chunk; lanes holding
 // the same id are found with one ballot per id bit, which gives each index its rank among equal
-// ids of its warp, and per-warp histograms live in shared memory (32 x E ints).  R <= 1024 is
-// one launch; larger R is histogram -> (scan) -> scatter over a [chunks x E] workspace, the scan
-// folded into the scatter for 1024-index chunks.  Only integer arithmetic: the result is
+// ids of its warp, and per-warp histograms live in shared memory (32 x E ints).  R <= 2048 is
+// one launch of one block (up to 2 indices per thread, no workspace): at these sizes the pass is
+// latency-bound and a second launch costs more than the block's extra round (measured: at
+// R = 4096 four indices per thread in one block are slower than two launches).  Larger R is
+// histogram -> (scan) -> scatter over a [chunks x E] workspace, the scan folded into the
+// scatter for 1024-index chunks.  Only integer arithmetic: the result is
 // deterministic.
 #include "gsg_internal.cuh"
 
@@ -20,6 +23,7 @@ namespace gsg {
 constexpr int kRouteThreads = 1024;
 constexpr int kRouteMaxE = 1024;
 constexpr long long kSmallChunkMaxCells = 16384;   // chunks x experts of the 1024-index path
+constexpr int kSingleMaxR = 2048;                  // one block, up to 2 indices per thread
 
 int route_chunk_size(int R, int E) {
   return ((long long)(R + 1023) / 1024) * E <= kSmallChunkMaxCells ? 1024 : 8192;
@@ -129,7 +133,9 @@ __device__ __forceinline__ void warp_run(int c0, int c1, int& f0, int& f1) {
   f1 = min(f0 + 32 * kPer, c1);
 }
 
-// One chunk holds everything (R <= 1024): histogram, scan, scatter in one launch.
+// One block holds everything (R <= 1024 * kPer, kPer indices per thread): histogram, scan,
+// scatter in one launch.
+template <int kPer>
 __global__ void __launch_bounds__(kRouteThreads)
 route_single_kernel(const int32_t* __restrict__ ids, int R, int E, int32_t* off, int32_t* perm_src,
                     int32_t* inv_perm, int* status) {
@@ -140,13 +146,13 @@ route_single_kernel(const int32_t* __restrict__ ids, int R, int E, int32_t* off,
   for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) hist[i] = 0;
   const int warp = threadIdx.x >> 5;
   int f0, f1;
-  warp_run<1>(0, R, f0, f1);
+  warp_run<kPer>(0, R, f0, f1);
   pdl_wait();
-  int x[1];
-  unsigned m[1];
-  warp_load_ids<1>(ids, f0, f1, E, x, status);
+  int x[kPer];
+  unsigned m[kPer];
+  warp_load_ids<kPer>(ids, f0, f1, E, x, status);
   __syncthreads();
-  warp_histogram<1>(x, m, f0, f1, hist + warp * E, key_bits(E));
+  warp_histogram<kPer>(x, m, f0, f1, hist + warp * E, key_bits(E));
   __syncthreads();
   const int ex = threadIdx.x;
   int tot = 0;
@@ -164,7 +170,7 @@ route_single_kernel(const int32_t* __restrict__ ids, int R, int E, int32_t* off,
   }
   if (ex == 0) off[E] = total;
   __syncthreads();
-  warp_scatter<1>(x, m, f0, f1, hist + warp * E, perm_src, inv_perm);
+  warp_scatter<kPer>(x, m, f0, f1, hist + warp * E, perm_src, inv_perm);
 }
 
 // Multi-chunk path, launch 1: per-chunk histograms -> ws_hist[chunk][E].
@@ -269,7 +275,7 @@ route_scatter_kernel(const int32_t* __restrict__ ids, int R, int E, const int* w
 }
 
 int route_chunks(int R, int E) {
-  if (R <= 1024) return 1;
+  if (R <= kSingleMaxR) return 1;
   const int c = route_chunk_size(R, E);
   return (R + c - 1) / c;
 }
@@ -283,8 +289,9 @@ bool route_supported(int E) { return E >= 1 && E <= kRouteMaxE; }
 
 cudaError_t route_set_smem_attrs() {
   const int bytes = 32 * kRouteMaxE * (int)sizeof(int);
-  const cudaError_t errs[5] = {
-      cudaFuncSetAttribute(route_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
+  const cudaError_t errs[6] = {
+      cudaFuncSetAttribute(route_single_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
+      cudaFuncSetAttribute(route_single_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
       cudaFuncSetAttribute(route_hist_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
       cudaFuncSetAttribute(route_hist_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
       cudaFuncSetAttribute(route_scatter_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
@@ -299,8 +306,8 @@ cudaError_t launch_route(const int32_t* ids, int R, int E, int32_t* off, int32_t
   const size_t smem = (size_t)32 * E * sizeof(int);
   const int nc = route_chunks(R, E);
   if (nc <= 1) {
-    return launch_pdl(route_single_kernel, 1, kRouteThreads, smem, stream, ids, R, E, off, perm_src, inv_perm,
-                      status);
+    auto single = R <= 1024 ? route_single_kernel<1> : route_single_kernel<2>;
+    return launch_pdl(single, 1, kRouteThreads, smem, stream, ids, R, E, off, perm_src, inv_perm, status);
   }
   int* ws_hist = static_cast<int*>(ws);
   int* ws_base = ws_hist + (size_t)nc * E;

@@ -237,7 +237,7 @@ gsg_status_t gsg_unpermute_scale(const uint16_t* Y, const int32_t* inv_perm, con
  * outputs, result and errors as gsg_moe_route_permute; the workspace is replaced by a fixed
  * 256 KiB device array inside the library, which every GPU that loads the library holds until
  * the process exits.  The call allocates nothing.
- * Limit: R = T*k <= 1024 needs no scratch; above that ceil(R/8192) * E <= 32768
+ * Limit: R = T*k <= 2048 needs no scratch; above that ceil(R/8192) * E <= 32768
  * (E = 384: R <= 696,320; E = 128: R <= 2,097,152), else GSG_ERR_UNSUPPORTED_SHAPE with no
  * launch.  The first call on a device sets up that device (the library's per-device set-up and
  * the scratch's device address); make that first call before any stream capture begins.

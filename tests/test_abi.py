@@ -41,7 +41,9 @@ def test_sizes(L):
     assert L.gsg_act_scales_bytes(10, 256, 32) == 2 * (10 + 256) * 16
     assert L.gsg_workspace_size(gsg.OP_ROUTE, 384, 0, 0, 64, 8) == 0          # single-launch routing
     assert L.gsg_workspace_size(gsg.OP_ROUTE, 384, 0, 0, 8192, 8) == 2 * 8 * 384 * 4   # 8192-row chunks
+    assert L.gsg_workspace_size(gsg.OP_ROUTE, 128, 0, 0, 256, 8) == 0             # one block up to 2048 rows
     assert L.gsg_workspace_size(gsg.OP_ROUTE, 128, 0, 0, 512, 8) == 2 * 4 * 128 * 4    # 1024-row chunks
+    assert L.gsg_workspace_size(gsg.OP_ROUTE, 128, 0, 0, 2000, 8) == 2 * 16 * 128 * 4  # 1024-row chunks
     assert L.gsg_workspace_size(gsg.OP_GEMM, 384, 4096, 7168, 8192, 8) == 0
 
 

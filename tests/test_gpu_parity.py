@@ -69,7 +69,8 @@ def test_pack_flags_nonfinite(gsg):
 @pytest.mark.parametrize("T,k,E,mode", [(32, 2, 4, "uniform"), (512, 8, 128, "zipf"), (64, 8, 128, "uniform"),
                                         (1025, 4, 7, "zipf"), (8192, 8, 384, "zipf"), (3, 1, 1, "uniform"),
                                         (256, 8, 384, "uniform"), (9000, 8, 512, "zipf"),
-                                        (1500, 1, 1024, "uniform")])
+                                        (1500, 1, 1024, "uniform"), (256, 8, 128, "zipf"),
+                                        (2049, 1, 16, "zipf"), (2000, 8, 64, "zipf")])
 def test_route_matches_oracle(gsg, T, k, E, mode):
     cfg = inputs.custom_config("r", E=E, K=256, N=128, T=T, top_k=k, routing=mode, zipf_s=1.1)
     ids = inputs.routing(cfg) if k <= E else torch.zeros(T, k, dtype=torch.int32)
