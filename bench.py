@@ -2,8 +2,8 @@
 """Benchmark of the grouped sparse-NVFP4 expert GEMM path on B200.
 
 One step = one pass of the hot path over one batch of routed tokens, inputs resident in HBM:
-moe_route_permute -> quantize_act_nvfp4 (fused dispatch) -> grouped_sparse_gemm ->
-unpermute_scale, replayed as one CUDA graph (the weights are packed once, offline, as in
+moe_dispatch_nvfp4 (routing + activation quantization into routed order) -> grouped_sparse_gemm
+-> unpermute_scale, replayed as one CUDA graph (the weights are packed once, offline, as in
 serving).  The L2 cache is flushed before every timed step (a 256 MB write, then a 256 MB read
 of another buffer, so that L2 holds neither the step's inputs nor dirty lines whose write-back
 would land in the step); each step is timed with CUDA events on the launching stream and the
@@ -208,6 +208,7 @@ class Workload:
                                  inv_perm=torch.empty(R, dtype=torch.int32, device=dev), T=T, k=k, E=E)
         self.ws_route = torch.empty(max(gsg.workspace_size(gsg.OP_ROUTE, E, 0, 0, T, k), 16), **u8)
         self.ws_quant = torch.empty(max(gsg.workspace_size(gsg.OP_QUANTIZE, 0, 0, K, T, k), 16), **u8)
+        self.ws_disp = torch.empty(max(gsg.workspace_size(gsg.OP_DISPATCH, E, 0, K, T, k), 16), **u8)
         self.qa = gsg.QuantizedActivations(codes=torch.empty(R, K // 2, **u8),
                                            scales=torch.empty(gsg.act_scales_bytes(R, K, 32), **u8),
                                            x_scale=torch.empty(1, dtype=torch.float32, device=dev), R=R, K=K,
@@ -222,8 +223,8 @@ class Workload:
     # one step of the hot path
     def step(self):
         c = self.cfg
-        gsg.moe_route_permute(self.ids, c.E, out=self.route, workspace=self.ws_route)
-        gsg.quantize_act_nvfp4(self.X, 32, self.route.inv_perm, c.top_k, out=self.qa, workspace=self.ws_quant)
+        gsg.moe_dispatch_nvfp4(self.ids, self.X, c.E, 32, out_route=self.route, out_act=self.qa,
+                               workspace=self.ws_disp)
         gsg.grouped_sparse_gemm(self.qa, self.pw, self.route.offsets, self.max_rows, out=self.Y)
         gsg.unpermute_scale(self.Y, self.route.inv_perm, self.gates, c.top_k, out=self.out)
 
@@ -232,8 +233,8 @@ class Workload:
         c = self.cfg
         if getattr(self, "ws_comb", None) is None:
             self.ws_comb = gsg.combine_workspace(c.E, c.N, c.K, c.T, c.top_k, self.dev)
-        gsg.moe_route_permute(self.ids, c.E, out=self.route, workspace=self.ws_route)
-        gsg.quantize_act_nvfp4(self.X, 32, self.route.inv_perm, c.top_k, out=self.qa, workspace=self.ws_quant)
+        gsg.moe_dispatch_nvfp4(self.ids, self.X, c.E, 32, out_route=self.route, out_act=self.qa,
+                               workspace=self.ws_disp)
         gsg.grouped_sparse_gemm_combine(self.qa, self.pw, self.route, self.gates, self.ws_comb, self.max_rows,
                                         out=self.out)
 
@@ -242,7 +243,7 @@ class Workload:
         rows, histogram + scatter while ceil(R/1024)*E <= 16384, else histogram + scan + scatter)."""
         R, E = self.cfg.R, self.cfg.E
         route = 1 if R <= 2048 else (2 if -(-R // 1024) * E <= 16384 else 3)
-        return route + 2 + 1 + 1        # route, amax + quantize, GEMM, scatter
+        return route + 1 + 1 + 1        # routing (the amax pass in its first launch), quantize, GEMM, scatter
 
     def gemm(self):
         gsg.grouped_sparse_gemm(self.qa, self.pw, self.route.offsets, self.max_rows, out=self.Y)
@@ -378,9 +379,8 @@ class E2EPipeline:
         s.wait_event(self.uploaded[b])
         if not first:
             s.wait_event(self.downloaded[b])                  # step i-2's result has left out[b]
-        gsg.moe_route_permute(self.ids[b], c.E, out=wl.route, workspace=wl.ws_route, stream=s)
-        gsg.quantize_act_nvfp4(self.X[b], 32, wl.route.inv_perm, c.top_k, out=wl.qa, workspace=wl.ws_quant,
-                               stream=s)
+        gsg.moe_dispatch_nvfp4(self.ids[b], self.X[b], c.E, 32, out_route=wl.route, out_act=wl.qa,
+                               workspace=wl.ws_disp, stream=s)
         gsg.grouped_sparse_gemm(wl.qa, self.pw[i % self.NW], wl.route.offsets, wl.max_rows, out=wl.Y, stream=s)
         gsg.unpermute_scale(wl.Y, wl.route.inv_perm, self.gates[b], c.top_k, out=self.out[b], stream=s)
         self.computed[b].record(s)
@@ -612,7 +612,7 @@ def run_ours(args, world, rank, local):
         serial_ms = max_over_ranks(timed_ms(e2e_step, max(10, args.steps // 10), flush, world)[0], world, dev)
         e2e = {"value": job_value(flops, world, e2e_ms), "unit": "TFLOP/s", "ms_per_step": e2e_ms,
                "h2d_bytes_per_step": int(pipe.h2d_bytes()), "d2h_bytes_per_step": int(pipe.d2h_bytes()),
-               "path": "per step: pinned host -> device copies (upload stream), 4 library calls via the Python "
+               "path": "per step: pinned host -> device copies (upload stream), 3 library calls via the Python "
                        "binding (compute stream), result -> pinned host (download stream); double-buffered so "
                        "uploads and downloads overlap neighbouring steps' compute; weights rotate over 3 "
                        "replicas, no L2 flush",
@@ -786,6 +786,7 @@ class LayerWorkload:
                                  inv_perm=torch.empty(R, dtype=torch.int32, device=dev), T=T, k=k, E=E)
         self.ws_route = torch.empty(max(gsg.workspace_size(gsg.OP_ROUTE, E, 0, 0, T, k), 16), **u8)
         self.ws_quant = torch.empty(max(gsg.workspace_size(gsg.OP_QUANTIZE, 0, 0, H, T, k), 16), **u8)
+        self.ws_disp = torch.empty(max(gsg.workspace_size(gsg.OP_DISPATCH, E, 0, H, T, k), 16), **u8)
         self.qa = gsg.QuantizedActivations(codes=torch.empty(R, H // 2, **u8),
                                            scales=torch.empty(gsg.act_scales_bytes(R, H, 32), **u8),
                                            x_scale=torch.empty(1, dtype=torch.float32, device=dev), R=R, K=H,
@@ -808,8 +809,8 @@ class LayerWorkload:
 
     def step(self):
         L = self.L
-        gsg.moe_route_permute(self.ids, L.E, out=self.route, workspace=self.ws_route)
-        gsg.quantize_act_nvfp4(self.X, 32, self.route.inv_perm, L.top_k, out=self.qa, workspace=self.ws_quant)
+        gsg.moe_dispatch_nvfp4(self.ids, self.X, L.E, 32, out_route=self.route, out_act=self.qa,
+                               workspace=self.ws_disp)
         gsg.grouped_sparse_gemm_swiglu(self.qa, self.wu, self.route.offsets, self.h_scale, self.max_rows,
                                        out=self.hq)
         gsg.grouped_sparse_gemm(self.hq, self.wd, self.route.offsets, self.max_rows, out=self.Y2)

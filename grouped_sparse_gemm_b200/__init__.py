@@ -24,15 +24,15 @@ __all__ = [
     "GsgError", "lib", "load_library", "library_path",
     "PackedSparseWeights", "PackedDenseWeights", "Routing", "QuantizedActivations",
     "pack_sparse_nvfp4", "pack_dense_nvfp4", "moe_route_permute", "moe_route_permute_noalloc",
-    "quantize_act_nvfp4",
+    "quantize_act_nvfp4", "moe_dispatch_nvfp4",
     "grouped_sparse_gemm", "grouped_sparse_gemm_swiglu", "grouped_sparse_gemm_combine", "combine_workspace",
-    "grouped_dense_gemm", "unpermute_scale", "OP_COMBINE",
+    "grouped_dense_gemm", "unpermute_scale", "OP_COMBINE", "OP_DISPATCH",
     "get_device_status",
     "act_scales_bytes", "workspace_size", "OP_PACK_SPARSE", "OP_PACK_DENSE", "OP_ROUTE",
     "OP_QUANTIZE", "OP_GEMM", "EXPORTED_SYMBOLS",
 ]
 
-OP_PACK_SPARSE, OP_PACK_DENSE, OP_ROUTE, OP_QUANTIZE, OP_GEMM, OP_COMBINE = 1, 2, 3, 4, 5, 6
+OP_PACK_SPARSE, OP_PACK_DENSE, OP_ROUTE, OP_QUANTIZE, OP_GEMM, OP_COMBINE, OP_DISPATCH = 1, 2, 3, 4, 5, 6, 7
 OUT_BF16, OUT_F32 = 0, 1
 ACT_SCALE_PAD_ROWS = 256
 
@@ -43,6 +43,7 @@ EXPORTED_SYMBOLS = [
     "gsg_quantize_act_nvfp4", "gsg_grouped_sparse_gemm", "gsg_grouped_dense_gemm",
     "gsg_unpermute_scale", "gsg_get_device_status", "gsg_status_string", "gsg_version",
     "gsg_moe_route_permute_noalloc", "gsg_grouped_sparse_gemm_swiglu", "gsg_grouped_sparse_gemm_combine",
+    "gsg_moe_dispatch_nvfp4",
 ]
 
 _STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported shape", -3: "CUDA error",
@@ -84,6 +85,7 @@ def load_library(build_if_missing: bool = False) -> ctypes.CDLL:
         "gsg_pack_dense_nvfp4": (i, [vp, i, i, i, vp, fp, vp, sz, vp]),
         "gsg_moe_route_permute": (i, [vp, i, i, i, vp, vp, vp, vp, sz, vp]),
         "gsg_quantize_act_nvfp4": (i, [vp, i, i, i, vp, i, vp, vp, vp, vp, vp, sz, vp]),
+        "gsg_moe_dispatch_nvfp4": (i, [vp, vp, i, i, i, i, i, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "gsg_grouped_sparse_gemm": (i, [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, i, vp]),
         "gsg_grouped_dense_gemm": (i, [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, i, vp]),
         "gsg_unpermute_scale": (i, [vp, vp, vp, i, i, i, vp, vp]),
@@ -251,8 +253,10 @@ def moe_route_permute(topk_ids: torch.Tensor, E: int, out: Optional[Routing] = N
         out = Routing(offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
                       perm_src=torch.empty(max(T * k, 1), dtype=torch.int32, device=dev),
                       inv_perm=torch.empty(max(T * k, 1), dtype=torch.int32, device=dev), T=T, k=k, E=E)
-    need = workspace_size(OP_ROUTE, E, 0, 0, T, k)
-    ws = workspace if workspace is not None else (_workspace(need, dev) if need else None)
+    ws = workspace
+    if ws is None:   # the size query only when the call has to allocate
+        need = workspace_size(OP_ROUTE, E, 0, 0, T, k)
+        ws = _workspace(need, dev) if need else None
     _check("gsg_moe_route_permute", lib().gsg_moe_route_permute(
         _ptr(topk_ids), T, k, E, _ptr(out.offsets), _ptr(out.perm_src), _ptr(out.inv_perm),
         _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
@@ -286,12 +290,41 @@ def quantize_act_nvfp4(X: torch.Tensor, sf_block: int = 32, inv_perm: Optional[t
             codes=torch.empty(max(R, 1), K // 2, dtype=torch.uint8, device=dev),
             scales=torch.empty(act_scales_bytes(R, K, sf_block), dtype=torch.uint8, device=dev),
             x_scale=torch.empty(1, dtype=torch.float32, device=dev), R=R, K=K, sf_block=sf_block)
-    need = workspace_size(OP_QUANTIZE, 0, 0, K, T, top_k)
-    ws = workspace if workspace is not None else _workspace(need, dev)
+    ws = workspace if workspace is not None else _workspace(workspace_size(OP_QUANTIZE, 0, 0, K, T, top_k), dev)
     _check("gsg_quantize_act_nvfp4", lib().gsg_quantize_act_nvfp4(
         _ptr(X), T, K, sf_block, _ptr(inv_perm), top_k, _ptr(x_scale_in), _ptr(out.codes),
         _ptr(out.scales), _ptr(out.x_scale), _ptr(ws), ws.numel(), _stream(stream)))
     return out
+
+
+def moe_dispatch_nvfp4(topk_ids: torch.Tensor, X: torch.Tensor, E: int, sf_block: int = 32,
+                       x_scale_in: Optional[torch.Tensor] = None, out_route: Optional[Routing] = None,
+                       out_act: Optional[QuantizedActivations] = None, workspace: Optional[torch.Tensor] = None,
+                       stream=None):
+    """moe_route_permute + quantize_act_nvfp4 in one call (gsg_moe_dispatch_nvfp4): the same
+    outputs bit for bit, one launch fewer.  Returns (Routing, QuantizedActivations)."""
+    _need_cuda(topk_ids, X, x_scale_in)
+    assert topk_ids.dtype == torch.int32 and topk_ids.dim() == 2
+    assert X.dtype == torch.bfloat16 and X.dim() == 2 and X.shape[0] == topk_ids.shape[0]
+    T, k = topk_ids.shape
+    K = X.shape[1]
+    R = T * k
+    dev = X.device
+    if out_route is None:
+        out_route = Routing(offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+                            perm_src=torch.empty(max(R, 1), dtype=torch.int32, device=dev),
+                            inv_perm=torch.empty(max(R, 1), dtype=torch.int32, device=dev), T=T, k=k, E=E)
+    if out_act is None:
+        out_act = QuantizedActivations(
+            codes=torch.empty(max(R, 1), K // 2, dtype=torch.uint8, device=dev),
+            scales=torch.empty(act_scales_bytes(R, K, sf_block), dtype=torch.uint8, device=dev),
+            x_scale=torch.empty(1, dtype=torch.float32, device=dev), R=R, K=K, sf_block=sf_block)
+    ws = workspace if workspace is not None else _workspace(workspace_size(OP_DISPATCH, E, 0, K, T, k), dev)
+    _check("gsg_moe_dispatch_nvfp4", lib().gsg_moe_dispatch_nvfp4(
+        _ptr(topk_ids), _ptr(X), T, k, E, K, sf_block, _ptr(x_scale_in), _ptr(out_route.offsets),
+        _ptr(out_route.perm_src), _ptr(out_route.inv_perm), _ptr(out_act.codes), _ptr(out_act.scales),
+        _ptr(out_act.x_scale), _ptr(ws), ws.numel(), _stream(stream)))
+    return out_route, out_act
 
 
 def grouped_sparse_gemm(act: QuantizedActivations, w: PackedSparseWeights, offsets: torch.Tensor,

@@ -95,6 +95,10 @@ size_t gsg_workspace_size(int op, int E, int N, int K, int T, int k) {
     case GSG_OP_QUANTIZE:
       if (T < 0 || K < 1) return 0;
       return (size_t)gsg::quant_partials((long long)T * K) * sizeof(float);
+    case GSG_OP_DISPATCH:  // routing workspace (256-byte rounded), then the amax partials
+      if (E < 1 || T < 0 || k < 1 || K < 1) return 0;
+      return (gsg::route_workspace_bytes(T * k, E) + 255) / 256 * 256 +
+             (size_t)gsg::dispatch_amax_blocks((long long)T * K) * sizeof(float);
     case GSG_OP_COMBINE:   // slots bf16 [T*k][N], then counters int32 [T][N/32]
       if (T < 0 || k < 1 || N < 32) return 0;
       return combine_slot_bytes(T, k, N) + (size_t)T * (N / 32) * sizeof(int);
@@ -165,8 +169,40 @@ gsg_status_t gsg_quantize_act_nvfp4(const uint16_t* X, int T, int K, int sf_bloc
   gsg_status_t st = device_state(&d);
   if (st != GSG_OK) return st;
   return from_cuda(gsg::launch_quant(X, T, K, sf_block, inv_perm, k, x_tensor_scale_in, codes, scales,
-                                     x_tensor_scale_out, static_cast<float*>(workspace), d->status, d->num_sms,
+                                     x_tensor_scale_out, static_cast<float*>(workspace), 0, d->status, d->num_sms,
                                      as_stream(stream)));
+}
+
+gsg_status_t gsg_moe_dispatch_nvfp4(const int32_t* topk_ids, const uint16_t* X, int T, int k, int E, int K,
+                                    int sf_block, const float* x_tensor_scale_in, int32_t* expert_offsets,
+                                    int32_t* perm_src, int32_t* inv_perm, uint8_t* codes, uint8_t* scales,
+                                    float* x_tensor_scale_out, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+  // the checks of gsg_moe_route_permute and gsg_quantize_act_nvfp4
+  if (T < 0 || k < 1 || (sf_block != 16 && sf_block != 32)) return GSG_ERR_INVALID_ARG;
+  if (!gsg::route_supported(E)) return GSG_ERR_UNSUPPORTED_SHAPE;
+  if (K < 256 || K % 256 != 0) return GSG_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)T * k > (1ll << 30)) return GSG_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)T * (K / 8) >= (1ll << 31)) return GSG_ERR_UNSUPPORTED_SHAPE;
+  if (!expert_offsets || !scales || !x_tensor_scale_out) return GSG_ERR_INVALID_ARG;
+  if (T > 0 && (!topk_ids || !perm_src || !inv_perm || !X || !codes)) return GSG_ERR_INVALID_ARG;
+  if ((X && !aligned16(X)) || (codes && !aligned16(codes)) || !aligned16(scales)) return GSG_ERR_INVALID_ARG;
+  const size_t need = gsg_workspace_size(GSG_OP_DISPATCH, E, 0, K, T, k);
+  if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)) return GSG_ERR_WORKSPACE;
+  DeviceState* d = nullptr;
+  gsg_status_t st = device_state(&d);
+  if (st != GSG_OK) return st;
+  const size_t route_bytes = (gsg::route_workspace_bytes(T * k, E) + 255) / 256 * 256;
+  float* partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + route_bytes);
+  const bool amax = x_tensor_scale_in == nullptr;
+  int parts = 0;
+  cudaError_t e = gsg::launch_route_amax(topk_ids, T * k, E, expert_offsets, perm_src, inv_perm, workspace,
+                                         amax ? X : nullptr, amax ? (long long)T * K : 0, partial, &parts,
+                                         d->status, as_stream(stream));
+  if (e == cudaSuccess)
+    e = gsg::launch_quant(X, T, K, sf_block, inv_perm, k, x_tensor_scale_in, codes, scales, x_tensor_scale_out,
+                          partial, parts, d->status, d->num_sms, as_stream(stream));
+  return from_cuda(e);
 }
 
 static gsg_status_t gemm_common(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, const float* x_scale,

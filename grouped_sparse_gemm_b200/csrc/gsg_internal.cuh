@@ -163,4 +163,45 @@ __device__ __forceinline__ float warp_max(float v) {
 
 __host__ __device__ inline int ceil_div_i(int a, int b) { return (a + b - 1) / b; }
 
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
+
+// Partial max|X| of bf16 X (n8 128-bit units) for block `blk` of `nblk` (grid-stride over the
+// units, four 128-bit loads in flight per thread and round), written to partial[blk]; a
+// non-finite element sets GSG_ERR_NONFINITE.  Block-wide: every thread calls it; red holds
+// blockDim.x / 32 floats of shared memory.
+__device__ __forceinline__ void block_amax_partial(const uint16_t* __restrict__ X, long long n8, int blk, int nblk,
+                                                   float* partial, float* red, int* status) {
+  float mx = 0.0f;
+  bool finite = true;
+  const uint4* X4 = reinterpret_cast<const uint4*>(X);
+  const long long stride = (long long)nblk * blockDim.x;
+  for (long long i0 = (long long)blk * blockDim.x + threadIdx.x; i0 < n8; i0 += 4 * stride) {
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const long long i = i0 + u * stride;
+      v[u] = i < n8 ? __ldg(X4 + i) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t lo = w[j] & 0xFFFFu, hi = w[j] >> 16;
+        finite &= ((lo & 0x7F80u) != 0x7F80u) && ((hi & 0x7F80u) != 0x7F80u);
+        mx = fmaxf(mx, fmaxf(fabsf(bf16_bits_to_f32(lo)), fabsf(bf16_bits_to_f32(hi))));
+      }
+    }
+  }
+  if (!finite) set_status(status, GSG_ERR_NONFINITE);
+  mx = warp_max(mx);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (int)(blockDim.x >> 5) ? red[threadIdx.x] : 0.0f;
+    v = warp_max(v);
+    if (threadIdx.x == 0) partial[blk] = v;
+  }
+}
+
 }  // namespace gsg

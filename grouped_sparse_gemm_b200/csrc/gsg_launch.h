@@ -19,9 +19,11 @@ cudaError_t launch_pack(bool sparse, const float* W, int E, int N, int K, uint8_
 
 // gsg_quant.cu
 int quant_partials(long long n_elems);
+// partials_ready > 0: partial[0, partials_ready) already hold the partial maxima of X (the
+// dispatch launch computed them), so no amax launch is made.
 cudaError_t launch_quant(const uint16_t* X, int T, int K, int sf, const int32_t* inv_perm, int k, const float* s_in,
-                         uint8_t* codes, uint8_t* scales, float* s_out, float* partial, int* status, int num_sms,
-                         cudaStream_t stream);
+                         uint8_t* codes, uint8_t* scales, float* s_out, float* partial, int partials_ready,
+                         int* status, int num_sms, cudaStream_t stream);
 
 // gsg_route.cu
 int route_chunks(int R, int E);
@@ -30,6 +32,13 @@ bool route_supported(int E);
 cudaError_t route_set_smem_attrs();
 cudaError_t launch_route(const int32_t* ids, int R, int E, int32_t* off, int32_t* perm_src, int32_t* inv_perm,
                          void* ws, int* status, cudaStream_t stream);
+// Routing with the activation quantizer's amax pass folded into its first launch: X bf16 of
+// n_elems elements (nullptr / 0: no amax blocks); *amax_parts = number of partial maxima written
+// to amax_partial (0 when none).
+int dispatch_amax_blocks(long long n_elems);
+cudaError_t launch_route_amax(const int32_t* ids, int R, int E, int32_t* off, int32_t* perm_src, int32_t* inv_perm,
+                              void* ws, const uint16_t* X, long long n_elems, float* amax_partial, int* amax_parts,
+                              int* status, cudaStream_t stream);
 
 // gsg_unpermute.cu
 cudaError_t launch_unpermute(const uint16_t* Y, const int32_t* inv_perm, const float* gates, int T, int k, int N,

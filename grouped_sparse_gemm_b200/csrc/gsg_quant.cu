@@ -22,45 +22,12 @@ namespace gsg {
 constexpr int kQuantThreads = 256;
 constexpr int kQuantMainThreads = 128;   // the quantize launch: more, smaller blocks balance the SMs
 
-__device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
-
 __global__ void __launch_bounds__(kQuantThreads)
 act_amax_kernel(const uint16_t* __restrict__ X, long long n8, float* __restrict__ partial, int* status) {
   __shared__ float red[kQuantThreads / 32];
   pdl_launch_dependents();
   pdl_wait();
-  float mx = 0.0f;
-  bool finite = true;
-  const uint4* X4 = reinterpret_cast<const uint4*>(X);
-  const long long stride = (long long)gridDim.x * blockDim.x;
-  // four independent 128-bit loads in flight per thread and round
-  for (long long i0 = (long long)blockIdx.x * blockDim.x + threadIdx.x; i0 < n8; i0 += 4 * stride) {
-    uint4 v[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const long long i = i0 + u * stride;
-      v[u] = i < n8 ? __ldg(X4 + i) : make_uint4(0u, 0u, 0u, 0u);
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        uint32_t lo = w[j] & 0xFFFFu, hi = w[j] >> 16;
-        finite &= ((lo & 0x7F80u) != 0x7F80u) && ((hi & 0x7F80u) != 0x7F80u);
-        mx = fmaxf(mx, fmaxf(fabsf(bf16_bits_to_f32(lo)), fabsf(bf16_bits_to_f32(hi))));
-      }
-    }
-  }
-  if (!finite) set_status(status, GSG_ERR_NONFINITE);
-  mx = warp_max(mx);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = mx;
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    float v = threadIdx.x < kQuantThreads / 32 ? red[threadIdx.x] : 0.0f;
-    v = warp_max(v);
-    if (threadIdx.x == 0) partial[blockIdx.x] = v;
-  }
+  block_amax_partial(X, n8, blockIdx.x, gridDim.x, partial, red, status);
 }
 
 struct QuantParams {
@@ -319,10 +286,10 @@ int quant_partials(long long n_elems) {
 
 cudaError_t launch_quant(const uint16_t* X, int T, int K, int sf, const int32_t* inv_perm, int k,
                          const float* s_in, uint8_t* codes, uint8_t* scales, float* s_out,
-                         float* partial, int* status, int num_sms, cudaStream_t stream) {
+                         float* partial, int partials_ready, int* status, int num_sms, cudaStream_t stream) {
   const long long n = (long long)T * K;
-  int P = quant_partials(n);
-  if (s_in == nullptr && n > 0) {
+  int P = partials_ready > 0 ? partials_ready : quant_partials(n);
+  if (s_in == nullptr && n > 0 && partials_ready <= 0) {
     cudaError_t err = launch_pdl(act_amax_kernel, P, kQuantThreads, 0, stream, X, n / 8, partial, status);
     if (err != cudaSuccess) return err;
   }

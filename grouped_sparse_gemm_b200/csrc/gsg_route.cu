@@ -24,6 +24,7 @@ constexpr int kRouteThreads = 1024;
 constexpr int kRouteMaxE = 1024;
 constexpr long long kSmallChunkMaxCells = 16384;   // chunks x experts of the 1024-index path
 constexpr int kSingleMaxR = 2048;                  // one block, up to 2 indices per thread
+constexpr int kDispatchMaxAmaxBlocks = 256;        // amax blocks added to the first routing launch
 
 int route_chunk_size(int R, int E) {
   return ((long long)(R + 1023) / 1024) * E <= kSmallChunkMaxCells ? 1024 : 8192;
@@ -134,15 +135,12 @@ __device__ __forceinline__ void warp_run(int c0, int c1, int& f0, int& f1) {
 }
 
 // One block holds everything (R <= 1024 * kPer, kPer indices per thread): histogram, scan,
-// scatter in one launch.
+// scatter in one launch.  hist: 32 x E ints of shared memory.
 template <int kPer>
-__global__ void __launch_bounds__(kRouteThreads)
-route_single_kernel(const int32_t* __restrict__ ids, int R, int E, int32_t* off, int32_t* perm_src,
-                    int32_t* inv_perm, int* status) {
-  extern __shared__ int hist[];  // [32][E]
+__device__ __forceinline__ void route_single_body(const int32_t* __restrict__ ids, int R, int E, int32_t* off,
+                                                  int32_t* perm_src, int32_t* inv_perm, int* status, int* hist) {
   __shared__ int warp_sums[32];
   __shared__ int total;
-  pdl_launch_dependents();
   for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) hist[i] = 0;
   const int warp = threadIdx.x >> 5;
   int f0, f1;
@@ -173,15 +171,22 @@ route_single_kernel(const int32_t* __restrict__ ids, int R, int E, int32_t* off,
   warp_scatter<kPer>(x, m, f0, f1, hist + warp * E, perm_src, inv_perm);
 }
 
-// Multi-chunk path, launch 1: per-chunk histograms -> ws_hist[chunk][E].
 template <int kPer>
 __global__ void __launch_bounds__(kRouteThreads)
-route_hist_kernel(const int32_t* __restrict__ ids, int R, int E, int* ws_hist, int* status) {
-  extern __shared__ int hist[];
+route_single_kernel(const int32_t* __restrict__ ids, int R, int E, int32_t* off, int32_t* perm_src,
+                    int32_t* inv_perm, int* status) {
+  extern __shared__ int hist[];  // [32][E]
   pdl_launch_dependents();
+  route_single_body<kPer>(ids, R, E, off, perm_src, inv_perm, status, hist);
+}
+
+// Multi-chunk path, launch 1: the histogram of chunk `chunk` -> ws_hist[chunk][E].
+template <int kPer>
+__device__ __forceinline__ void route_hist_body(const int32_t* __restrict__ ids, int R, int E, int chunk,
+                                                int* ws_hist, int* status, int* hist) {
   for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) hist[i] = 0;
   pdl_wait();
-  const int c0 = blockIdx.x * 1024 * kPer, c1 = min(c0 + 1024 * kPer, R);
+  const int c0 = chunk * 1024 * kPer, c1 = min(c0 + 1024 * kPer, R);
   int f0, f1;
   warp_run<kPer>(c0, c1, f0, f1);
   int x[kPer];
@@ -193,8 +198,38 @@ route_hist_kernel(const int32_t* __restrict__ ids, int R, int E, int* ws_hist, i
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     int s = 0;
     for (int w = 0; w < 32; ++w) s += hist[w * E + e];
-    ws_hist[(size_t)blockIdx.x * E + e] = s;
+    ws_hist[(size_t)chunk * E + e] = s;
   }
+}
+
+template <int kPer>
+__global__ void __launch_bounds__(kRouteThreads)
+route_hist_kernel(const int32_t* __restrict__ ids, int R, int E, int* ws_hist, int* status) {
+  extern __shared__ int hist[];
+  pdl_launch_dependents();
+  route_hist_body<kPer>(ids, R, E, blockIdx.x, ws_hist, status, hist);
+}
+
+// The routing launch above (one-block routing when kSingle, else the chunk histograms) in
+// blocks [0, nroute), and the activation quantizer's partial max|X| in blocks [nroute, grid):
+// both only read their inputs, so the amax pass needs no launch of its own.
+template <int kPer, bool kSingle>
+__global__ void __launch_bounds__(kRouteThreads)
+route_amax_kernel(const int32_t* __restrict__ ids, int R, int E, int nroute, int32_t* off, int32_t* perm_src,
+                  int32_t* inv_perm, int* ws_hist, const uint16_t* __restrict__ X, long long n8, float* partial,
+                  int* status) {
+  extern __shared__ int hist[];
+  __shared__ float red[kRouteThreads / 32];
+  pdl_launch_dependents();
+  if ((int)blockIdx.x >= nroute) {
+    pdl_wait();
+    block_amax_partial(X, n8, (int)blockIdx.x - nroute, (int)gridDim.x - nroute, partial, red, status);
+    return;
+  }
+  if constexpr (kSingle)
+    route_single_body<kPer>(ids, R, E, off, perm_src, inv_perm, status, hist);
+  else
+    route_hist_body<kPer>(ids, R, E, blockIdx.x, ws_hist, status, hist);
 }
 
 // Launch 2 (one block): offsets and each chunk's first row per expert -> ws_base[chunk][E].
@@ -289,9 +324,13 @@ bool route_supported(int E) { return E >= 1 && E <= kRouteMaxE; }
 
 cudaError_t route_set_smem_attrs() {
   const int bytes = 32 * kRouteMaxE * (int)sizeof(int);
-  const cudaError_t errs[6] = {
+  const cudaError_t errs[10] = {
       cudaFuncSetAttribute(route_single_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
       cudaFuncSetAttribute(route_single_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
+      cudaFuncSetAttribute(route_amax_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
+      cudaFuncSetAttribute(route_amax_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
+      cudaFuncSetAttribute(route_amax_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
+      cudaFuncSetAttribute(route_amax_kernel<8, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
       cudaFuncSetAttribute(route_hist_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
       cudaFuncSetAttribute(route_hist_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
       cudaFuncSetAttribute(route_scatter_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
@@ -301,24 +340,47 @@ cudaError_t route_set_smem_attrs() {
   return cudaSuccess;
 }
 
-cudaError_t launch_route(const int32_t* ids, int R, int E, int32_t* off, int32_t* perm_src,
-                         int32_t* inv_perm, void* ws, int* status, cudaStream_t stream) {
+int dispatch_amax_blocks(long long n_elems) {
+  const long long n8 = n_elems / 8;
+  long long b = (n8 + 4LL * kRouteThreads - 1) / (4LL * kRouteThreads);   // 4 units per thread
+  if (b < 1) b = 1;
+  if (b > kDispatchMaxAmaxBlocks) b = kDispatchMaxAmaxBlocks;
+  return int(b);
+}
+
+// The routing launches; with X != nullptr and n_elems > 0 the first one also computes the amax
+// partials of X in P extra blocks (*amax_parts = P).
+static cudaError_t route_launches(const int32_t* ids, int R, int E, int32_t* off, int32_t* perm_src,
+                                  int32_t* inv_perm, void* ws, const uint16_t* X, long long n_elems,
+                                  float* amax_partial, int* amax_parts, int* status, cudaStream_t stream) {
   const size_t smem = (size_t)32 * E * sizeof(int);
   const int nc = route_chunks(R, E);
+  const int P = (X != nullptr && n_elems > 0) ? dispatch_amax_blocks(n_elems) : 0;
+  if (amax_parts != nullptr) *amax_parts = P;
+  const long long n8 = n_elems / 8;
   if (nc <= 1) {
-    auto single = R <= 1024 ? route_single_kernel<1> : route_single_kernel<2>;
-    return launch_pdl(single, 1, kRouteThreads, smem, stream, ids, R, E, off, perm_src, inv_perm, status);
+    if (P == 0) {
+      auto single = R <= 1024 ? route_single_kernel<1> : route_single_kernel<2>;
+      return launch_pdl(single, 1, kRouteThreads, smem, stream, ids, R, E, off, perm_src, inv_perm, status);
+    }
+    auto single = R <= 1024 ? route_amax_kernel<1, true> : route_amax_kernel<2, true>;
+    return launch_pdl(single, 1 + P, kRouteThreads, smem, stream, ids, R, E, 1, off, perm_src, inv_perm,
+                      (int*)nullptr, X, n8, amax_partial, status);
   }
   int* ws_hist = static_cast<int*>(ws);
   int* ws_base = ws_hist + (size_t)nc * E;
   cudaError_t e;
   if (route_chunk_size(R, E) == 1024) {
-    e = launch_pdl(route_hist_kernel<1>, nc, kRouteThreads, smem, stream, ids, R, E, ws_hist, status);
+    e = P == 0 ? launch_pdl(route_hist_kernel<1>, nc, kRouteThreads, smem, stream, ids, R, E, ws_hist, status)
+               : launch_pdl(route_amax_kernel<1, false>, nc + P, kRouteThreads, smem, stream, ids, R, E, nc, off,
+                            perm_src, inv_perm, ws_hist, X, n8, amax_partial, status);
     if (e == cudaSuccess)
       e = launch_pdl(route_scatter_kernel<1, true>, nc, kRouteThreads, smem, stream, ids, R, E,
                      (const int*)ws_hist, nc, off, perm_src, inv_perm);
   } else {
-    e = launch_pdl(route_hist_kernel<8>, nc, kRouteThreads, smem, stream, ids, R, E, ws_hist, status);
+    e = P == 0 ? launch_pdl(route_hist_kernel<8>, nc, kRouteThreads, smem, stream, ids, R, E, ws_hist, status)
+               : launch_pdl(route_amax_kernel<8, false>, nc + P, kRouteThreads, smem, stream, ids, R, E, nc, off,
+                            perm_src, inv_perm, ws_hist, X, n8, amax_partial, status);
     if (e == cudaSuccess)
       e = launch_pdl(route_scan_kernel, 1, kRouteThreads, 0, stream, (const int*)ws_hist, nc, E, off, ws_base);
     if (e == cudaSuccess)
@@ -326,6 +388,18 @@ cudaError_t launch_route(const int32_t* ids, int R, int E, int32_t* off, int32_t
                      (const int*)ws_base, nc, off, perm_src, inv_perm);
   }
   return e;
+}
+
+cudaError_t launch_route(const int32_t* ids, int R, int E, int32_t* off, int32_t* perm_src,
+                         int32_t* inv_perm, void* ws, int* status, cudaStream_t stream) {
+  return route_launches(ids, R, E, off, perm_src, inv_perm, ws, nullptr, 0, nullptr, nullptr, status, stream);
+}
+
+cudaError_t launch_route_amax(const int32_t* ids, int R, int E, int32_t* off, int32_t* perm_src, int32_t* inv_perm,
+                              void* ws, const uint16_t* X, long long n_elems, float* amax_partial, int* amax_parts,
+                              int* status, cudaStream_t stream) {
+  return route_launches(ids, R, E, off, perm_src, inv_perm, ws, X, n_elems, amax_partial, amax_parts, status,
+                        stream);
 }
 
 }  // namespace gsg

@@ -69,7 +69,8 @@ enum {
   GSG_OP_ROUTE = 3,
   GSG_OP_QUANTIZE = 4,
   GSG_OP_GEMM = 5,
-  GSG_OP_COMBINE = 6    /* gsg_grouped_sparse_gemm_combine: token slots + completion counters */
+  GSG_OP_COMBINE = 6,   /* gsg_grouped_sparse_gemm_combine: token slots + completion counters */
+  GSG_OP_DISPATCH = 7   /* gsg_moe_dispatch_nvfp4: routing workspace + amax partials          */
 };
 
 /* Output element types of the grouped GEMMs. */
@@ -132,6 +133,23 @@ gsg_status_t gsg_moe_route_permute(const int32_t* topk_ids, int T, int k, int E,
 gsg_status_t gsg_quantize_act_nvfp4(const uint16_t* X, int T, int K, int sf_block,
                                     const int32_t* inv_perm, int k,
                                     const float* x_tensor_scale_in,
+                                    uint8_t* codes, uint8_t* scales, float* x_tensor_scale_out,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* ----------------------------------------------------------------------------------------
+ * gsg_moe_dispatch_nvfp4 -- routing and the activation quantizer in one call.
+ * Paper: §D.1 (p.19): dispatch fused with activation quantization ahead of the first expert
+ * GEMM; §2 "Execution gap" (p.3): grouped expert problems.
+ * Computes exactly what gsg_moe_route_permute(topk_ids, T, k, E, ...) followed by
+ * gsg_quantize_act_nvfp4(X, T, K, sf_block, inv_perm, k, x_tensor_scale_in, ...) compute, bit
+ * for bit, with the same arguments, outputs, limits and errors as the two.  The difference is
+ * the launches: the quantizer's max|X| pass runs inside the routing's first launch (extra
+ * blocks beside the routing blocks; both only read their inputs), so the pair takes one launch
+ * fewer.  workspace: gsg_workspace_size(GSG_OP_DISPATCH, E, 0, K, T, k) bytes, 16-byte aligned.
+ */
+gsg_status_t gsg_moe_dispatch_nvfp4(const int32_t* topk_ids, const uint16_t* X, int T, int k, int E, int K,
+                                    int sf_block, const float* x_tensor_scale_in,
+                                    int32_t* expert_offsets, int32_t* perm_src, int32_t* inv_perm,
                                     uint8_t* codes, uint8_t* scales, float* x_tensor_scale_out,
                                     void* workspace, size_t workspace_bytes, void* stream);
 

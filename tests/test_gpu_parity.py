@@ -129,6 +129,45 @@ def test_quantize_many_routed_rows(gsg, T, k, E, K, sf):
     _status_ok(gsg)
 
 
+# ---------------------------------------------------------------- routing + quantizer in one call
+@pytest.mark.parametrize("name,T,k,E,K,sf,given_scale", [
+    ("tiny", 0, 0, 0, 0, 32, False),
+    ("30b_up_prefill", 0, 0, 0, 0, 32, False),        # R = 4096: 1024-row chunks
+    ("30b_down_decode", 0, 0, 0, 0, 32, False),       # R = 512: one routing block
+    ("1t_down_decode_b1", 0, 0, 0, 0, 32, False),
+    ("tiny", 0, 0, 0, 0, 16, False),                  # dense control's 16-element blocks
+    ("tiny", 0, 0, 0, 0, 32, True),                   # caller-supplied tensor scale: no amax blocks
+    ("custom", 9000, 8, 512, 256, 32, False),         # R = 72000: 8192-row chunks, scan launch
+    ("custom", 300, 7, 64, 512, 32, False),           # R = 2100: just past one block
+    ("custom", 0, 8, 16, 256, 32, False),             # no tokens
+])
+def test_dispatch_matches_separate_calls_and_oracle(gsg, name, T, k, E, K, sf, given_scale):
+    cfg = inputs.CONFIGS[name] if name != "custom" else inputs.custom_config("dp", E=E, K=K, N=128, T=T, top_k=k)
+    X = inputs.activations(cfg).to(DEV)
+    ids = inputs.routing(cfg) if cfg.T > 0 else torch.zeros(0, cfg.top_k, dtype=torch.int32)
+    ids_d = ids.to(DEV)
+    s_in = torch.tensor([0.0625], dtype=torch.float32, device=DEV) if given_scale else None
+    r, qa = gsg.moe_dispatch_nvfp4(ids_d, X, cfg.E, sf_block=sf, x_scale_in=s_in)
+    r2 = gsg.moe_route_permute(ids_d, cfg.E)
+    qa2 = gsg.quantize_act_nvfp4(X, sf, r2.inv_perm, cfg.top_k, x_scale_in=s_in)
+    _status_ok(gsg)
+    R = cfg.T * cfg.top_k
+    for a_, b_ in ((r.offsets, r2.offsets), (r.perm_src[:R], r2.perm_src[:R]), (r.inv_perm[:R], r2.inv_perm[:R]),
+                   (qa.codes[:R], qa2.codes[:R]), (qa.scales, qa2.scales), (qa.x_scale, qa2.x_scale)):
+        assert torch.equal(a_, b_)
+    if given_scale:
+        assert qa.x_scale.item() == 0.0625
+    if R > 0 and R <= 8192:   # the oracle, on the sizes it finishes in seconds
+        off, ps, ip = tl.route_np(ids, cfg.E)
+        np.testing.assert_array_equal(r.offsets.cpu().numpy(), off)
+        np.testing.assert_array_equal(r.perm_src.cpu().numpy()[:R], ps)
+        if not given_scale:
+            codes, quad, s, _, _ = tl.oracle_act(X.float().cpu().numpy(), sf, ps, cfg.top_k)
+            assert qa.x_scale.item() == s
+            np.testing.assert_array_equal(qa.codes.cpu().numpy()[:R], codes)
+            np.testing.assert_array_equal(qa.scales.cpu().numpy(), quad)
+
+
 def _rounding_rows():
     """bf16 rows whose 32-element blocks put values exactly on E2M1 rounding midpoints and block
     maxima exactly on UE4M3 midpoints, subnormals and the saturation limit (with s_x = 1)."""
