@@ -977,6 +977,29 @@ def run_profile_steps(args, local):
         raise RuntimeError(f"device status {st}")
 
 
+def run_profile_quantize(args, local):
+    """Routing + activation quantization (gsg_moe_dispatch_nvfp4) at a configuration's activation
+    shape, warmup + steps times, with nothing else on the device (no weights): a small process
+    for profiler captures of the quantizer's kernels."""
+    dev = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(dev)
+    gsg.load_library()
+    cfg = inputs.CONFIGS[args.config]
+    X = inputs.activations(cfg).to(dev)
+    ids = inputs.routing(cfg).to(dev)
+    ws = torch.empty(max(gsg.workspace_size(gsg.OP_DISPATCH, cfg.E, 0, cfg.K, cfg.T, cfg.top_k), 16),
+                     dtype=torch.uint8, device=dev)
+    r, qa = gsg.moe_dispatch_nvfp4(ids, X, cfg.E, 32, workspace=ws)
+    for _ in range(args.warmup + args.steps):
+        gsg.moe_dispatch_nvfp4(ids, X, cfg.E, 32, out_route=r, out_act=qa, workspace=ws)
+    torch.cuda.synchronize()
+    st = gsg.get_device_status()
+    print(json.dumps({"profile_quantize": 1 + args.warmup + args.steps, "config": cfg.name, "status": st}),
+          flush=True)
+    if st != 0:
+        raise RuntimeError(f"device status {st}")
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -999,6 +1022,8 @@ def main():
     ap.add_argument("--sweep-n", default="1,8,32,128,512")
     ap.add_argument("--profile-steps", action="store_true",
                     help="for profiler launch lists: only replay the step graph (warmup + steps), print no bench line")
+    ap.add_argument("--profile-quantize", action="store_true",
+                    help="for profiler captures: only routing + quantization at --config's activation shape")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -1008,6 +1033,8 @@ def main():
             run_reference(args, world, rank)
         elif args.profile_steps:
             run_profile_steps(args, local)
+        elif args.profile_quantize:
+            run_profile_quantize(args, local)
         elif args.sweep:
             run_sweep(args, local)
         elif args.layer:

@@ -92,13 +92,17 @@ size_t gsg_workspace_size(int op, int E, int N, int K, int T, int k) {
     case GSG_OP_ROUTE:
       if (E < 1 || T < 0 || k < 1) return 0;
       return gsg::route_workspace_bytes(T * k, E);
-    case GSG_OP_QUANTIZE:
-      if (T < 0 || K < 1) return 0;
-      return (size_t)gsg::quant_partials((long long)T * K) * sizeof(float);
-    case GSG_OP_DISPATCH:  // routing workspace (256-byte rounded), then the amax partials
+    case GSG_OP_QUANTIZE: {  // amax partials, then (large R*K) the raw scale words
+      if (T < 0 || K < 1 || k < 1) return 0;
+      const size_t raw = gsg::quant_raw_bytes((long long)T * k, K);
+      return raw > 0 ? gsg::quant_raw_offset((long long)T * K) + raw
+                     : (size_t)gsg::quant_partials((long long)T * K) * sizeof(float);
+    }
+    case GSG_OP_DISPATCH:  // routing workspace, amax partials (each 256-byte rounded), raw scale words
       if (E < 1 || T < 0 || k < 1 || K < 1) return 0;
       return (gsg::route_workspace_bytes(T * k, E) + 255) / 256 * 256 +
-             (size_t)gsg::dispatch_amax_blocks((long long)T * K) * sizeof(float);
+             ((size_t)gsg::dispatch_amax_blocks((long long)T * K) * sizeof(float) + 255) / 256 * 256 +
+             gsg::quant_raw_bytes((long long)T * k, K);
     case GSG_OP_COMBINE:   // slots bf16 [T*k][N], then counters int32 [T][N/32]
       if (T < 0 || k < 1 || N < 32) return 0;
       return combine_slot_bytes(T, k, N) + (size_t)T * (N / 32) * sizeof(int);
@@ -161,16 +165,20 @@ gsg_status_t gsg_quantize_act_nvfp4(const uint16_t* X, int T, int K, int sf_bloc
   if (!scales || !x_tensor_scale_out) return GSG_ERR_INVALID_ARG;
   if (T > 0 && (!X || !codes)) return GSG_ERR_INVALID_ARG;
   if ((X && !aligned16(X)) || (codes && !aligned16(codes)) || !aligned16(scales)) return GSG_ERR_INVALID_ARG;
-  if (x_tensor_scale_in == nullptr) {
+  const size_t raw_bytes = sf_block == 32 ? gsg::quant_raw_bytes((long long)T * k, K) : 0;
+  if (x_tensor_scale_in == nullptr || raw_bytes > 0) {
     const size_t need = gsg_workspace_size(GSG_OP_QUANTIZE, 0, 0, K, T, k);
-    if (workspace == nullptr || workspace_bytes < need) return GSG_ERR_WORKSPACE;
+    if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)) return GSG_ERR_WORKSPACE;
   }
   DeviceState* d = nullptr;
   gsg_status_t st = device_state(&d);
   if (st != GSG_OK) return st;
+  uint32_t* raw = raw_bytes > 0 ? reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) +
+                                                              gsg::quant_raw_offset((long long)T * K))
+                                : nullptr;
   return from_cuda(gsg::launch_quant(X, T, K, sf_block, inv_perm, k, x_tensor_scale_in, codes, scales,
-                                     x_tensor_scale_out, static_cast<float*>(workspace), 0, d->status, d->num_sms,
-                                     as_stream(stream)));
+                                     x_tensor_scale_out, static_cast<float*>(workspace), 0, raw, d->status,
+                                     d->num_sms, as_stream(stream)));
 }
 
 gsg_status_t gsg_moe_dispatch_nvfp4(const int32_t* topk_ids, const uint16_t* X, int T, int k, int E, int K,
@@ -193,7 +201,11 @@ gsg_status_t gsg_moe_dispatch_nvfp4(const int32_t* topk_ids, const uint16_t* X, 
   gsg_status_t st = device_state(&d);
   if (st != GSG_OK) return st;
   const size_t route_bytes = (gsg::route_workspace_bytes(T * k, E) + 255) / 256 * 256;
+  const size_t part_bytes = ((size_t)gsg::dispatch_amax_blocks((long long)T * K) * sizeof(float) + 255) / 256 * 256;
   float* partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + route_bytes);
+  uint32_t* raw = (sf_block == 32 && gsg::quant_raw_bytes((long long)T * k, K) > 0)
+                      ? reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + route_bytes + part_bytes)
+                      : nullptr;
   const bool amax = x_tensor_scale_in == nullptr;
   int parts = 0;
   cudaError_t e = gsg::launch_route_amax(topk_ids, T * k, E, expert_offsets, perm_src, inv_perm, workspace,
@@ -201,7 +213,7 @@ gsg_status_t gsg_moe_dispatch_nvfp4(const int32_t* topk_ids, const uint16_t* X, 
                                          d->status, as_stream(stream));
   if (e == cudaSuccess)
     e = gsg::launch_quant(X, T, K, sf_block, inv_perm, k, x_tensor_scale_in, codes, scales, x_tensor_scale_out,
-                          partial, parts, d->status, d->num_sms, as_stream(stream));
+                          partial, parts, raw, d->status, d->num_sms, as_stream(stream));
   return from_cuda(e);
 }
 

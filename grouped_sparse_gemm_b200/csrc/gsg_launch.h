@@ -19,11 +19,16 @@ cudaError_t launch_pack(bool sparse, const float* W, int E, int N, int K, uint8_
 
 // gsg_quant.cu
 int quant_partials(long long n_elems);
+// Raw scale-word buffer of the two-phase scale path (0 when R*K is below its threshold) and its
+// offset in the quantizer's workspace (after the amax partials).
+size_t quant_raw_bytes(long long R, int K);
+size_t quant_raw_offset(long long n_elems);
 // partials_ready > 0: partial[0, partials_ready) already hold the partial maxima of X (the
 // dispatch launch computed them), so no amax launch is made.
+// raw: workspace of quant_raw_bytes(T*k, K) bytes for the two-phase scale path (nullptr: direct).
 cudaError_t launch_quant(const uint16_t* X, int T, int K, int sf, const int32_t* inv_perm, int k, const float* s_in,
                          uint8_t* codes, uint8_t* scales, float* s_out, float* partial, int partials_ready,
-                         int* status, int num_sms, cudaStream_t stream);
+                         uint32_t* raw, int* status, int num_sms, cudaStream_t stream);
 
 // gsg_route.cu
 int route_chunks(int R, int E);

@@ -16,11 +16,17 @@
 // rows read once per warp (lane j holds row j) and the scale words spread over the lanes.  The same launch zero-fills
 // the padding entries of the quad scale layout.
 #include "gsg_internal.cuh"
+#include "gsg_launch.h"
 
 namespace gsg {
 
 constexpr int kQuantThreads = 256;
 constexpr int kQuantMainThreads = 128;   // the quantize launch: more, smaller blocks balance the SMs
+// From R*K = 2^27 (R routed rows) the 32-element quantizer writes its scale words row-major to a
+// workspace and a second launch builds the quad layout: writing the quad entries directly is
+// four scattered 4-byte stores per routed row and k-block, each its own 32-byte sector, and at
+// these sizes the partial sectors leave L2 before they fill (DRAM read-modify-write).
+constexpr long long kQuantRawMinRK = 1ll << 27;
 
 __global__ void __launch_bounds__(kQuantThreads)
 act_amax_kernel(const uint16_t* __restrict__ X, long long n8, float* __restrict__ partial, int* status) {
@@ -41,6 +47,7 @@ struct QuantParams {
   uint8_t* scales;
   float* s_out;
   int* status;
+  uint32_t* raw;   // non-null: scale words go to raw[row][K/128] (then act_scales_quad_kernel)
 };
 
 // The tensor scale: the caller's value, or max|X| folded from the partial maxima (block-wide;
@@ -161,6 +168,10 @@ act_quant32_kernel(QuantParams p) {
       if (row < 0 || row >= p.R) { set_status(p.status, GSG_ERR_BAD_ROUTING); return; }
       *reinterpret_cast<uint4*>(p.codes + (size_t)row * (p.K / 2) + (size_t)q.b * 16) =
           make_uint4(cw[0], cw[1], cw[2], cw[3]);
+      if (p.raw != nullptr) {   // one word per row and k-block (K % 1024 == 0: a warp's 32 contiguous bytes)
+        if (cq == 0) p.raw[(size_t)row * (p.K / 128) + kb] = word;
+        return;
+      }
       const int rr = row - 32 * cq;
       if (rr >= 0) sw[((size_t)kb * p.rcap + rr) * 4 + cq] = word;
     };
@@ -169,7 +180,36 @@ act_quant32_kernel(QuantParams p) {
       if (j < p.k) dispatch(q.rows[j]);
     for (int j = kQ32Rows; j < p.k; ++j) dispatch(__ldg(p.inv_perm + (size_t)q.t * p.k + j));
   }
-  quant_zero_padding(p);
+  if (p.raw == nullptr) quant_zero_padding(p);
+}
+
+// Second launch of the two-phase path: raw scale words [R][KBa] -> the quad layout,
+//   quad[kb][rr][c] = raw[rr + 32c][kb]  (0 where rr + 32c >= R),  rr in [0, rcap).
+// A block builds 128 quad rows x 16 k-blocks from 224 raw rows staged in shared memory (row
+// pitch 17 words: conflict-free column reads); reads are 64-byte row segments, writes 16-byte
+// entries, 2 KB contiguous per k-block.  The padding entries are written too.
+constexpr int kQuadTileRows = 128;
+constexpr int kQuadTileKb = 16;
+
+__global__ void __launch_bounds__(256)
+act_scales_quad_kernel(const uint32_t* __restrict__ raw, int R, int KBa, int rcap, uint32_t* __restrict__ quad) {
+  __shared__ uint32_t tile[kQuadTileRows + 96][kQuadTileKb + 1];
+  pdl_launch_dependents();
+  pdl_wait();
+  const int r0 = blockIdx.x * kQuadTileRows, kb0 = blockIdx.y * kQuadTileKb;
+  for (int i = threadIdx.x; i < (kQuadTileRows + 96) * kQuadTileKb; i += blockDim.x) {
+    const int rr = i / kQuadTileKb, kk = i % kQuadTileKb;
+    const int row = r0 + rr, kb = kb0 + kk;
+    tile[rr][kk] = (row < R && kb < KBa) ? __ldg(raw + (size_t)row * KBa + kb) : 0u;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < kQuadTileRows * kQuadTileKb; i += blockDim.x) {
+    const int kk = i / kQuadTileRows, rr = i % kQuadTileRows;
+    const int row = r0 + rr, kb = kb0 + kk;
+    if (row >= rcap || kb >= KBa) continue;
+    *reinterpret_cast<uint4*>(quad + ((size_t)kb * rcap + row) * 4) =
+        make_uint4(tile[rr][kk], tile[rr + 32][kk], tile[rr + 64][kk], tile[rr + 96][kk]);
+  }
 }
 
 // One warp-iteration covers 256 consecutive elements of one token row (K % 256 == 0): lane L
@@ -276,6 +316,14 @@ act_quant_kernel(QuantParams p) {
   quant_zero_padding(p);
 }
 
+size_t quant_raw_offset(long long n_elems) {
+  return ((size_t)quant_partials(n_elems) * sizeof(float) + 255) / 256 * 256;
+}
+
+size_t quant_raw_bytes(long long R, int K) {
+  return R * (long long)K >= kQuantRawMinRK ? (size_t)(R * (long long)(K / 128) * 4) : 0;
+}
+
 int quant_partials(long long n_elems) {
   long long n8 = n_elems / 8;
   long long b = (n8 + kQuantThreads * 4 - 1) / (kQuantThreads * 4);
@@ -286,7 +334,8 @@ int quant_partials(long long n_elems) {
 
 cudaError_t launch_quant(const uint16_t* X, int T, int K, int sf, const int32_t* inv_perm, int k,
                          const float* s_in, uint8_t* codes, uint8_t* scales, float* s_out,
-                         float* partial, int partials_ready, int* status, int num_sms, cudaStream_t stream) {
+                         float* partial, int partials_ready, uint32_t* raw, int* status, int num_sms,
+                         cudaStream_t stream) {
   const long long n = (long long)T * K;
   int P = partials_ready > 0 ? partials_ready : quant_partials(n);
   if (s_in == nullptr && n > 0 && partials_ready <= 0) {
@@ -298,12 +347,22 @@ cudaError_t launch_quant(const uint16_t* X, int T, int K, int sf, const int32_t*
   p.X = X; p.inv_perm = inv_perm; p.s_in = s_in; p.partial = partial; p.nparts = P;
   p.T = T; p.K = K; p.sf = sf; p.k = k; p.R = T * k; p.rcap = T * k + kActScalePadRows;
   p.codes = codes; p.scales = scales; p.s_out = s_out; p.status = status;
+  // two-phase scales (32-element blocks, large R*K, raw buffer given): see act_scales_quad_kernel
+  p.raw = (sf == 32 && raw != nullptr && quant_raw_bytes(p.R, K) > 0) ? raw : nullptr;
   const long long units = (long long)T * (K / (sf == 32 ? 32 : 8));   // lanes of work
-  const long long pad = (long long)(K / (4 * sf)) * (T * k + kActScalePadRows - (T * k > 96 ? T * k - 96 : 0)) * 4;
+  const long long pad = p.raw != nullptr ? 0
+      : (long long)(K / (4 * sf)) * (T * k + kActScalePadRows - (T * k > 96 ? T * k - 96 : 0)) * 4;
   long long blocks = ((units > pad ? units : pad) + kQuantMainThreads - 1) / kQuantMainThreads;
   if (blocks < 1) blocks = 1;
   if (blocks > (long long)num_sms * 16) blocks = (long long)num_sms * 16;
-  if (sf == 32) return launch_pdl(act_quant32_kernel, (unsigned)blocks, kQuantMainThreads, 0, stream, p);
+  if (sf == 32) {
+    cudaError_t e = launch_pdl(act_quant32_kernel, (unsigned)blocks, kQuantMainThreads, 0, stream, p);
+    if (e != cudaSuccess || p.raw == nullptr) return e;
+    const int KBa = K / 128;
+    const dim3 grid((unsigned)ceil_div_i(p.rcap, kQuadTileRows), (unsigned)ceil_div_i(KBa, kQuadTileKb));
+    return launch_pdl(act_scales_quad_kernel, grid, 256, 0, stream, (const uint32_t*)p.raw, p.R, KBa, p.rcap,
+                      reinterpret_cast<uint32_t*>(scales));
+  }
   return launch_pdl(act_quant_kernel, (unsigned)blocks, kQuantMainThreads, 0, stream, p);
 }
 

@@ -70,7 +70,7 @@ enum {
   GSG_OP_QUANTIZE = 4,
   GSG_OP_GEMM = 5,
   GSG_OP_COMBINE = 6,   /* gsg_grouped_sparse_gemm_combine: token slots + completion counters */
-  GSG_OP_DISPATCH = 7   /* gsg_moe_dispatch_nvfp4: routing workspace + amax partials          */
+  GSG_OP_DISPATCH = 7   /* gsg_moe_dispatch_nvfp4: routing workspace + quantizer workspace    */
 };
 
 /* Output element types of the grouped GEMMs. */
@@ -129,6 +129,11 @@ gsg_status_t gsg_moe_route_permute(const int32_t* topk_ids, int T, int k, int E,
  * (inv_perm NULL: row t, and k must be 1).  sf_block: 32 (sparse GEMM) or 16 (dense control).
  * Outputs: codes [R][K/2], scales in the quad layout above (R = T*k), x_tensor_scale_out fp32[1].
  * Limits: T*k <= 2^30 and T*K/8 < 2^31, else GSG_ERR_UNSUPPORTED_SHAPE.
+ * workspace: gsg_workspace_size(GSG_OP_QUANTIZE, 0, 0, K, T, k) bytes, 16-byte aligned, needed
+ * when s_x is computed (the partial maxima) and, for sf_block 32, once R*K >= 2^27: there the
+ * scale words are first written row-major to the workspace and a second launch rearranges
+ * them into the quad layout (scattered 4-byte quad writes cost DRAM read-modify-writes at
+ * that size).  The result is the same either way.  Otherwise it may be NULL.
  */
 gsg_status_t gsg_quantize_act_nvfp4(const uint16_t* X, int T, int K, int sf_block,
                                     const int32_t* inv_perm, int k,

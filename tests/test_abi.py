@@ -45,9 +45,14 @@ def test_sizes(L):
     assert L.gsg_workspace_size(gsg.OP_ROUTE, 128, 0, 0, 512, 8) == 2 * 4 * 128 * 4    # 1024-row chunks
     assert L.gsg_workspace_size(gsg.OP_ROUTE, 128, 0, 0, 2000, 8) == 2 * 16 * 128 * 4  # 1024-row chunks
     assert L.gsg_workspace_size(gsg.OP_GEMM, 384, 4096, 7168, 8192, 8) == 0
-    # routing workspace (4 chunks x 128 experts x 2 int32, 256-byte rounded) + one float per amax block
-    assert L.gsg_workspace_size(gsg.OP_DISPATCH, 128, 0, 2048, 512, 8) == 4096 + 32 * 4
-    assert L.gsg_workspace_size(gsg.OP_DISPATCH, 128, 0, 768, 64, 8) == 2 * 4      # one routing block
+    # routing workspace (4 chunks x 128 experts x 2 int32) + one float per amax block, each 256-byte rounded
+    assert L.gsg_workspace_size(gsg.OP_DISPATCH, 128, 0, 2048, 512, 8) == 4096 + 256
+    assert L.gsg_workspace_size(gsg.OP_DISPATCH, 128, 0, 768, 64, 8) == 256        # one routing block
+    # from R*K = 2^27 the quantizer stages its scale words row-major: R * K/128 words after the partials
+    raw = 65536 * (7168 // 128) * 4
+    assert L.gsg_workspace_size(gsg.OP_QUANTIZE, 0, 0, 7168, 8192, 8) == 512 * 4 + raw
+    assert L.gsg_workspace_size(gsg.OP_DISPATCH, 384, 0, 7168, 8192, 8) == 2 * 8 * 384 * 4 + 1024 + raw
+    assert L.gsg_workspace_size(gsg.OP_QUANTIZE, 0, 0, 2048, 512, 8) == 128 * 4     # partials only
 
 
 def test_status_strings(L):

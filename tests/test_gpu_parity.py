@@ -168,6 +168,27 @@ def test_dispatch_matches_separate_calls_and_oracle(gsg, name, T, k, E, K, sf, g
             np.testing.assert_array_equal(qa.scales.cpu().numpy(), quad)
 
 
+@pytest.mark.parametrize("T,k,K,given_scale", [(2048, 8, 8192, False), (2304, 8, 7424, True), (1100, 16, 7680, False)])
+def test_quantize_two_phase_scales(gsg, T, k, K, given_scale):
+    # R*K >= 2^27: scale words staged row-major in the workspace, then rearranged into the quad
+    # layout by a second launch (K = 7424: a warp's blocks straddle two tokens; k = 16: rows
+    # beyond the eight fetched ahead)
+    assert T * k * K >= 1 << 27
+    cfg = inputs.custom_config("q2", E=64, K=K, N=128, T=T, top_k=k)
+    X = inputs.activations(cfg)
+    ids = inputs.routing(cfg)
+    off, ps, ip = tl.route_np(ids, cfg.E)
+    s_in = torch.tensor([0.03125], dtype=torch.float32, device=DEV) if given_scale else None
+    qa = gsg.quantize_act_nvfp4(X.to(DEV), 32, torch.from_numpy(ip).to(DEV), k, x_scale_in=s_in)
+    r, qd = gsg.moe_dispatch_nvfp4(ids.to(DEV), X.to(DEV), cfg.E, 32, x_scale_in=s_in)
+    _status_ok(gsg)
+    codes, quad, s, _, _ = tl.oracle_act(X.float().numpy(), 32, ps, k, 0.03125 if given_scale else None)
+    assert qa.x_scale.item() == s
+    np.testing.assert_array_equal(qa.codes.cpu().numpy(), codes)
+    np.testing.assert_array_equal(qa.scales.cpu().numpy(), quad)
+    assert torch.equal(qd.codes, qa.codes) and torch.equal(qd.scales, qa.scales) and torch.equal(qd.x_scale, qa.x_scale)
+
+
 def _rounding_rows():
     """bf16 rows whose 32-element blocks put values exactly on E2M1 rounding midpoints and block
     maxima exactly on UE4M3 midpoints, subnormals and the saturation limit (with s_x = 1)."""
