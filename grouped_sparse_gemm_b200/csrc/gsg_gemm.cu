@@ -52,6 +52,7 @@ struct GemmParams {
   int* status;
   int E, N, K, R, y_f32, rcap;
   int stages, nacc, tcap;
+  int sched;               // tile schedule: kSchedRoundRobin or kSchedRuns (see tile_of)
   uint8_t* h_scales;       // SwiGLU epilogue: h scales, quad layout [N/256][R+256][4][4]
   const float* h_scale;    // SwiGLU epilogue: tensor scale of h
   // combine epilogue (perm_src non-null): Y is the slot buffer [T*k][N] bf16 (row = flat index
@@ -203,6 +204,7 @@ __host__ __device__ inline uint32_t make_idesc(bool sparse, int BN) {
 struct Ctl {
   int abort;
   uint32_t tmem_base;
+  int tile_begin, tile_end;   // this CTA's contiguous range of tiles
 };
 
 // Bounded wait: true when the phase completed; false on timeout or when another role aborted.
@@ -251,15 +253,58 @@ __device__ __forceinline__ TileDesc decode_tile(int t, const int* pref, const in
   return d;
 }
 
-// The j-th tile of this CTA (tile index blockIdx.x + j * gridDim.x): from the shared-memory
-// table filled at set-up, or decoded on the spot past its capacity.
+// Tile schedules (tiles numbered expert-major, then n-tile, then token tile):
+//  kSchedRoundRobin: tile j * grid + CTA.  Neighbouring tiles run at the same time on different
+//    CTAs, so the token tiles of one weight tile and the n-tiles of one activation tile are read
+//    from DRAM once and shared through L2.
+//  kSchedRuns: each CTA takes a contiguous run of tiles holding an equal share of the bytes (see
+//    tile_at_cost) and streams its own stretch of the weight array.  Used when every expert has
+//    one token tile and the CTAs hold dozens of tiles (decode batches of 32-256 tokens on 384
+//    experts: 5-10 % faster); with several token tiles per expert it loses the sharing above
+//    (the 30B and 1T prefill GEMMs ran 20-60 % slower), and with a handful of tiles per CTA
+//    (one token on 8 experts) it measured 20 % slower.  A reversed-order (snake) round-robin,
+//    tried for the load balance of heavy token tiles, measured slower than the plain one.
+constexpr int kSchedRoundRobin = 0;
+constexpr int kSchedRuns = 1;
+
+__device__ __forceinline__ int tile_of(int j, int sched, int tb) {
+  if (sched == kSchedRuns) return tb + j;
+  return j * (int)gridDim.x + (int)blockIdx.x;
+}
+
+// The j-th tile of this CTA: from the shared-memory table filled at set-up, or decoded on the
+// spot past its capacity.
 __device__ __forceinline__ TileDesc my_tile(int j, const int4* table, int tcap, const int* pref, const int* offs,
-                                            int E, int BN) {
+                                            int E, int BN, int sched, int tb) {
   if (j < tcap) {
     const int4 v = table[j];
     return TileDesc{v.x, v.y, v.z, v.w};
   }
-  return decode_tile(blockIdx.x + j * (int)gridDim.x, pref, offs, E, BN);
+  return decode_tile(tile_of(j, sched, tb), pref, offs, E, BN);
+}
+
+// Tile schedule: every CTA takes a contiguous run of tiles (expert-major, then n-tile, then token
+// tile) holding an equal share of the launch's bytes.  A tile's cost is its weight bytes wc plus
+// ac per token row (activation codes and scales, output); costp[e] = cost of experts < e.  Returns
+// the first tile that starts at or after `target` bytes (total_tiles when none does).
+__device__ __forceinline__ int tile_at_cost(long long target, const long long* costp, const int* pref,
+                                            const int* offs, int E, int BN, long long wc, long long ac) {
+  if (target >= costp[E]) return pref[E];
+  int lo = 0, hi = E;   // largest e with costp[e] <= target: a non-empty expert
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (costp[mid] <= target) lo = mid; else hi = mid;
+  }
+  const int rows = offs[lo + 1] - offs[lo];
+  const int mte = (rows + BN - 1) / BN;
+  const long long cn = mte * wc + rows * ac;            // one n-tile's token tiles
+  const long long rel = target - costp[lo];
+  long long nt = rel / cn;
+  const long long rem = rel - nt * cn;
+  const long long cf = wc + (long long)BN * ac;         // a full token tile (all but the last)
+  long long tt = (rem + cf - 1) / cf;
+  if (tt >= mte) { ++nt; tt = 0; }
+  return pref[lo] + (int)(nt * mte + tt);
 }
 
 // Compile-time stage geometry of one (sparse/dense, token tile, SwiGLU) instantiation.  With the
@@ -308,7 +353,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
   int* offs = reinterpret_cast<int*>(ctl + 1);   // [E+1]
   int* pref = offs + (E + 1);                    // [E+1]
   float* wsc = reinterpret_cast<float*>(pref + (E + 1));   // [E]
-  int4* ttab = reinterpret_cast<int4*>((reinterpret_cast<uintptr_t>(wsc + E) + 15) & ~uintptr_t(15));   // [tcap]
+  long long* costp = reinterpret_cast<long long*>((reinterpret_cast<uintptr_t>(wsc + E) + 15) & ~uintptr_t(15));
+  int4* ttab = reinterpret_cast<int4*>((reinterpret_cast<uintptr_t>(costp + (E + 1)) + 15) & ~uintptr_t(15));
   // per-epilogue-warp staging buffer: 16 tokens x 32 output features (fp32 worst case), or the
   // SwiGLU epilogue's 32 x 36 fp32
   uint8_t* ostage = reinterpret_cast<uint8_t*>(ttab + p.tcap);   // [4][kOutStageBytes or kGluStageBytes]
@@ -395,13 +441,58 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
     }
     if (threadIdx.x == kGemmThreads - 1) pref[E] = before + incl;
   }
+  // bytes per tile: weights wc, plus ac per token row (codes, scales, output row segment)
+  const long long wc = (long long)G::kNT * kTileN * p.K * (kSparse ? 11 : 18) / 32;
+  const long long ac = p.K / 2 + p.K / (kSparse ? 32 : 16) + (long long)G::kNT * kTileN * (p.y_f32 ? 4 : 2);
+  {
+    // chunked exclusive scan of cost_e = NTt * (ceil(rows_e / BN) * wc + rows_e * ac)
+    const int per = (E + kGemmThreads - 1) / kGemmThreads;
+    const int e0 = threadIdx.x * per, e1 = min(e0 + per, E);
+    long long local = 0;
+    for (int e = e0; e < e1; ++e) {
+      const int rows = max(offs[e + 1] - offs[e], 0);
+      local += (long long)NTt * (((rows + kBN - 1) / kBN) * wc + rows * ac);
+    }
+    long long incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long n = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += n;
+    }
+    __shared__ long long csum[kGemmThreads / 32];
+    if (lane == 31) csum[warp] = incl;
+    __syncthreads();
+    long long run = incl - local;
+    for (int w = 0; w < warp; ++w) run += csum[w];
+    for (int e = e0; e < e1; ++e) {
+      costp[e] = run;
+      const int rows = max(offs[e + 1] - offs[e], 0);
+      run += (long long)NTt * (((rows + kBN - 1) / kBN) * wc + rows * ac);
+    }
+    if (threadIdx.x == kGemmThreads - 1) costp[E] = run;
+  }
   if (bad) set_status(p.status, GSG_ERR_BAD_ROUTING);
   __syncthreads();
   const int total_tiles = pref[E];
+  if (threadIdx.x == 0) {
+    const int b = (int)blockIdx.x, G_ = (int)gridDim.x;
+    if (p.sched == kSchedRuns) {
+      const long long C = costp[E];
+      const int tb = tile_at_cost(C * b / G_, costp, pref, offs, E, kBN, wc, ac);
+      const int te = b == G_ - 1 ? total_tiles : tile_at_cost(C * (b + 1) / G_, costp, pref, offs, E, kBN, wc, ac);
+      ctl->tile_begin = tb;
+      ctl->tile_end = te;
+    } else {
+      ctl->tile_begin = 0;
+      ctl->tile_end = b < total_tiles ? (total_tiles - b + G_ - 1) / G_ : 0;
+    }
+  }
+  __syncthreads();
+  const int tb = ctl->tile_begin;
   // this CTA's tiles, decoded once
-  const int n_my = (int)blockIdx.x < total_tiles ? (total_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+  const int n_my = ctl->tile_end - tb;
   for (int j = threadIdx.x; j < n_my && j < p.tcap; j += blockDim.x) {
-    const TileDesc d = decode_tile((int)blockIdx.x + j * (int)gridDim.x, pref, offs, E, kBN);
+    const TileDesc d = decode_tile(tile_of(j, p.sched, tb), pref, offs, E, kBN);
     ttab[j] = make_int4(d.e, d.nt, d.r0, d.valid);
   }
   tc_fence_before();
@@ -415,7 +506,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
     int s = 0, issued = 0;
     uint32_t ph = 0;
     for (int j = 0; j < n_my && !*abort_flag; ++j) {
-      const TileDesc c = my_tile(j, ttab, p.tcap, pref, offs, E, kBN);
+      const TileDesc c = my_tile(j, ttab, p.tcap, pref, offs, E, kBN, p.sched, tb);
       const uint8_t* wsrc = p.w_packed + ((size_t)c.e * NT + c.nt) * KC * G::kCB;
       const uint8_t* wsrc_up = wsrc + (size_t)(NT / 2) * KC * G::kCB;   // SwiGLU: the matching up n-tile
       const int r0 = c.r0;
@@ -522,7 +613,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
     uint32_t ph = 0, aph = 0;   // ring phase, accumulator phase
     bool any = false;
     for (int j = 0; j < n_my && !*abort_flag; ++j) {
-      const TileDesc c = my_tile(j, ttab, p.tcap, pref, offs, E, kBN);
+      const TileDesc c = my_tile(j, ttab, p.tcap, pref, offs, E, kBN, p.sched, tb);
       const uint32_t idesc = make_idesc(kSparse, (c.valid + 15) & ~15);
       if (!wait_warp(acce_bar(acc), aph ^ 1u, abort_flag, p.status)) break;
       tc_fence_after();
@@ -587,7 +678,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
     int acc = 0;
     uint32_t aph = 0;
     for (int j = 0; j < n_my; ++j) {
-      const TileDesc c = my_tile(j, ttab, p.tcap, pref, offs, E, kBN);
+      const TileDesc c = my_tile(j, ttab, p.tcap, pref, offs, E, kBN, p.sched, tb);
       const int r0 = c.r0, valid = c.valid;
       if (!wait_warp(accf_bar(acc), aph, abort_flag, p.status)) break;
       tc_fence_after();
@@ -782,7 +873,7 @@ static GemmPlan make_plan(bool sparse, int BN, int E, int tcap, bool glu = false
   // everything but the stage ring and the tile table, at its largest
   const int ostage = 4 * (glu ? kGluStageBytes : kOutStageBytes);
   const int fixed = 1024 + (2 * kMaxStages + kNSets + 2 * kMaxAcc + 1) * 8 + (int)sizeof(Ctl) + (3 * E + 2) * 4 +
-                    16 + ostage;
+                    16 + (E + 1) * 8 + 16 + ostage;
   int budget = g_smem_limit - fixed;
   if (BN == 128 && budget > kStageBudget128) budget = kStageBudget128;
   g.stages = (budget - tcap * 16) / g.stage;
@@ -792,6 +883,7 @@ static GemmPlan make_plan(bool sparse, int BN, int E, int tcap, bool glu = false
   if (g.nacc > kMaxAcc) g.nacc = kMaxAcc;
   const int nbars = 2 * g.stages + kNSets + 2 * g.nacc + 1;
   g.smem = 1024 + (size_t)g.stages * g.stage + nbars * 8 + sizeof(Ctl) + (size_t)(3 * E + 2) * 4 + 16 +
+           (size_t)(E + 1) * 8 + 16 +
            (size_t)tcap * 16 + ostage;
   return g;
 }
@@ -883,7 +975,22 @@ int launch_gemm(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, co
   int BN = gemm_pick_bn(max_rows, R, E);
   if (glu && BN > 64) BN = 64;   // two accumulators per tile: 64-token tiles at most
   const long long bound = (((long long)R + BN - 1) / BN + E) * (N / kTileN / (glu ? 2 : 1));
-  long long tcap = (bound + num_sms - 1) / num_sms;
+  // schedule: contiguous byte-balanced runs when every expert fits one token tile (max_rows known)
+  // and the CTAs can hold at least 32 tiles each (at most min(E, R) experts are touched), else
+  // round-robin
+  const int NTt = N / kTileN / (glu ? 2 : 1);
+  const long long touched_max = R < E ? R : E;
+  const int sched = (max_rows >= 0 && max_rows <= BN && touched_max * NTt >= 32LL * num_sms) ? kSchedRuns
+                                                                                              : kSchedRoundRobin;
+  long long tcap;
+  if (sched == kSchedRuns) {
+    // a CTA's share of the bytes holds at most (wc + BN ac) / (wc + ac) times the average tile count
+    const long long wc = (glu ? 2LL : 1LL) * kTileN * K * (sparse ? 11 : 18) / 32;
+    const long long ac = K / 2 + K / (sparse ? 32 : 16) + (glu ? 2LL : 1LL) * kTileN * (y_f32 ? 4 : 2);
+    tcap = (bound * (wc + BN * ac) / (wc + ac) + num_sms - 1) / num_sms + 2;
+  } else {
+    tcap = (bound + num_sms - 1) / num_sms;
+  }
   if (tcap > kMaxTableTiles) tcap = kMaxTableTiles;
   const GemmPlan g = make_plan(sparse, BN, E, (int)tcap, glu);
   if (g.stages < kNSets || g.smem > (size_t)g_smem_limit) return 1;   // ring too shallow: refuse, launch nothing
@@ -919,7 +1026,7 @@ int launch_gemm(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, co
   p.a_scales = a_scales; p.x_scale = x_scale; p.w_packed = w_packed;
   p.w_scale = w_scale; p.off = off; p.Y = Y; p.status = status;
   p.E = E; p.N = N; p.K = K; p.R = R; p.y_f32 = y_f32; p.rcap = rcap;
-  p.stages = g.stages; p.nacc = g.nacc; p.tcap = g.tcap;
+  p.stages = g.stages; p.nacc = g.nacc; p.tcap = g.tcap; p.sched = sched;
   p.h_scales = h_scales; p.h_scale = h_scale;
   p.perm_src = comb ? comb->perm_src : nullptr;
   p.gates = comb ? comb->gates : nullptr;
