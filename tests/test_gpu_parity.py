@@ -385,9 +385,12 @@ def test_pipeline_matches_oracle(gsg, name):
     assert np.all(err <= tol), float(np.max(err / tol))
 
 
-def test_gemm_full_size_sampled_30b_up(gsg):
-    """The bench workload (30B-A3B-shaped up-projection prefill) at full size; sampled rows."""
-    cfg = inputs.CONFIGS["30b_up_prefill"]
+@pytest.mark.parametrize("name", ["30b_up_prefill", "1t_down_decode_b32"])
+def test_gemm_full_size_sampled(gsg, name):
+    """Full-size workloads, sampled rows: the bench's 30B-A3B up-projection prefill (round-robin
+    tile schedule) and the 1T down-projection decode at 32 tokens (one token tile per expert,
+    byte-balanced contiguous runs of tiles)."""
+    cfg = inputs.CONFIGS[name]
     E, N, K = cfg.E, cfg.N, cfg.K
     pw = gsg.PackedSparseWeights(
         packed=torch.empty(gsg.lib().gsg_sparse_packed_bytes(E, N, K), dtype=torch.uint8, device=DEV),
@@ -395,7 +398,8 @@ def test_gemm_full_size_sampled_30b_up(gsg):
     ids = inputs.routing(cfg)
     off, ps, ip = tl.route_np(ids, E)
     counts = np.diff(off)
-    sample_e = sorted({int(np.argmax(counts)), int(np.argmin(counts)), 0, E - 1, 17, 64})
+    sample_e = sorted({int(np.argmax(counts)), int(np.argmin(counts)), 0, E - 1, 17, 64} if E <= 128 else
+                      {int(np.argmax(counts)), int(np.flatnonzero(counts)[0]), int(np.flatnonzero(counts)[-1])})
     canon, sws = {}, np.zeros(E, dtype=np.float32)
     for e in range(E):
         We = inputs.expert_weight(cfg, e, DEV)
@@ -420,7 +424,7 @@ def test_gemm_full_size_sampled_30b_up(gsg):
         if hi > lo:
             rows += sorted({lo, hi - 1, (lo + hi) // 2, min(lo + 128, hi - 1), min(lo + 129, hi - 1)})
     y_ref, bound = tl.reference_rows(np.array(rows), off, q, sc, 32, canon, s_x, sws)
-    tl.assert_gemm_close(Y[torch.tensor(rows, device=DEV)], y_ref, bound, "30b_up_prefill sampled")
+    tl.assert_gemm_close(Y[torch.tensor(rows, device=DEV)], y_ref, bound, f"{name} sampled")
 
 
 # ---------------------------------------------------------------- up-projection with the SwiGLU epilogue
