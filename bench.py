@@ -853,7 +853,7 @@ def run_layer(args, local):
         "us_per_layer": ms * 1e3, "tokens_per_s": L.T / (ms * 1e-3),
         "tflops_dense_equivalent": wl.flops() / (ms * 1e-3) / 1e12,
         "weight_gbs": wl.weight_bytes() / (ms * 1e-3) / 1e9, "h_tensor_scale": float(wl.h_scale.item()),
-        "kernels": "route, amax + quantize, up-projection + SwiGLU + NVFP4 of h, down-projection, unpermute",
+        "kernels": "routing with the amax pass, quantize, up-projection + SwiGLU + NVFP4 of h, down-projection, unpermute",
         "timing": "in-graph CUDA events around the layer, L2 flushed (256 MB write + 256 MB read of another "
                   "buffer) before every replay"}),
           flush=True)
