@@ -980,8 +980,8 @@ int launch_gemm(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, co
   // round-robin
   const int NTt = N / kTileN / (glu ? 2 : 1);
   const long long touched_max = R < E ? R : E;
-  const int sched = (max_rows >= 0 && max_rows <= BN && touched_max * NTt >= 32LL * num_sms) ? kSchedRuns
-                                                                                              : kSchedRoundRobin;
+  const int sched = (max_rows > 0 && max_rows <= BN && touched_max * NTt >= 32LL * num_sms) ? kSchedRuns
+                                                                                             : kSchedRoundRobin;
   long long tcap;
   if (sched == kSchedRuns) {
     // a CTA's share of the bytes holds at most (wc + BN ac) / (wc + ac) times the average tile count

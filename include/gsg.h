@@ -167,7 +167,8 @@ gsg_status_t gsg_moe_dispatch_nvfp4(const int32_t* topk_ids, const uint16_t* X, 
  * a_codes/a_scales from gsg_quantize_act_nvfp4 (sf_block 32); w_packed and w_tensor_scale from
  * gsg_pack_sparse_nvfp4.
  * expert_offsets int32 [E+1], monotone, off[0] = 0, off[E] <= R.  max_rows_per_expert is a
- * host-side hint that picks the token tile (<= 0: unknown).  Y [R][N] bf16 (y_dtype
+ * host-side hint that picks the token tile and the tile schedule (<= 0: unknown); any value
+ * gives a correct result, a wrong one only a slower launch.  Y [R][N] bf16 (y_dtype
  * GSG_OUT_BF16) or fp32 (GSG_OUT_F32); rows >= off[E] are not written.  No workspace.
  * Persistent kernel, one CTA per SM: TMA/bulk copies into a shared-memory ring, tcgen05
  * block-scaled sparse MMA into TMEM, epilogue applies s_x*s_w[e].
