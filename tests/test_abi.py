@@ -83,6 +83,17 @@ def test_host_argument_checks(L):
     assert L.gsg_quantize_act_nvfp4(P, 4, 256, 32, P, 2, None, P, P, P, None, 0, None) == -7
     assert L.gsg_unpermute_scale(P, P, P, 4, 2, 12, P, None) == -1
     assert L.gsg_unpermute_scale(P, P, P, 0, 2, 128, P, None) == 0
+    # two-phase scale path (R*K >= 2^27): its workspace is needed even with a caller-supplied s_x
+    assert L.gsg_quantize_act_nvfp4(P, 2048, 8192, 32, P, 8, P, P, P, P, None, 0, None) == -7
+    # the combined routing + quantize call: the checks of both calls, and its own workspace
+    ws_need = L.gsg_workspace_size(gsg.OP_DISPATCH, 16, 0, 256, 4, 2)
+    assert L.gsg_moe_dispatch_nvfp4(P, P, 4, 2, 16, 256, 24, None, P, P, P, P, P, P, P, 1 << 20, None) == -1
+    assert L.gsg_moe_dispatch_nvfp4(P, P, 4, 2, 0, 256, 32, None, P, P, P, P, P, P, P, 1 << 20, None) == -2
+    assert L.gsg_moe_dispatch_nvfp4(P, P, 4, 2, 16, 200, 32, None, P, P, P, P, P, P, P, 1 << 20, None) == -2
+    assert L.gsg_moe_dispatch_nvfp4(P, None, 4, 2, 16, 256, 32, None, P, P, P, P, P, P, P, 1 << 20, None) == -1
+    assert L.gsg_moe_dispatch_nvfp4(P, P, 4, 2, 16, 256, 32, None, P, P, P, P, P, P, None, 0, None) == -7
+    assert L.gsg_moe_dispatch_nvfp4(P, P, 4, 2, 16, 256, 32, None, P, P, P, P, P, P, P, ws_need - 1, None) == -7
+    assert L.gsg_moe_dispatch_nvfp4(P, P, 4, 2, 16, 256, 32, None, P, P, P, P, P, P, ctypes.c_void_p(20), 1 << 20, None) == -7
 
 
 def test_binding_refuses_cpu_tensors():
