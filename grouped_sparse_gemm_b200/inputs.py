@@ -65,6 +65,12 @@ for _b in (1, 32, 128, 256):
     CONFIGS[f"1t_down_decode_b{_b}"] = MoEConfig(
         f"1t_down_decode_b{_b}", E=384, K=2048, N=7168, T=_b, top_k=8,
         routing="uniform", w_sigma=0.015)
+# The 1T prefill up-projection on 64 of its experts with the same average rows per expert
+# (1368 tokens top-8 = 171 per expert): the same kernel instantiation (128-token tiles) on
+# 0.65 GB of weights, small enough for profiler captures of all counters.
+CONFIGS["1t_up_prefill_e64"] = MoEConfig("1t_up_prefill_e64", E=64, K=7168, N=4096, T=1368, top_k=8,
+                                         routing="zipf", zipf_s=1.1, w_sigma=0.015,
+                                         outlier_frac=0.005, outlier_scale=30.0)
 
 
 @dataclasses.dataclass(frozen=True)
