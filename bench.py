@@ -209,8 +209,6 @@ class Workload:
         self.route = gsg.Routing(offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
                                  perm_src=torch.empty(R, dtype=torch.int32, device=dev),
                                  inv_perm=torch.empty(R, dtype=torch.int32, device=dev), T=T, k=k, E=E)
-        self.ws_route = torch.empty(max(gsg.workspace_size(gsg.OP_ROUTE, E, 0, 0, T, k), 16), **u8)
-        self.ws_quant = torch.empty(max(gsg.workspace_size(gsg.OP_QUANTIZE, 0, 0, K, T, k), 16), **u8)
         self.ws_disp = torch.empty(max(gsg.workspace_size(gsg.OP_DISPATCH, E, 0, K, T, k), 16), **u8)
         self.qa = gsg.QuantizedActivations(codes=torch.empty(R, K // 2, **u8),
                                            scales=torch.empty(gsg.act_scales_bytes(R, K, 32), **u8),
