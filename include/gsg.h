@@ -20,7 +20,8 @@
  *     gsg_get_device_status.  Outputs of a call that raised a device error are unspecified.
  *   - Shapes: K % 256 == 0, N % 128 == 0, E >= 1.  bf16 tensors are passed as uint16_t bit
  *     patterns.  Multi-dimensional buffers are dense, last index fastest.
- *   - Re-entrant across streams; the only global state is the device status word.
+ *   - Re-entrant across streams; the only global state is the device status word (and the
+ *     fixed scratch of gsg_moe_route_permute_noalloc, described there).
  *
  * Packed weight layout (one buffer, tile-major, the order the GEMM streams it): for expert e,
  * n-tile nt (128 output rows, NT = N/128) and 256-wide K chunk kc, one contiguous chunk block
