@@ -22,16 +22,27 @@ __device__ __forceinline__ void select_pairs(const float w[8], int& i0, int& i1)
 #pragma unroll
   for (int p = 0; p < 4; ++p)
     m[p] = __fadd_rn(__fmul_rn(w[2 * p], w[2 * p]), __fmul_rn(w[2 * p + 1], w[2 * p + 1]));
+  // running maxima carried by value (an index into m would put m in local memory)
   int a = 0;
+  float ma = m[0];
 #pragma unroll
   for (int p = 1; p < 4; ++p)
-    if (m[p] > m[a]) a = p;
+    if (m[p] > ma) { ma = m[p]; a = p; }
   int b = (a == 0) ? 1 : 0;
+  float mb = (a == 0) ? m[1] : m[0];
 #pragma unroll
   for (int p = 0; p < 4; ++p)
-    if (p != a && m[p] > m[b]) b = p;
+    if (p != a && m[p] > mb) { mb = m[p]; b = p; }
   i0 = a < b ? a : b;
   i1 = a < b ? b : a;
+}
+
+// Element 2*i + half of w (i = pair index 0..3) by selects, not an indexed load: a runtime index
+// into w would put the array in local memory.
+__device__ __forceinline__ float pair_elem(const float w[8], int i, int half) {
+  const float lo = i == 0 ? w[0] : i == 1 ? w[2] : i == 2 ? w[4] : w[6];
+  const float hi = i == 0 ? w[1] : i == 1 ? w[3] : i == 2 ? w[5] : w[7];
+  return half ? hi : lo;
 }
 
 __device__ __forceinline__ bool all_finite8(const float w[8]) {
@@ -83,8 +94,8 @@ pack_amax_kernel(const float* __restrict__ W, long long groups_per_expert, float
     if (kSparse) {
       int i0, i1;
       select_pairs(w, i0, i1);
-      mx = fmaxf(mx, fmaxf(fmaxf(fabsf(w[2 * i0]), fabsf(w[2 * i0 + 1])),
-                           fmaxf(fabsf(w[2 * i1]), fabsf(w[2 * i1 + 1]))));
+      mx = fmaxf(mx, fmaxf(fmaxf(fabsf(pair_elem(w, i0, 0)), fabsf(pair_elem(w, i0, 1))),
+                           fmaxf(fabsf(pair_elem(w, i1, 0)), fabsf(pair_elem(w, i1, 1)))));
     } else {
 #pragma unroll
       for (int i = 0; i < 8; ++i) mx = fmaxf(mx, fabsf(w[i]));
@@ -126,10 +137,10 @@ pack_sparse_encode_kernel(const float* __restrict__ W, int N, int K, const float
       load8(src + 8 * g, w);
       int i0, i1;
       select_pairs(w, i0, i1);
-      kept[4 * g + 0] = w[2 * i0];
-      kept[4 * g + 1] = w[2 * i0 + 1];
-      kept[4 * g + 2] = w[2 * i1];
-      kept[4 * g + 3] = w[2 * i1 + 1];
+      kept[4 * g + 0] = pair_elem(w, i0, 0);
+      kept[4 * g + 1] = pair_elem(w, i0, 1);
+      kept[4 * g + 2] = pair_elem(w, i1, 0);
+      kept[4 * g + 3] = pair_elem(w, i1, 1);
       pat[g] = uint32_t(i0) | (uint32_t(i1) << 2);
 #pragma unroll
       for (int i = 0; i < 4; ++i) bmax = fmaxf(bmax, fabsf(kept[4 * g + i]));
