@@ -5,9 +5,11 @@
 // and is fused with dispatch for the first expert GEMM; §3.4 (pp.5-6): weights and quantized
 // activations are packed in corresponding scale blocks.
 //
-// Launch 1 (skipped when the caller supplies s_x): partial max|X| per block, 128-bit loads,
-// warp-shuffle reductions.  Launch 2, 32-element blocks (the sparse path): one lane per block
-// (act_quant32_kernel, below).  Launch 2, 16-element blocks (the dense control): every block
+// Launch 1 (skipped when the caller supplies s_x, or made by the routing's first launch in
+// gsg_moe_dispatch_nvfp4): partial max|X| per block, 128-bit loads, warp-shuffle reductions.
+// Launch 2, 32-element blocks (the sparse path): one lane per block (act_quant32_kernel, below;
+// from R*K = 2^27 followed by act_scales_quad_kernel).  Launch 2, 16-element blocks (the dense
+// control): every block
 // folds the partials into s_x = amax/2688,
 // then each warp quantizes 256 consecutive elements of one token row at a time (8 per lane, one
 // 128-bit load), groups of 4 lanes (2 for 16-element blocks) combine their maxima into the

@@ -14,8 +14,9 @@
 // latency-bound and a second launch costs more than the block's extra round (measured: at
 // R = 4096 four indices per thread in one block are slower than two launches).  Larger R is
 // histogram -> (scan) -> scatter over a [chunks x E] workspace, the scan folded into the
-// scatter for 1024-index chunks.  Only integer arithmetic: the result is
-// deterministic.
+// scatter for 1024-index chunks.  For gsg_moe_dispatch_nvfp4 the first of these launches also
+// carries the activation quantizer's amax blocks (route_amax_kernel).  Only integer arithmetic:
+// the result is deterministic.
 #include "gsg_internal.cuh"
 
 namespace gsg {
