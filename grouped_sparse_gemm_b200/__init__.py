@@ -7,7 +7,9 @@ There is no CPU fallback: if the library is missing or no GPU is present the cal
 
 The path (after "Hardware-Native Joint Sparse-Quantization for Trillion-Scale Mixture-of-Experts",
 paperlayer.ai summary, §3.4 and §D.1): pack_sparse_nvfp4 (offline weights) ->
-moe_route_permute -> quantize_act_nvfp4 -> grouped_sparse_gemm -> unpermute_scale.
+moe_route_permute -> quantize_act_nvfp4 -> grouped_sparse_gemm -> unpermute_scale
+(moe_dispatch_nvfp4 = the routing and quantizer calls in one).  save_packed / load_packed keep
+packed weights in a file: the packed format is the storage format.
 """
 from __future__ import annotations
 
@@ -28,6 +30,7 @@ __all__ = [
     "grouped_sparse_gemm", "grouped_sparse_gemm_swiglu", "grouped_sparse_gemm_combine", "combine_workspace",
     "grouped_dense_gemm", "unpermute_scale", "OP_COMBINE", "OP_DISPATCH",
     "get_device_status",
+    "save_packed", "load_packed",
     "act_scales_bytes", "workspace_size", "OP_PACK_SPARSE", "OP_PACK_DENSE", "OP_ROUTE",
     "OP_QUANTIZE", "OP_GEMM", "EXPORTED_SYMBOLS",
 ]
@@ -201,6 +204,46 @@ class QuantizedActivations:
     R: int
     K: int
     sf_block: int
+
+
+# ------------------------------------------------------------------ storage
+PACKED_FILE_VERSION = 1
+
+
+def save_packed(w, path: str) -> None:
+    """Packed weights (PackedSparseWeights or PackedDenseWeights, any device) to an .npz file: the
+    packed bytes exactly as the GEMM reads them, the per-expert FP32 tensor scales, E, N, K and
+    the format.  No re-encoding: load_packed gives back the same bytes."""
+    import numpy as np
+    fmt = "sparse" if isinstance(w, PackedSparseWeights) else "dense"
+    np.savez(path, version=PACKED_FILE_VERSION, format=fmt, E=w.E, N=w.N, K=w.K,
+             packed=w.packed.detach().cpu().numpy(), w_scale=w.w_scale.detach().cpu().numpy())
+
+
+def load_packed(path: str, device=None):
+    """Packed weights from a save_packed file, on `device` (default: CPU).  Checks the version,
+    the format and that the byte count is the library's size for (E, N, K); raises ValueError
+    otherwise."""
+    import numpy as np
+    with np.load(path, allow_pickle=False) as d:
+        if int(d["version"]) != PACKED_FILE_VERSION:
+            raise ValueError(f"{path}: packed-weights file version {int(d['version'])}, expected "
+                             f"{PACKED_FILE_VERSION}")
+        fmt = str(d["format"])
+        E, N, K = int(d["E"]), int(d["N"]), int(d["K"])
+        packed, w_scale = d["packed"], d["w_scale"]
+    if fmt not in ("sparse", "dense"):
+        raise ValueError(f"{path}: unknown packed format {fmt!r}")
+    L = lib()
+    need = L.gsg_sparse_packed_bytes(E, N, K) if fmt == "sparse" else L.gsg_dense_packed_bytes(E, N, K)
+    if packed.dtype != np.uint8 or packed.ndim != 1 or packed.size != need:
+        raise ValueError(f"{path}: {packed.size} packed bytes, expected {need} for {fmt} E={E} N={N} K={K}")
+    if w_scale.dtype != np.float32 or w_scale.shape != (E,):
+        raise ValueError(f"{path}: tensor scales of shape {w_scale.shape} / {w_scale.dtype}, expected ({E},) float32")
+    pk = torch.from_numpy(packed.copy()).to(device or "cpu")
+    ws = torch.from_numpy(w_scale.copy()).to(device or "cpu")
+    cls = PackedSparseWeights if fmt == "sparse" else PackedDenseWeights
+    return cls(packed=pk, w_scale=ws, E=E, N=N, K=K)
 
 
 # ------------------------------------------------------------------ entry points
