@@ -319,6 +319,24 @@ def test_gemm_deterministic(gsg):
     assert torch.equal(y1, y2)
 
 
+def test_gemm_flags_corrupt_offsets(gsg):
+    """Offsets that decrease or leave [0, R] are clamped in the kernel (a decreasing pair makes
+    that expert empty), so nothing is read or written out of bounds, and the call reports
+    GSG_ERR_BAD_ROUTING; the rows of the experts whose offsets are intact are still right."""
+    c = _gemm_case([16, 8, 24, 8], 128, 256, sparse=True)
+    good = c["off"].copy()                       # [0, 16, 24, 48, 56]
+    bad = dict(c)
+    bad["off"] = np.array([0, 16, 10, 999999, 56], dtype=np.int32)
+    y = _run_gemm(gsg, bad, True, -1, torch.float32)
+    torch.cuda.synchronize()
+    assert gsg.get_device_status() == -4
+    _status_ok(gsg)
+    # clamped offsets [0, 16, 10, 56, 56]: rows [0, 10) belong to expert 0 alone (rows 10..15 are
+    # claimed by expert 2 as well), and they still hold the oracle's values
+    y_ref, bound = tl.reference_rows(np.arange(10), good, c["q"], c["sc"], 32, c["canon"], c["s_x"], c["sws"])
+    tl.assert_gemm_close(y[:10], y_ref, bound, "expert 0 beside corrupt offsets")
+
+
 def test_dense_and_sparse_agree_on_48_weights(gsg):
     """The control differs from the sparse kernel only in sparsity: a W that is already paired
     4:8 gives results within tolerance of one reference on both (32-blocks copied into 16-blocks)."""
