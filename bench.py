@@ -47,7 +47,8 @@ if ROOT not in sys.path:
 import grouped_sparse_gemm_b200 as gsg  # noqa: E402
 from grouped_sparse_gemm_b200 import inputs  # noqa: E402
 
-DEFAULT_CONFIG = "30b_up_prefill"
+DEFAULT_CONFIG = "1t_up_prefill"          # the largest configuration: the headline
+SECONDARY_CONFIG = "30b_up_prefill"       # reported beside it (GEMM and step times only)
 METRIC = "grouped sparse-NVFP4 GEMM TFLOP/s + weight GB/s, as % of B200 roofline"
 SPARSE_NVFP4_PEAK_TFLOPS_NOMINAL = 18000.0     # the pages' sparse NVFP4 figure (dense-equivalent)
 HBM_NOMINAL_GBS = 8000.0
@@ -122,17 +123,32 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+def gpu_uuid(dev) -> str | None:
+    """The UUID ("GPU-...") of the device torch uses as `dev`.  nvidia-smi and NVML number GPUs
+    physically, while under CUDA_VISIBLE_DEVICES torch's device 0 can be any of them: the UUID
+    names the same GPU on both sides."""
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        return None
+    return u if u.startswith("GPU-") else "GPU-" + u
+
+
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """nvidia-smi clocks and throttle reasons sampled during the timed region, on the GPU with
+    the given UUID (the one the process runs on)."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, uuid: str | None):
         self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.uuid = uuid
         try:
+            if uuid is None:
+                raise RuntimeError("no device UUID")
             self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                                       "-i", str(gpu_index), "-lms", "50"], stdout=self.f, stderr=subprocess.DEVNULL)
+                                       "-i", uuid, "-lms", "50"], stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.p = None
         # the first query initialises NVML and can stall the device briefly: wait for it to land
@@ -166,10 +182,11 @@ class ClockSampler:
             except (ValueError, IndexError):
                 continue
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": 0,
+                    "gpu_uuid": self.uuid}
         busy = [s for s in sm if s > 0.5 * max(sm)]
         return {"sm_mhz": statistics.median(busy), "sm_max_mhz": smax, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "gpu_uuid": self.uuid}
 
 
 # ------------------------------------------------------------------ workload
@@ -546,20 +563,29 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
-def traffic_from_profiles(config_name: str):
-    """DRAM bytes per GEMM launch from the committed ncu summary, if the kernel is unchanged."""
+def traffic_from_profiles(config_name: str, algorithmic_bytes: int):
+    """DRAM bytes per GEMM launch from the committed ncu summary, if the kernel is unchanged.
+    An entry captured on a smaller case of the same instantiation ("scaled_from") is scaled to
+    this launch by its algorithmic bytes (the kernel's DRAM traffic grows in proportion to them).
+    Returns (bytes or None, how)."""
     p = os.path.join(ROOT, "profiles", "gemm_traffic.json")
     if not os.path.exists(p):
-        return None
+        return None, "no capture"
     with open(p) as f:
         d = json.load(f)
     src = os.path.join(ROOT, "grouped_sparse_gemm_b200", "csrc", "gsg_gemm.cu")
     with open(src, "rb") as f:
         sha = hashlib.sha256(f.read()).hexdigest()[:16]
     ent = d.get(config_name)
-    if not ent or ent.get("gemm_src_sha") != sha:
-        return None
-    return ent.get("dram_bytes_per_launch")
+    if not ent:
+        return None, "no capture of this workload"
+    if ent.get("gemm_src_sha") != sha:
+        return None, "kernel changed since the capture"
+    if ent.get("scaled_from"):
+        ratio = algorithmic_bytes / float(ent["algorithmic_bytes_captured"])
+        return int(ent["dram_bytes_per_launch_captured"] * ratio), (
+            f"ncu capture of {ent['scaled_from']} scaled by algorithmic bytes ({ratio:.3f}x)")
+    return ent.get("dram_bytes_per_launch"), "ncu capture of this launch"
 
 
 def run_ours(args, world, rank, local):
@@ -583,7 +609,7 @@ def run_ours(args, world, rank, local):
         (gt_step[0] if in_graph else g_step).replay()
     torch.cuda.synchronize()
 
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(gpu_uuid(dev))
     if in_graph:
         step_ms, _ = timed_graph_ms(gt_step, args.steps, flush, world)
         gemm_ms, _ = timed_graph_ms(gt_gemm, args.steps, flush, world)
@@ -608,6 +634,9 @@ def run_ours(args, world, rank, local):
 
     flops = 2.0 * cfg.R * cfg.N * cfg.K
     w_b, a_b, y_b = wl.gemm_bytes()
+    touched, max_rows = wl.touched, wl.max_rows
+    X_h, ids_h = wl.X_h, wl.ids_h
+    launches = wl.launches_per_step()
     value = job_value(flops, world, step_ms)
     peaks, peak_kind = measured_peaks()
     hbm_peak = float(peaks["hbm_gbs"])
@@ -671,9 +700,14 @@ def run_ours(args, world, rank, local):
                    "hbm_gbs": wl.dense_gemm_bytes() / (dense_ms * 1e-3) / 1e9,
                    "sparse_speedup": dense_ms / gemm_ms}
 
+    traffic = traffic_from_profiles(cfg.name, int(gemm_bytes))
+    secondary = None
+    if not args.quick and SECONDARY_CONFIG != cfg.name:
+        secondary = secondary_figures(SECONDARY_CONFIG, dev, args, world)
+
     cpu = None
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
-        smp = OracleSample(cfg, wl.X_h, wl.ids_h, args.cpu_experts)
+        smp = OracleSample(cfg, X_h, ids_h, cpu_sample_experts(cfg, args.cpu_experts))
         dt, fl = smp.run(smp.units)
         passes = 1
         while dt < 10.0:          # repeat the same sample until about 10 s of CPU work
@@ -706,11 +740,11 @@ def run_ours(args, world, rank, local):
                 "tensor_sparse_nvfp4_nominal_18pf": 100.0 * value / world / SPARSE_NVFP4_PEAK_TFLOPS_NOMINAL,
                 "hbm_nominal_8tbs": 100.0 * (gemm_bytes / (step_ms * 1e-3) / 1e9) / HBM_NOMINAL_GBS},
             "gemm": {"ms": gemm_ms_max, "tflops": gemm_tflops, "weight_gbs": w_b / (gemm_ms * 1e-3) / 1e9,
-                     "total_gbs": achieved_gbs, "token_tile": gsg_token_tile(wl.max_rows, cfg.R, cfg.E),
-                     "touched_experts": wl.touched, "max_rows_per_expert": wl.max_rows,
+                     "total_gbs": achieved_gbs, "token_tile": gsg_token_tile(max_rows, cfg.R, cfg.E),
+                     "touched_experts": touched, "max_rows_per_expert": max_rows,
                      "tensor_frac_of_measured": gemm_tflops / tensor_peak},
             "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
-                         "frac": achieved_gbs / hbm_peak, "traffic": traffic_from_profiles(cfg.name),
+                         "frac": achieved_gbs / hbm_peak, "traffic": traffic[0], "traffic_source": traffic[1],
                          "kernel": "grouped_gemm_kernel<sparse>",
                          "algorithmic_bytes_per_launch": int(gemm_bytes),
                          "peak_source": f"{peak_kind} hbm_gbs (burst copy)"},
@@ -721,10 +755,52 @@ def run_ours(args, world, rank, local):
             "e2e": e2e,
             "cpu_baseline": cpu,
             "control": control,
-            "gpu_launches": wl.launches_per_step() * args.steps,
+            "gpu_launches": launches * args.steps,
+            "secondary": secondary,
             "clocks": clk,
         }
         print(json.dumps(line), flush=True)
+
+
+def cpu_sample_experts(cfg, requested):
+    """Experts in the CPU oracle's sample: as requested, else about 1.2e8 weights' worth (24 at the
+    30B shapes, 4 at the 1T shapes) so that the sample's untimed preparation stays near 15 s."""
+    if requested:
+        return requested
+    return int(min(24, max(2, 1.2e8 // (cfg.N * cfg.K))))
+
+
+def secondary_figures(name: str, dev, args, world):
+    """A second configuration's GEMM and step times (same flush and two timings as the headline,
+    no control, no end-to-end, no CPU sample)."""
+    cfg = inputs.CONFIGS[name]
+    wl = Workload(cfg, dev, with_dense=False)
+    flush = L2Flush(dev)
+    wl.step()
+    torch.cuda.synchronize()
+    res = {"workload": workload_config(cfg)["workload"]}
+    for tag, fn in (("step", wl.step), ("gemm", wl.gemm)):
+        gt = capture_timed(fn)
+        for _ in range(args.warmup):
+            flush.fill_(1)
+            gt[0].replay()
+        ev, _ = timed_graph_ms(gt, args.steps, flush, world)
+        bb = batched_ms(capture(fn).replay, flush, 200, world)
+        res[tag + "_ms"] = max_over_ranks(max(ev, bb), world, dev)
+        del gt
+    st = gsg.get_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} on {name}")
+    flops = 2.0 * cfg.R * cfg.N * cfg.K
+    w_b, a_b, y_b = wl.gemm_bytes()
+    peaks, _ = measured_peaks()
+    res.update({"step_tflops": job_value(flops, world, res["step_ms"]),
+                "gemm_tflops": flops / (res["gemm_ms"] * 1e-3) / 1e12,
+                "gemm_hbm_gbs": (w_b + a_b + y_b) / (res["gemm_ms"] * 1e-3) / 1e9,
+                "gemm_hbm_frac": (w_b + a_b + y_b) / (res["gemm_ms"] * 1e-3) / 1e9 / float(peaks["hbm_gbs"])})
+    del wl, flush
+    torch.cuda.empty_cache()
+    return res
 
 
 def gsg_token_tile(max_rows: int, R: int, E: int) -> int:
@@ -915,11 +991,11 @@ SWEEP_SHAPES = {            # expert projection shapes: (K, N)
 class Energy:
     """Board energy counter through NVML (read only); None when NVML is not available."""
 
-    def __init__(self, index: int):
+    def __init__(self, uuid: str | None):
         try:
             import pynvml
             pynvml.nvmlInit()
-            self.nv, self.h = pynvml, pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.nv, self.h = pynvml, pynvml.nvmlDeviceGetHandleByUUID(uuid)
             self.nv.nvmlDeviceGetTotalEnergyConsumption(self.h)
         except Exception:
             self.nv = None
@@ -939,7 +1015,7 @@ def run_sweep(args, local):
     L = gsg.lib()
     u8 = dict(dtype=torch.uint8, device=dev)
     flush = L2Flush(dev)
-    energy = Energy(local)
+    energy = Energy(gpu_uuid(dev))
     Gs = [int(x) for x in args.sweep_g.split(",")]
     Ns = [int(x) for x in args.sweep_n.split(",")]
     shapes = args.sweep_shapes.split(",")
@@ -1057,7 +1133,8 @@ def main():
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(inputs.CONFIGS))
     ap.add_argument("--quick", action="store_true", help="skip e2e, dense control and CPU baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-experts", type=int, default=24)
+    ap.add_argument("--cpu-experts", type=int, default=None,
+                    help="experts in the CPU oracle's sample (default: by expert size, 24 at 30B, 4 at 1T)")
     ap.add_argument("--all-configs", action="store_true",
                     help="GEMM, step and dense control for every configuration (one JSON line each)")
     ap.add_argument("--configs", default=None, help="comma-separated subset for --all-configs")

@@ -46,7 +46,7 @@ EXPORTED_SYMBOLS = [
     "gsg_quantize_act_nvfp4", "gsg_grouped_sparse_gemm", "gsg_grouped_dense_gemm",
     "gsg_unpermute_scale", "gsg_get_device_status", "gsg_status_string", "gsg_version",
     "gsg_moe_route_permute_noalloc", "gsg_grouped_sparse_gemm_swiglu", "gsg_grouped_sparse_gemm_combine",
-    "gsg_moe_dispatch_nvfp4",
+    "gsg_moe_dispatch_nvfp4", "gsg_test_set_gemm_stall_ns",
 ]
 
 _STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported shape", -3: "CUDA error",
@@ -98,6 +98,7 @@ def load_library(build_if_missing: bool = False) -> ctypes.CDLL:
         "gsg_moe_route_permute_noalloc": (i, [vp, i, i, i, vp, vp, vp, vp]),
         "gsg_grouped_sparse_gemm_swiglu": (i, [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, vp, vp, vp]),
         "gsg_grouped_sparse_gemm_combine": (i, [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, vp, vp, sz, vp, vp]),
+        "gsg_test_set_gemm_stall_ns": (None, [ctypes.c_ulonglong]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -234,6 +235,13 @@ def load_packed(path: str, device=None):
         packed, w_scale = d["packed"], d["w_scale"]
     if fmt not in ("sparse", "dense"):
         raise ValueError(f"{path}: unknown packed format {fmt!r}")
+    # the shape rule of the packers (whole 128-row n-tiles, whole 256-wide K chunks, int range),
+    # checked before the byte count so that a wrong N or K of the right size is still rejected
+    int_max = 2 ** 31 - 1
+    if not (1 <= E <= int_max and 128 <= N <= int_max and 256 <= K <= int_max and N % 128 == 0
+            and K % 256 == 0):
+        raise ValueError(f"{path}: E={E} N={N} K={K} is not a packed shape (E >= 1, N a multiple of 128, "
+                         f"K a multiple of 256)")
     L = lib()
     need = L.gsg_sparse_packed_bytes(E, N, K) if fmt == "sparse" else L.gsg_dense_packed_bytes(E, N, K)
     if packed.dtype != np.uint8 or packed.ndim != 1 or packed.size != need:

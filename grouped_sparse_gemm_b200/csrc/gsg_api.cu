@@ -356,4 +356,6 @@ const char* gsg_status_string(gsg_status_t s) {
 
 int gsg_version(void) { return 1; }
 
+void gsg_test_set_gemm_stall_ns(unsigned long long ns) { gsg::gemm_set_test_stall(ns); }
+
 }  // extern "C"

@@ -24,6 +24,8 @@
 // Experts with no rows produce no tiles.  Every mbarrier wait is bounded:
 // on expiry the kernel records GSG_ERR_DEVICE_TIMEOUT, drains its own copies and MMAs, frees
 // TMEM and returns.
+#include <atomic>
+
 #include <cuda.h>
 
 #include "gsg_internal.cuh"
@@ -62,6 +64,11 @@ struct GemmParams {
   int* counters;
   uint16_t* out;
   int k;
+  // test hook (0 = off): before its second tile (its first, if it has only one) the MMA warp waits
+  // this long on a barrier that nothing arrives on, so that the bounded wait runs out and the
+  // abort path -- status word, drain of copies and MMAs, TMEM release -- runs as it would after
+  // a real stall
+  unsigned long long stall_ns;
 };
 
 // ------------------------------------------------------------------ PTX wrappers
@@ -208,14 +215,15 @@ struct Ctl {
 };
 
 // Bounded wait: true when the phase completed; false on timeout or when another role aborted.
-__device__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* status) {
+__device__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* status,
+                             uint64_t limit_ns = kWaitTimeoutNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 63u) == 0u) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         set_status(status, GSG_ERR_DEVICE_TIMEOUT);
         return false;
@@ -226,8 +234,9 @@ __device__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_
 
 // Warp-uniform bounded wait: every lane polls, and the warp agrees on the outcome so that the
 // .sync instructions that follow (elect.sync, tcgen05.ld/st) always see a converged warp.
-__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* status) {
-  const bool ok = wait_bounded(bar, parity, abort_flag, status);
+__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag, int* status,
+                                          uint64_t limit_ns = kWaitTimeoutNs) {
+  const bool ok = wait_bounded(bar, parity, abort_flag, status, limit_ns);
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -347,8 +356,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
   const int S = p.stages, NACC = p.nacc;
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + (size_t)S * G::kStage);
-  // bars: full[S], empty[S], tfull[kNSets], accf[NACC], acce[NACC], drain
-  const int nbars = 2 * S + kNSets + 2 * NACC + 1;
+  // bars: full[S], empty[S], tfull[kNSets], accf[NACC], acce[NACC], drain, never (test hook)
+  const int nbars = 2 * S + kNSets + 2 * NACC + 2;
   Ctl* ctl = reinterpret_cast<Ctl*>(bars + nbars);
   int* offs = reinterpret_cast<int*>(ctl + 1);   // [E+1]
   int* pref = offs + (E + 1);                    // [E+1]
@@ -369,6 +378,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
   auto accf_bar = [&](int a) { return bar0 + 8u * (2 * S + kNSets + a); };
   auto acce_bar = [&](int a) { return bar0 + 8u * (2 * S + kNSets + NACC + a); };
   const uint32_t drain_bar = bar0 + 8u * (2 * S + kNSets + 2 * NACC);
+  const uint32_t never_bar = drain_bar + 8u;
 
   // ---- set-up: barriers, TMEM, tile schedule, tensor scales (global memory only after pdl_wait)
   pdl_launch_dependents();
@@ -382,6 +392,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
     for (int s = 0; s < kNSets; ++s) mbar_init(tfull_bar(s), 4);
     for (int a = 0; a < NACC; ++a) { mbar_init(accf_bar(a), 1); mbar_init(acce_bar(a), 4); }
     mbar_init(drain_bar, 1);
+    mbar_init(never_bar, 1);
     ctl->abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -615,6 +626,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
     for (int j = 0; j < n_my && !*abort_flag; ++j) {
       const TileDesc c = my_tile(j, ttab, p.tcap, pref, offs, E, kBN, p.sched, tb);
       const uint32_t idesc = make_idesc(kSparse, (c.valid + 15) & ~15);
+      if (p.stall_ns != 0ull && j == (n_my > 1 ? 1 : 0) &&
+          !wait_warp(never_bar, 0u, abort_flag, p.status, p.stall_ns))
+        break;
       if (!wait_warp(acce_bar(acc), aph ^ 1u, abort_flag, p.status)) break;
       tc_fence_after();
       const uint32_t d_tmem = tmem + kColAcc + (uint32_t)(acc * G::kNT * G::kAccStride);
@@ -778,12 +792,17 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
           // combine: lane j < 16 holds the flat index f = t*k + j of chunk row j; the row goes to
           // slot f instead of row r
           const bool comb = p.perm_src != nullptr;
-          const int myf = (comb && lane < 16 && c0 + lane < valid) ? __ldg(p.perm_src + r0 + c0 + lane) : 0;
+          int myf = (comb && lane < 16 && c0 + lane < valid) ? __ldg(p.perm_src + r0 + c0 + lane) : 0;
+          // a slot index outside [0, T*k) (corrupt routing) gets nothing stored or counted
+          const unsigned badf = __ballot_sync(0xffffffffu, comb && lane < 16 && c0 + lane < valid &&
+                                                               (myf < 0 || myf >= p.R));
+          if (badf != 0u && lane == 0) set_status(p.status, GSG_ERR_BAD_ROUTING);
+          if ((badf >> lane) & 1u) myf = 0;
 #pragma unroll
           for (int k = 0; k < 2; ++k) {          // 16 tokens x 4 chunks of 16 B
             const int ci = lane + 32 * k, tok = ci >> 2, part = ci & 3;
             const int f = __shfl_sync(0xffffffffu, myf, tok);
-            if (c0 + tok < valid) {
+            if (c0 + tok < valid && !((badf >> tok) & 1u)) {
               uint32_t a, b, cc, d;
               lds128(obuf_s + (uint32_t)(tok * 64 + part * 16), a, b, cc, d);
               const size_t dst = comb ? (size_t)f : (size_t)(r0 + c0 + tok);
@@ -798,7 +817,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
             __syncwarp();
             const int g32 = (int)(col0 >> 5), ng32 = p.N >> 5;
             bool last = false;
-            if (lane < 16 && c0 + lane < valid) {
+            if (lane < 16 && c0 + lane < valid && !((badf >> lane) & 1u)) {
               const int t = myf / p.k;
               last = atomicAdd(p.counters + (size_t)t * ng32 + g32, 1) == p.k - 1;
             }
@@ -872,7 +891,7 @@ static GemmPlan make_plan(bool sparse, int BN, int E, int tcap, bool glu = false
   g.stage = (body + 1023) / 1024 * 1024;
   // everything but the stage ring and the tile table, at its largest
   const int ostage = 4 * (glu ? kGluStageBytes : kOutStageBytes);
-  const int fixed = 1024 + (2 * kMaxStages + kNSets + 2 * kMaxAcc + 1) * 8 + (int)sizeof(Ctl) + (3 * E + 2) * 4 +
+  const int fixed = 1024 + (2 * kMaxStages + kNSets + 2 * kMaxAcc + 2) * 8 + (int)sizeof(Ctl) + (3 * E + 2) * 4 +
                     16 + (E + 1) * 8 + 16 + ostage;
   int budget = g_smem_limit - fixed;
   if (BN == 128 && budget > kStageBudget128) budget = kStageBudget128;
@@ -881,7 +900,7 @@ static GemmPlan make_plan(bool sparse, int BN, int E, int tcap, bool glu = false
   const int acc_stride = (BN < 32 ? 32 : BN) * nt;
   g.nacc = (int)((kTmemCols - kColAcc) / acc_stride);
   if (g.nacc > kMaxAcc) g.nacc = kMaxAcc;
-  const int nbars = 2 * g.stages + kNSets + 2 * g.nacc + 1;
+  const int nbars = 2 * g.stages + kNSets + 2 * g.nacc + 2;
   g.smem = 1024 + (size_t)g.stages * g.stage + nbars * 8 + sizeof(Ctl) + (size_t)(3 * E + 2) * 4 + 16 +
            (size_t)(E + 1) * 8 + 16 +
            (size_t)tcap * 16 + ostage;
@@ -889,6 +908,10 @@ static GemmPlan make_plan(bool sparse, int BN, int E, int tcap, bool glu = false
 }
 
 constexpr int kMaxTableTiles = 1024;
+
+// test hook: the MMA warp's stall of GemmParams::stall_ns for the launches that follow (0 = off)
+static std::atomic<unsigned long long> g_test_stall_ns{0ull};
+void gemm_set_test_stall(unsigned long long ns) { g_test_stall_ns.store(ns); }
 
 // Token tile: the smallest of 16/32/64 that holds the largest expert; past 64 rows, 128 only when
 // experts average at least 64 rows (R / E), since a 128-row activation chunk takes shared memory
@@ -1033,6 +1056,7 @@ int launch_gemm(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, co
   p.counters = comb ? comb->counters : nullptr;
   p.out = comb ? comb->out : nullptr;
   p.k = comb ? comb->k : 1;
+  p.stall_ns = g_test_stall_ns.load();
   const cudaError_t e = sparse ? launch_bn<true>(g.BN, num_sms, g.smem, stream, tb, tb64, ts, p, glu)
                                : launch_bn<false>(g.BN, num_sms, g.smem, stream, tb, tb64, ts, p, false);
   return e == cudaSuccess ? 0 : 1;

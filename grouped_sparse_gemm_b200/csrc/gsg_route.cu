@@ -94,6 +94,8 @@ __device__ __forceinline__ void warp_scatter(const int x[kPer], const unsigned m
       const int pos = base[x[i]] + __popc(m[i] & lt);
       perm_src[pos] = f;
       inv_perm[f] = pos;
+    } else if (f < f1) {
+      inv_perm[f] = -1;   // a pair with an out-of-range id has no row: later kernels skip it
     }
     __syncwarp();
     if (x[i] >= 0 && lane == __ffs(m[i]) - 1) base[x[i]] += __popc(m[i]);

@@ -113,8 +113,9 @@ gsg_status_t gsg_pack_dense_nvfp4(const float* W, int E, int N, int K, uint8_t* 
  * counts run together; §D.1 (p.19): dispatch.  topk_ids int32 [T][k] in [0, E).
  * Routed pair (t, j) has flat index f = t*k + j.  Rows of expert e are [off[e], off[e+1]),
  * in ascending f.  Outputs: expert_offsets int32 [E+1], perm_src int32 [R] (row -> f),
- * inv_perm int32 [R] (f -> row).  Out-of-range ids set GSG_ERR_BAD_ROUTING (outputs then
- * unspecified).  Deterministic.
+ * inv_perm int32 [R] (f -> row).  Out-of-range ids set GSG_ERR_BAD_ROUTING: such a pair gets
+ * no row and inv_perm[f] = -1 (the quantizer and the scatter skip it); the offsets and the rows of
+ * the valid pairs are then unspecified.  Deterministic.
  */
 gsg_status_t gsg_moe_route_permute(const int32_t* topk_ids, int T, int k, int E,
                                    int32_t* expert_offsets, int32_t* perm_src, int32_t* inv_perm,
@@ -226,7 +227,8 @@ gsg_status_t gsg_grouped_sparse_gemm_swiglu(const uint8_t* a_codes, const uint8_
  *     out[t][n] = bf16_rne( sum_{j<k} fp32(gates[t][j] * slot[t*k + j][n]) )   (j ascending, from 0)
  * -- the scatter's arithmetic and order, so the result does not depend on which warp finishes
  * last.  R = T*k routed rows; perm_src int32 [R] and expert_offsets from gsg_moe_route_permute;
- * gates fp32 [T][k]; out bf16 [T][N].
+ * gates fp32 [T][k]; out bf16 [T][N].  A routed row whose perm_src entry lies outside [0, T*k)
+ * is skipped (nothing stored for it) and sets GSG_ERR_BAD_ROUTING.
  * workspace: gsg_workspace_size(GSG_OP_COMBINE, E, N, K, T, k) bytes, 16-byte aligned: the slots
  * bf16 [T*k][N] and then int32 completion counters [T][N/32].  The counters must be zero before
  * the first call (e.g. allocate the workspace zeroed); every call that completes leaves them zero
@@ -273,6 +275,18 @@ gsg_status_t gsg_unpermute_scale(const uint16_t* Y, const int32_t* inv_perm, con
 gsg_status_t gsg_moe_route_permute_noalloc(const int32_t* topk_ids, int T, int k, int E,
                                            int32_t* expert_offsets, int32_t* perm_src,
                                            int32_t* inv_perm, void* stream);
+
+/* ----------------------------------------------------------------------------------------
+ * gsg_test_set_gemm_stall_ns -- fault injection for tests of the device timeout path.  Not a step
+ * of the method: the paper has no counterpart.  ns > 0: every grouped GEMM launched afterwards
+ * (sparse, dense control, SwiGLU and combine epilogues) makes its MMA warp wait up to `ns`
+ * nanoseconds, before its second tile (its first if it has one), on an internal barrier that
+ * nothing arrives on.  The wait runs out; the launch sets GSG_ERR_DEVICE_TIMEOUT, waits for its
+ * own copies and tensor-core work, frees its tensor memory and returns, with its outputs
+ * unspecified -- exactly what happens when a real wait exceeds its 2 s limit.  ns = 0 (the
+ * default) switches the hook off.  Process-wide: set it only while no other thread launches.
+ */
+void gsg_test_set_gemm_stall_ns(unsigned long long ns);
 
 /* ----------------------------------------------------------------------------------------
  * Status.  gsg_get_device_status synchronizes `stream`, returns the device status word of the

@@ -52,7 +52,12 @@ def test_loader_rejects_wrong_sizes_and_versions(tmp_path):
              dict(K=512),                                     # shape that does not match the bytes
              dict(w_scale=np.zeros(2, dtype=np.float32)),     # one scale per expert
              dict(version=99),
-             dict(format="fp8")]
+             dict(format="fp8"),
+             dict(N=130),                                     # N not whole n-tiles, same byte count
+             dict(K=300),                                     # K not whole chunks, same byte count
+             dict(E=0, w_scale=np.zeros(0, dtype=np.float32)),
+             dict(E=-1),
+             dict(N=2 ** 40)]                                 # beyond int range
     for i, bad in enumerate(cases):
         p = tmp_path / f"bad{i}.npz"
         np.savez(p, **{**good, **bad})
