@@ -708,17 +708,20 @@ def run_ours(args, world, rank, local):
     cpu = None
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         smp = OracleSample(cfg, X_h, ids_h, cpu_sample_experts(cfg, args.cpu_experts))
-        dt, fl = smp.run(smp.units)
-        passes = 1
-        while dt < 10.0:          # repeat the same sample until about 10 s of CPU work
-            d2, f2 = smp.run(smp.units)
-            dt, fl, passes = dt + d2, fl + f2, passes + 1
+        # (expert, weight tile) units in a seeded order, one at a time, until about 12 s of CPU work
+        order = np.random.default_rng(5).permutation(len(smp.units))
+        dt, fl, done, rows = 0.0, 0.0, 0, 0
+        while dt < 12.0:
+            e, nt = smp.units[order[done % len(order)]]
+            d2, f2 = smp.run([(e, nt)])
+            dt, fl, done = dt + d2, fl + f2, done + 1
+            rows += int(smp.off[e + 1] - smp.off[e])
         cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
-               "sample": (f"{passes} passes of the oracle grouped GEMM (packed-weight and activation decode + fp64 "
-                          f"matmul) over all {cfg.N // 128} weight tiles of {len(smp.experts)} experts (the largest "
-                          f"half and seeded random others, "
-                          f"{int(sum(smp.off[e + 1] - smp.off[e] for e in smp.experts))} of {cfg.R} routed rows), "
-                          f"{dt:.1f} s in all; routing, quantization and packing untimed")}
+               "sample": (f"the oracle grouped GEMM (packed-weight and activation decode + fp64 matmul) of {done} "
+                          f"(expert, 128-row weight tile) units drawn in a seeded order from the "
+                          f"{len(smp.units)} units of {len(smp.experts)} experts (the largest half and seeded random "
+                          f"others), {rows} routed rows x 128 outputs x K={cfg.K} in all, {dt:.1f} s; routing, "
+                          f"quantization and packing untimed")}
 
     if rank == 0:
         line = {

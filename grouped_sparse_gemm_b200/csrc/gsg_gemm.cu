@@ -89,6 +89,32 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
+
+// ---- CTA pairs (thread-block clusters of two CTAs on two SMs; see kCG below)
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// The shared::cluster address of the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_addr(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+// Arrive on an mbarrier given by its shared::cluster address (a barrier of this CTA or of the
+// other CTA of the pair).  Default semantics (no cluster-scope release, which costs a fence per
+// arrive): what the arrive hands over is already complete when it is issued -- copies that landed
+// (their full barrier completed) and TMEM stores waited on with tcgen05.wait::st -- and is read
+// only by the leader's tensor-core work issued after the leader observed the phase.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cl_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cl_addr) : "memory");
+}
+// Every thread of both CTAs of the cluster: all earlier writes (barrier initialisation included)
+// are visible to the other CTA afterwards.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 // The issue wrappers below are executed by a whole converged warp: elect.sync picks one lane
 // and predicates the instruction on it, so the warp never diverges around a TMA or tcgen05
 // instruction (issuing them from a lone lane of a diverged warp costs several times more).
@@ -164,6 +190,14 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
                "@P tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
                : "memory");
 }
+// Pair form: once the pair's earlier tensor-core work has completed, arrive once on the barrier at
+// this shared-memory offset in every CTA of `mask` (bit r = CTA rank r).
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar, uint16_t mask) {
+  asm volatile("{\n\t.reg .pred P;\n\t" GSG_ELECT
+               "@P tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+               "\n\t}" ::"r"(bar), "h"(mask)
+               : "memory");
+}
 __device__ __forceinline__ void tc_mma_sparse(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                               uint32_t accumulate, uint32_t sfa, uint32_t sfb, uint32_t meta) {
   asm volatile(
@@ -179,6 +213,28 @@ __device__ __forceinline__ void tc_mma_dense(uint32_t d, uint64_t adesc, uint64_
       "{\n\t.reg .pred p, P;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t" GSG_ELECT
       "@P tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+// The same two MMAs issued for a CTA pair (M = 256: each CTA supplies its 128 weight rows and half
+// of the tile's token columns from its own shared memory at the same offsets, and holds its rows'
+// accumulator, metadata and scales -- the scales of all N token columns -- in its own TMEM at the
+// same addresses).
+__device__ __forceinline__ void tc_mma_sparse_pair(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                   uint32_t accumulate, uint32_t sfa, uint32_t sfb, uint32_t meta) {
+  asm volatile(
+      "{\n\t.reg .pred p, P;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t" GSG_ELECT
+      "@P tcgen05.mma.sp.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, [%7], %3, [%5], [%6], p;\n\t}" ::"r"(d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb), "r"(meta)
+      : "memory");
+}
+__device__ __forceinline__ void tc_mma_dense_pair(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                                  uint32_t accumulate, uint32_t sfa, uint32_t sfb) {
+  asm volatile(
+      "{\n\t.reg .pred p, P;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t" GSG_ELECT
+      "@P tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
       : "memory");
 }
@@ -203,9 +259,11 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
 }
 
 // Instruction descriptor of kind::mxf4nvf4 block-scaled MMA: A/B E2M1, UE4M3 scales,
-// K-major A and B, M = 128, N = BN; bit 2 marks the sparse form (K = 128 logical).
-__host__ __device__ inline uint32_t make_idesc(bool sparse, int BN) {
-  return (sparse ? (1u << 2) : 0u) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | ((128u >> 4) << 24);
+// K-major A and B, M = 128 (256 for a CTA pair), N = BN; bit 2 marks the sparse form (K = 128
+// logical).
+__host__ __device__ inline uint32_t make_idesc(bool sparse, int BN, int M = 128) {
+  return (sparse ? (1u << 2) : 0u) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
 }
 
 struct Ctl {
@@ -276,20 +334,22 @@ __device__ __forceinline__ TileDesc decode_tile(int t, const int* pref, const in
 constexpr int kSchedRoundRobin = 0;
 constexpr int kSchedRuns = 1;
 
-__device__ __forceinline__ int tile_of(int j, int sched, int tb) {
+// `unit` / `nunits`: this CTA's index and the number of CTAs, or for CTA pairs the pair's index
+// and the number of pairs (both CTAs of a pair take the same tiles).
+__device__ __forceinline__ int tile_of(int j, int sched, int tb, int unit, int nunits) {
   if (sched == kSchedRuns) return tb + j;
-  return j * (int)gridDim.x + (int)blockIdx.x;
+  return j * nunits + unit;
 }
 
 // The j-th tile of this CTA: from the shared-memory table filled at set-up, or decoded on the
 // spot past its capacity.
 __device__ __forceinline__ TileDesc my_tile(int j, const int4* table, int tcap, const int* pref, const int* offs,
-                                            int E, int BN, int sched, int tb) {
+                                            int E, int BN, int sched, int tb, int unit, int nunits) {
   if (j < tcap) {
     const int4 v = table[j];
     return TileDesc{v.x, v.y, v.z, v.w};
   }
-  return decode_tile(tile_of(j, sched, tb), pref, offs, E, BN);
+  return decode_tile(tile_of(j, sched, tb, unit, nunits), pref, offs, E, BN);
 }
 
 // Tile schedule: every CTA takes a contiguous run of tiles (expert-major, then n-tile, then token
@@ -316,11 +376,16 @@ __device__ __forceinline__ int tile_at_cost(long long target, const long long* c
   return pref[lo] + (int)(nt * mte + tt);
 }
 
-// Compile-time stage geometry of one (sparse/dense, token tile, SwiGLU) instantiation.  With the
-// SwiGLU epilogue a tile holds two weight n-tiles (gate rows nt*128.., up rows N/2 + nt*128..) that
-// share the activation tile: two MMAs per k-block into two accumulators side by side.
-template <bool kSparse, int kBN, bool kGLU = false>
+// Compile-time stage geometry of one (sparse/dense, token tile, SwiGLU, CTA group) instantiation.
+// With the SwiGLU epilogue a tile holds two weight n-tiles (gate rows nt*128.., up rows
+// N/2 + nt*128..) that share the activation tile: two MMAs per k-block into two accumulators side
+// by side.  With kCG = 2 a tile is 256 weight rows (n-tiles 2*np and 2*np + 1) x kBN tokens, run
+// by a pair of CTAs on two SMs: CTA r holds n-tile 2*np + r and half of the token rows, and the
+// pair's MMAs (M = 256) read both CTAs' shared memory, so each SM stages its own weights but only
+// half of the shared activation tile.
+template <bool kSparse, int kBN, bool kGLU = false, int kCG = 1>
 struct Geo {
+  static_assert(kCG == 1 || (kCG == 2 && !kGLU && kBN == 128), "CTA pairs: 128-token tiles, plain epilogue");
   static constexpr int kNT = kGLU ? 2 : 1;                         // weight n-tiles per tile
   static constexpr int kKbLogical = kSparse ? 128 : 64;            // logical K per MMA
   static constexpr int kKbPerChunk = kChunkK / kKbLogical;         // 2 sparse, 4 dense
@@ -330,7 +395,8 @@ struct Geo {
   static constexpr int kCB = kSparse ? kSparseChunkBytes : kDenseChunkBytes;   // packed chunk block
   static constexpr int kCBMeta = 8192;                             // metadata offset in a chunk block
   static constexpr int kCBScale = kSparse ? 10240 : 16384;         // scale atoms offset in a chunk block
-  static constexpr int kBChunk = kBN * 128;                        // activation codes per chunk
+  static constexpr int kBRows = kBN / kCG;                         // token rows this CTA stages
+  static constexpr int kBChunk = kBRows * 128;                     // activation codes per chunk
   static constexpr int kOffW = kCPS * kBChunk;                     // stage layout: B chunks | W blocks | SFB
   static constexpr int kOffSFB = kOffW + kNT * kCPS * kCB;
   static constexpr int kStage = (kOffSFB + kKbps * 512 + 1023) / 1024 * 1024;
@@ -339,20 +405,29 @@ struct Geo {
   static constexpr int kColSFB = kMetaCols + 4 * kKbps * kNT;
   static constexpr int kSetUsed = kColSFB + 4 * kKbps;
   static constexpr uint32_t kBStep = kSparse ? 64 : 32;            // B bytes per row per MMA
-  static constexpr int kBoxH = kBN < 32 ? kBN : 32;                // token rows per TMA box
+  static constexpr int kBoxH = kBRows < 32 ? kBRows : 32;          // token rows per TMA box
   static constexpr int kAccStride = kBN < 32 ? 32 : kBN;
   static_assert(kSetUsed <= (int)kSetCols, "TMEM set too small");
 };
 
-template <bool kSparse, int kBN, bool kGLU>
+// kCG = 2: launched as clusters of two CTAs (a CTA pair on two SMs) that run 256-row weight tiles
+// together; see Geo.  CTA rank 0 of the pair (the leader) issues the pair's MMAs and owns the
+// barriers the MMAs wait on (tfull, acce: arrived on by both CTAs' loader and epilogue warps);
+// every MMA completion is signalled to the barriers of both CTAs (empty, accf).
+template <bool kSparse, int kBN, bool kGLU, int kCG>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ CUtensorMap tmap_b64,
                     const __grid_constant__ CUtensorMap tmap_sfb,
                     const GemmParams p) {
-  using G = Geo<kSparse, kBN, kGLU>;
+  using G = Geo<kSparse, kBN, kGLU, kCG>;
+  constexpr bool kPair = kCG == 2;
   extern __shared__ uint8_t smem_raw[];
-  // NT: weight n-tiles; tiles run over NT / kNT columns (the gate n-tiles with the SwiGLU epilogue)
-  const int E = p.E, NT = p.N / kTileN, NTt = NT / G::kNT, KC = p.K / kChunkK;
+  // NT: weight n-tiles; tiles run over NT / (kNT * kCG) columns (the gate n-tiles with the SwiGLU
+  // epilogue, n-tile pairs for CTA pairs)
+  const int E = p.E, NT = p.N / kTileN, NTt = NT / (G::kNT * kCG), KC = p.K / kChunkK;
+  const uint32_t rank = kPair ? cluster_ctarank() : 0u;         // this CTA's rank in its pair
+  const int unit = kPair ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int nunits = kPair ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   const int S = p.stages, NACC = p.nacc;
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + (size_t)S * G::kStage);
@@ -389,8 +464,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) { mbar_init(full_bar(s), 2); mbar_init(empty_bar(s), 1); }
-    for (int s = 0; s < kNSets; ++s) mbar_init(tfull_bar(s), 4);
-    for (int a = 0; a < NACC; ++a) { mbar_init(accf_bar(a), 1); mbar_init(acce_bar(a), 4); }
+    for (int s = 0; s < kNSets; ++s) mbar_init(tfull_bar(s), 4 * kCG);
+    for (int a = 0; a < NACC; ++a) { mbar_init(accf_bar(a), 1); mbar_init(acce_bar(a), 4 * kCG); }
     mbar_init(drain_bar, 1);
     mbar_init(never_bar, 1);
     ctl->abort = 0;
@@ -398,10 +473,19 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&ctl->tmem_base)),
-                 "r"(kTmemCols)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    if constexpr (kPair) {   // the same columns in both CTAs of the pair (both warps 1 allocate)
+      asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(&ctl->tmem_base)),
+                   "r"(kTmemCols)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    } else {
+      asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                       smem_u32(&ctl->tmem_base)),
+                   "r"(kTmemCols)
+                   : "memory");
+      asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
   }
   pdl_wait();
   // expert offsets, clamped to [0, R] so a corrupt array can never send a copy or a store out
@@ -453,8 +537,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
     if (threadIdx.x == kGemmThreads - 1) pref[E] = before + incl;
   }
   // bytes per tile: weights wc, plus ac per token row (codes, scales, output row segment)
-  const long long wc = (long long)G::kNT * kTileN * p.K * (kSparse ? 11 : 18) / 32;
-  const long long ac = p.K / 2 + p.K / (kSparse ? 32 : 16) + (long long)G::kNT * kTileN * (p.y_f32 ? 4 : 2);
+  const long long wc = (long long)G::kNT * kCG * kTileN * p.K * (kSparse ? 11 : 18) / 32;
+  const long long ac = p.K / 2 + p.K / (kSparse ? 32 : 16) + (long long)G::kNT * kCG * kTileN * (p.y_f32 ? 4 : 2);
   {
     // chunked exclusive scan of cost_e = NTt * (ceil(rows_e / BN) * wc + rows_e * ac)
     const int per = (E + kGemmThreads - 1) / kGemmThreads;
@@ -486,7 +570,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
   __syncthreads();
   const int total_tiles = pref[E];
   if (threadIdx.x == 0) {
-    const int b = (int)blockIdx.x, G_ = (int)gridDim.x;
+    const int b = unit, G_ = nunits;
     if (p.sched == kSchedRuns) {
       const long long C = costp[E];
       const int tb = tile_at_cost(C * b / G_, costp, pref, offs, E, kBN, wc, ac);
@@ -503,11 +587,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
   // this CTA's tiles, decoded once
   const int n_my = ctl->tile_end - tb;
   for (int j = threadIdx.x; j < n_my && j < p.tcap; j += blockDim.x) {
-    const TileDesc d = decode_tile(tile_of(j, p.sched, tb), pref, offs, E, kBN);
+    const TileDesc d = decode_tile(tile_of(j, p.sched, tb, unit, nunits), pref, offs, E, kBN);
     ttab[j] = make_int4(d.e, d.nt, d.r0, d.valid);
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (kPair) {
+    cluster_sync_all();   // both CTAs' barriers initialised before either arrives on the other's
+  } else {
+    __syncthreads();
+  }
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_base;
 
@@ -517,14 +605,18 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
     int s = 0, issued = 0;
     uint32_t ph = 0;
     for (int j = 0; j < n_my && !*abort_flag; ++j) {
-      const TileDesc c = my_tile(j, ttab, p.tcap, pref, offs, E, kBN, p.sched, tb);
-      const uint8_t* wsrc = p.w_packed + ((size_t)c.e * NT + c.nt) * KC * G::kCB;
+      const TileDesc c = my_tile(j, ttab, p.tcap, pref, offs, E, kBN, p.sched, tb, unit, nunits);
+      const uint8_t* wsrc = p.w_packed + ((size_t)c.e * NT + c.nt * kCG + rank) * KC * G::kCB;
       const uint8_t* wsrc_up = wsrc + (size_t)(NT / 2) * KC * G::kCB;   // SwiGLU: the matching up n-tile
-      const int r0 = c.r0;
+      // this CTA's token rows [r0, r0 + cnt): all of the tile's, or for a CTA pair the half of the
+      // MMA's N = valid rounded up to 16 that this CTA supplies (rank 1: the upper half)
+      const int nh = kPair ? ((c.valid + 15) & ~15) / 2 : kBN;
+      const int r0 = c.r0 + (int)rank * nh;
+      const int cnt = min(max(c.valid - (int)rank * nh, 0), nh);
       // token rows to fetch: whole 32-row boxes (BN <= 32: one box of BN rows), as few 64-row
       // boxes as possible for the larger tiles -- every TMA instruction costs the issuing warp
-      const int rows = (c.valid + G::kBoxH - 1) / G::kBoxH * G::kBoxH;
-      const int n64 = kBN >= 64 ? rows / 64 : 0;
+      const int rows = (cnt + G::kBoxH - 1) / G::kBoxH * G::kBoxH;
+      const int n64 = G::kBRows >= 64 ? rows / 64 : 0;
       const int n32 = (rows - 64 * n64) / G::kBoxH;
       bool ok = true;
       for (int kc = 0; kc < KC; kc += G::kCPS) {
@@ -534,11 +626,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
         const uint32_t fb = full_bar(s);
         if (wprod) {
           // weights (+ metadata + weight scales) and the activation scale atoms: the activation
-          // producer issues one TMA per box already
+          // producer issues one TMA per box already.  The scale atoms cover the whole tile's
+          // tokens from its first row (in both CTAs of a pair: each CTA's MMA share needs the
+          // scales of all N token columns).
           mbar_arrive_expect_tx(fb, (uint32_t)(G::kNT * nch * G::kCB + G::kKbps * 512));
           bulk_g2s(st + G::kOffW, wsrc + (size_t)kc * G::kCB, nch * G::kCB, fb);
           if (kGLU) bulk_g2s(st + G::kOffW + G::kCPS * G::kCB, wsrc_up + (size_t)kc * G::kCB, nch * G::kCB, fb);
-          tma_load_3d(st + G::kOffSFB, &tmap_sfb, 0, r0, kc * G::kKbPerChunk, fb);
+          tma_load_3d(st + G::kOffSFB, &tmap_sfb, 0, c.r0, kc * G::kKbPerChunk, fb);
         } else {
           mbar_arrive_expect_tx(fb, (uint32_t)(nch * rows * 128));
           for (int ch = 0; ch < nch; ++ch) {
@@ -577,7 +671,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
         // the TMEM set is free once the MMAs of the stage that last used it have completed
         if (i >= kNSets) {
           const int j = i - kNSets;
-          if (!wait_warp(empty_bar(j % S), (uint32_t)(j / S) & 1u, abort_flag, p.status)) { ok = false; break; }
+          if (!wait_warp(empty_bar(j % S), (uint32_t)(j / S) & 1u, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
         }
         if (!wait_warp(full_bar(s), ph, abort_flag, p.status)) { ok = false; break; }
         const uint32_t st = sbase + (uint32_t)s * G::kStage;
@@ -611,7 +708,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
         tc_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(tfull_bar(set));
+        if (lane == 0) {   // the set (and, for a pair, this CTA's stage) is ready for the MMA issuer
+          if constexpr (kPair) mbar_arrive_cluster(cluster_addr(tfull_bar(set), 0u));
+          else mbar_arrive(tfull_bar(set));
+        }
         ++i;
         if (++set == kNSets) set = 0;
         if (++s == S) { s = 0; ph ^= 1u; }
@@ -619,14 +719,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
       if (!ok) break;
     }
   } else if (warp == 1) {
-    // =============================== MMA issuer (whole warp, one elected lane issues)
+    // =============================== MMA issuer (whole warp, one elected lane issues); for a CTA
+    // pair only the leader's, whose MMAs run on both SMs (the other CTA's warp 1 has no tiles)
     int s = 0, set = 0, i = 0, acc = 0;
     uint32_t ph = 0, aph = 0;   // ring phase, accumulator phase
     bool any = false;
-    for (int j = 0; j < n_my && !*abort_flag; ++j) {
-      const TileDesc c = my_tile(j, ttab, p.tcap, pref, offs, E, kBN, p.sched, tb);
-      const uint32_t idesc = make_idesc(kSparse, (c.valid + 15) & ~15);
-      if (p.stall_ns != 0ull && j == (n_my > 1 ? 1 : 0) &&
+    const int n_mma = rank == 0u ? n_my : 0;
+    for (int j = 0; j < n_mma && !*abort_flag; ++j) {
+      const TileDesc c = my_tile(j, ttab, p.tcap, pref, offs, E, kBN, p.sched, tb, unit, nunits);
+      const uint32_t idesc = make_idesc(kSparse, (c.valid + 15) & ~15, kTileN * kCG);
+      if (p.stall_ns != 0ull && j == (n_mma > 1 ? 1 : 0) &&
           !wait_warp(never_bar, 0u, abort_flag, p.status, p.stall_ns))
         break;
       if (!wait_warp(acce_bar(acc), aph ^ 1u, abort_flag, p.status)) break;
@@ -657,30 +759,36 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
                     smem_desc(st + G::kOffW + (t * G::kCPS + ch) * G::kCB + 4096u * h, 128, 256, 0);
                 const uint32_t d = d_tmem + (uint32_t)(t * G::kAccStride);
                 const int kt = t * G::kKbps + kbi;
-                if (kSparse)
-                  tc_mma_sparse(d, adesc, bdesc, idesc, accum, tset + G::kColSFA + 4 * kt,
-                                tset + G::kColSFB + 4 * kbi, tset + 2 * kt);
+                const uint32_t sfa = tset + G::kColSFA + 4 * kt, sfb = tset + G::kColSFB + 4 * kbi;
+                if constexpr (kSparse && kPair)
+                  tc_mma_sparse_pair(d, adesc, bdesc, idesc, accum, sfa, sfb, tset + 2 * kt);
+                else if constexpr (kSparse)
+                  tc_mma_sparse(d, adesc, bdesc, idesc, accum, sfa, sfb, tset + 2 * kt);
+                else if constexpr (kPair)
+                  tc_mma_dense_pair(d, adesc, bdesc, idesc, accum, sfa, sfb);
                 else
-                  tc_mma_dense(d, adesc, bdesc, idesc, accum, tset + G::kColSFA + 4 * kt,
-                               tset + G::kColSFB + 4 * kbi);
+                  tc_mma_dense(d, adesc, bdesc, idesc, accum, sfa, sfb);
               }
             }
           }
         }
-        tc_commit(empty_bar(s));
+        if constexpr (kPair) tc_commit_pair(empty_bar(s), 3);   // the stage is free in both CTAs
+        else tc_commit(empty_bar(s));
         any = true;
         ++i;
         if (++set == kNSets) set = 0;
         if (++s == S) { s = 0; ph ^= 1u; }
       }
       if (!ok) break;
-      tc_commit(accf_bar(acc));
+      if constexpr (kPair) tc_commit_pair(accf_bar(acc), 3);   // both CTAs' epilogues
+      else tc_commit(accf_bar(acc));
       if (++acc == NACC) { acc = 0; aph ^= 1u; }
     }
     __syncwarp();
     if (any) {
       // all MMAs issued by this warp have completed once the drain barrier fires
-      tc_commit(drain_bar);
+      if constexpr (kPair) tc_commit_pair(drain_bar, 1);
+      else tc_commit(drain_bar);
       const uint64_t t0 = globaltimer_ns();
       while (!mbar_try_wait(drain_bar, 0) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
       }
@@ -692,7 +800,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
     int acc = 0;
     uint32_t aph = 0;
     for (int j = 0; j < n_my; ++j) {
-      const TileDesc c = my_tile(j, ttab, p.tcap, pref, offs, E, kBN, p.sched, tb);
+      const TileDesc c = my_tile(j, ttab, p.tcap, pref, offs, E, kBN, p.sched, tb, unit, nunits);
       const int r0 = c.r0, valid = c.valid;
       if (!wait_warp(accf_bar(acc), aph, abort_flag, p.status)) break;
       tc_fence_after();
@@ -762,7 +870,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
       // segments (64 B bf16 / 128 B fp32 per token).
       uint8_t* obuf = ostage + (size_t)(warp - 3) * kOutStageBytes;
       const uint32_t obuf_s = smem_u32(obuf);
-      const size_t col0 = (size_t)c.nt * kTileN + 32 * q;       // first feature of this warp
+      const size_t col0 = ((size_t)c.nt * kCG + rank) * kTileN + 32 * q;   // first feature of this warp
       for (int c0 = 0; c0 < valid; c0 += 16) {
         float v[16];
         tc_ld_16(taddr + c0, v);
@@ -853,17 +961,30 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(acce_bar(acc));
+      if (lane == 0) {   // the accumulator may be overwritten (for a pair: once both CTAs read it)
+        if constexpr (kPair) mbar_arrive_cluster(cluster_addr(acce_bar(acc), 0u));
+        else mbar_arrive(acce_bar(acc));
+      }
       if (++acc == NACC) { acc = 0; aph ^= 1u; }
     }
   }
 
-  // ---- teardown
+  // ---- teardown (a CTA of a pair leaves only once the other is done with its shared memory and
+  // barriers: the leader's MMAs read both CTAs' stages, and both CTAs arrive on the leader's
+  // barriers)
   tc_fence_before();
-  __syncthreads();
+  if constexpr (kPair) {
+    __syncwarp();          // the cluster barrier is executed by converged warps
+    cluster_sync_all();
+  } else {
+    __syncthreads();
+  }
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    if constexpr (kPair)
+      asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+    else
+      asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
   }
 }
 
@@ -879,22 +1000,24 @@ constexpr int kStageBudget128 = 192 * 1024;   // 128-token tiles: a deeper ring 
 static int g_smem_limit = 232448 - 1024;
 
 // tcap: capacity of the per-CTA tile table (tiles beyond it are decoded on the fly); an upper
-// bound on a CTA's tiles is ceil((ceil(R/BN) + E) * NT / grid).
-static GemmPlan make_plan(bool sparse, int BN, int E, int tcap, bool glu = false) {
+// bound on a CTA's tiles is ceil((ceil(R/BN) + E) * NT / grid).  cg = 2: a CTA of a pair, which
+// stages half of the tile's token rows (the geometry of Geo<..., 2>).
+static GemmPlan make_plan(bool sparse, int BN, int E, int tcap, bool glu = false, int cg = 1) {
   GemmPlan g;
   g.BN = BN;
   g.tcap = tcap;
   const int nt = glu ? 2 : 1;   // weight n-tiles per tile (gate + up with the SwiGLU epilogue)
   g.cps = glu ? 2 : sparse ? (BN <= 32 ? 3 : 2) : (BN <= 32 ? 2 : 1);
   const int kbps = g.cps * (sparse ? 2 : 4);
-  const int body = g.cps * BN * 128 + nt * g.cps * (sparse ? kSparseChunkBytes : kDenseChunkBytes) + kbps * 512;
+  const int body =
+      g.cps * (BN / cg) * 128 + nt * g.cps * (sparse ? kSparseChunkBytes : kDenseChunkBytes) + kbps * 512;
   g.stage = (body + 1023) / 1024 * 1024;
   // everything but the stage ring and the tile table, at its largest
   const int ostage = 4 * (glu ? kGluStageBytes : kOutStageBytes);
   const int fixed = 1024 + (2 * kMaxStages + kNSets + 2 * kMaxAcc + 2) * 8 + (int)sizeof(Ctl) + (3 * E + 2) * 4 +
                     16 + (E + 1) * 8 + 16 + ostage;
   int budget = g_smem_limit - fixed;
-  if (BN == 128 && budget > kStageBudget128) budget = kStageBudget128;
+  if (BN == 128 && cg == 1 && budget > kStageBudget128) budget = kStageBudget128;
   g.stages = (budget - tcap * 16) / g.stage;
   if (g.stages > kMaxStages) g.stages = kMaxStages;
   const int acc_stride = (BN < 32 ? 32 : BN) * nt;
@@ -941,10 +1064,35 @@ static EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-template <bool kSparse, int kBN, bool kGLU = false>
+template <bool kSparse, int kBN, bool kGLU = false, int kCG = 1>
 static cudaError_t set_attr_one(int bytes) {
-  return cudaFuncSetAttribute(grouped_gemm_kernel<kSparse, kBN, kGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              bytes);
+  return cudaFuncSetAttribute(grouped_gemm_kernel<kSparse, kBN, kGLU, kCG>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+// CTA pairs the device can hold at once at one CTA per SM (the pairs' SMs must share a GPC), per
+// sparse/dense; 0 when the device cannot run them (then 128-token tiles run one CTA per tile).
+static int g_pair_units[2] = {0, 0};
+
+template <bool kSparse>
+static int max_pairs(int smem) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_kernel<kSparse, 128, false, 2>, &cfg) != cudaSuccess) {
+    cudaGetLastError();   // clear the error: pairs are then simply not used
+    return 0;
+  }
+  return n;
 }
 
 cudaError_t gemm_set_smem_attrs() {
@@ -955,14 +1103,17 @@ cudaError_t gemm_set_smem_attrs() {
   if (e != cudaSuccess) return e;
   maxb -= 1024;   // room for the kernels' static shared memory
   g_smem_limit = maxb;
-  cudaError_t errs[11] = {set_attr_one<true, 16>(maxb),       set_attr_one<true, 32>(maxb),
+  cudaError_t errs[13] = {set_attr_one<true, 16>(maxb),       set_attr_one<true, 32>(maxb),
                           set_attr_one<true, 64>(maxb),       set_attr_one<true, 128>(maxb),
                           set_attr_one<false, 16>(maxb),      set_attr_one<false, 32>(maxb),
                           set_attr_one<false, 64>(maxb),      set_attr_one<false, 128>(maxb),
                           set_attr_one<true, 16, true>(maxb), set_attr_one<true, 32, true>(maxb),
-                          set_attr_one<true, 64, true>(maxb)};
+                          set_attr_one<true, 64, true>(maxb), set_attr_one<true, 128, false, 2>(maxb),
+                          set_attr_one<false, 128, false, 2>(maxb)};
   for (cudaError_t x : errs)
     if (x != cudaSuccess) return x;
+  g_pair_units[1] = max_pairs<true>(maxb);
+  g_pair_units[0] = max_pairs<false>(maxb);
   return cudaSuccess;
 }
 
@@ -970,18 +1121,22 @@ template <bool kSparse, bool kGLU = false>
 static cudaError_t launch_bn(int BN, int grid, size_t smem, cudaStream_t stream, const CUtensorMap& tb,
                              const CUtensorMap& tb64, const CUtensorMap& ts, const GemmParams& p) {
   switch (BN) {
-    case 16: return launch_pdl(grouped_gemm_kernel<kSparse, 16, kGLU>, grid, kGemmThreads, smem, stream, tb, tb64, ts, p);
-    case 32: return launch_pdl(grouped_gemm_kernel<kSparse, 32, kGLU>, grid, kGemmThreads, smem, stream, tb, tb64, ts, p);
-    default: return launch_pdl(grouped_gemm_kernel<kSparse, 64, kGLU>, grid, kGemmThreads, smem, stream, tb, tb64, ts, p);
+    case 16: return launch_pdl(grouped_gemm_kernel<kSparse, 16, kGLU, 1>, grid, kGemmThreads, smem, stream, tb, tb64, ts, p);
+    case 32: return launch_pdl(grouped_gemm_kernel<kSparse, 32, kGLU, 1>, grid, kGemmThreads, smem, stream, tb, tb64, ts, p);
+    default: return launch_pdl(grouped_gemm_kernel<kSparse, 64, kGLU, 1>, grid, kGemmThreads, smem, stream, tb, tb64, ts, p);
   }
 }
 
 template <bool kSparse>
 static cudaError_t launch_bn(int BN, int grid, size_t smem, cudaStream_t stream, const CUtensorMap& tb,
-                             const CUtensorMap& tb64, const CUtensorMap& ts, const GemmParams& p, bool glu) {
+                             const CUtensorMap& tb64, const CUtensorMap& ts, const GemmParams& p, bool glu,
+                             bool pair) {
   if (glu) return launch_bn<true, true>(BN, grid, smem, stream, tb, tb64, ts, p);
+  if (BN == 128 && pair)
+    return launch_pdl_cluster(grouped_gemm_kernel<kSparse, 128, false, 2>, grid, kGemmThreads, smem, stream, 2u, tb,
+                              tb64, ts, p);
   if (BN == 128)
-    return launch_pdl(grouped_gemm_kernel<kSparse, 128, false>, grid, kGemmThreads, smem, stream, tb, tb64, ts, p);
+    return launch_pdl(grouped_gemm_kernel<kSparse, 128, false, 1>, grid, kGemmThreads, smem, stream, tb, tb64, ts, p);
   return launch_bn<kSparse, false>(BN, grid, smem, stream, tb, tb64, ts, p);
 }
 
@@ -997,34 +1152,41 @@ int launch_gemm(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, co
   const bool glu = h_scales != nullptr;
   int BN = gemm_pick_bn(max_rows, R, E);
   if (glu && BN > 64) BN = 64;   // two accumulators per tile: 64-token tiles at most
-  const long long bound = (((long long)R + BN - 1) / BN + E) * (N / kTileN / (glu ? 2 : 1));
+  // 128-token tiles run as CTA pairs (256 weight rows per tile) when N holds whole n-tile pairs
+  // and the device can co-schedule pairs
+  const int pair_units = g_pair_units[sparse ? 1 : 0];
+  const bool pair = BN == 128 && !glu && (N / kTileN) % 2 == 0 && pair_units > 0;
+  const int cg = pair ? 2 : 1;
+  const int units = pair ? (pair_units < num_sms / 2 ? pair_units : num_sms / 2) : num_sms;   // pairs or CTAs
+  const int grid = units * cg;
+  const long long bound = (((long long)R + BN - 1) / BN + E) * (N / kTileN / (glu ? 2 : 1) / cg);
   // schedule: contiguous byte-balanced runs when every expert fits one token tile (max_rows known)
   // and the CTAs can hold at least 32 tiles each (at most min(E, R) experts are touched), else
   // round-robin
-  const int NTt = N / kTileN / (glu ? 2 : 1);
+  const int NTt = N / kTileN / (glu ? 2 : 1) / cg;
   const long long touched_max = R < E ? R : E;
-  const int sched = (max_rows > 0 && max_rows <= BN && touched_max * NTt >= 32LL * num_sms) ? kSchedRuns
-                                                                                             : kSchedRoundRobin;
+  const int sched = (!pair && max_rows > 0 && max_rows <= BN && touched_max * NTt >= 32LL * units) ? kSchedRuns
+                                                                                                  : kSchedRoundRobin;
   long long tcap;
   if (sched == kSchedRuns) {
     // a CTA's share of the bytes holds at most (wc + BN ac) / (wc + ac) times the average tile count
     const long long wc = (glu ? 2LL : 1LL) * kTileN * K * (sparse ? 11 : 18) / 32;
     const long long ac = K / 2 + K / (sparse ? 32 : 16) + (glu ? 2LL : 1LL) * kTileN * (y_f32 ? 4 : 2);
-    tcap = (bound * (wc + BN * ac) / (wc + ac) + num_sms - 1) / num_sms + 2;
+    tcap = (bound * (wc + BN * ac) / (wc + ac) + units - 1) / units + 2;
   } else {
-    tcap = (bound + num_sms - 1) / num_sms;
+    tcap = (bound + units - 1) / units;
   }
   if (tcap > kMaxTableTiles) tcap = kMaxTableTiles;
-  const GemmPlan g = make_plan(sparse, BN, E, (int)tcap, glu);
+  const GemmPlan g = make_plan(sparse, BN, E, (int)tcap, glu, cg);
   if (g.stages < kNSets || g.smem > (size_t)g_smem_limit) return 1;   // ring too shallow: refuse, launch nothing
-  const int box_h = g.BN < 32 ? g.BN : 32;
+  const int box_h = g.BN / cg < 32 ? g.BN / cg : 32;
   const int kbps = g.cps * (sparse ? 2 : 4);
   const int rcap = R + kActScalePadRows;
   const int KBa = K / (sparse ? 128 : 64);
   CUtensorMap tb, tb64, ts;
   // activation codes [R][K/2]: boxes of 128 bytes x box_h rows, and (token tiles >= 64) x 64 rows
   for (int m = 0; m < 2; ++m) {
-    if (m == 1 && g.BN < 64) { tb64 = tb; break; }
+    if (m == 1 && g.BN / cg < 64) { tb64 = tb; break; }
     cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)R};
     cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
     cuuint32_t box[2] = {128u, (cuuint32_t)(m == 0 ? box_h : 64)};
@@ -1057,8 +1219,8 @@ int launch_gemm(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, co
   p.out = comb ? comb->out : nullptr;
   p.k = comb ? comb->k : 1;
   p.stall_ns = g_test_stall_ns.load();
-  const cudaError_t e = sparse ? launch_bn<true>(g.BN, num_sms, g.smem, stream, tb, tb64, ts, p, glu)
-                               : launch_bn<false>(g.BN, num_sms, g.smem, stream, tb, tb64, ts, p, false);
+  const cudaError_t e = sparse ? launch_bn<true>(g.BN, grid, g.smem, stream, tb, tb64, ts, p, glu, pair)
+                               : launch_bn<false>(g.BN, grid, g.smem, stream, tb, tb64, ts, p, false, pair);
   return e == cudaSuccess ? 0 : 1;
 }
 

@@ -292,7 +292,11 @@ GEMM_CASES = [
     ([16], 128, 256),                              # one tile
     ([5, 0, 33], 256, 512),                        # ragged, an empty expert, two n-tiles
     ([0, 1, 7, 8, 9, 127, 128, 129], 128, 768),    # the ragged-tail ladder
-    ([300, 2, 64], 384, 1024),
+    ([300, 2, 64], 384, 1024),                     # 128-token tiles, an odd n-tile count: one CTA per tile
+    # 128-token tiles run by CTA pairs (256 weight rows per tile, each CTA half of the tokens): tiles
+    # whose second CTA gets no rows (8, 1), one row (17), a partial half (100 -> N = 112), exactly
+    # half (64, 128) and every ragged edge around them
+    ([1, 8, 9, 16, 17, 56, 57, 63, 64, 65, 100, 127, 128, 129, 255, 256, 257, 0, 300], 512, 512),
 ]
 
 
@@ -349,14 +353,15 @@ def test_gemm_flags_corrupt_offsets(gsg):
     tl.assert_gemm_close(y[:10], y_ref, bound, "expert 0 beside corrupt offsets")
 
 
-@pytest.mark.parametrize("sparse", [True, False])
-def test_gemm_wait_timeout_aborts_cleanly(gsg, sparse):
+@pytest.mark.parametrize("sparse,counts", [(True, [40, 3, 77, 130, 0, 9]), (False, [40, 3, 77, 130, 0, 9]),
+                                           (True, [300, 130, 0, 9]), (False, [300, 130, 0, 9])])
+def test_gemm_wait_timeout_aborts_cleanly(gsg, sparse, counts):
     """Failure detection: the test hook makes the MMA warp wait on a barrier that nothing
     arrives on, with a 1 ms limit.  The launch must come back (no hang) with
     GSG_ERR_DEVICE_TIMEOUT in the status word after draining its own copies and tensor-core work
     and freeing its tensor memory; the next normal launch on the same context is correct."""
     import time
-    c = _gemm_case([40, 3, 77, 130, 0, 9], 256, 512, sparse=sparse)
+    c = _gemm_case(counts, 256, 512, sparse=sparse)   # 64-token tiles; 128-token tiles on CTA pairs
     L = gsg.lib()
     try:
         L.gsg_test_set_gemm_stall_ns(1_000_000)
