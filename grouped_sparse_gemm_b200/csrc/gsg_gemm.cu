@@ -8,10 +8,10 @@
 //
 // One CTA per SM, 352 threads (11 warps), warp-specialised around one shared-memory ring whose
 // stages hold 256 to 768 logical K of one tile (weights, activation codes and both scales):
-//   warp 0      weight producer: one bulk copy per stage of the interleaved packed weight blocks and
-//               one 3-D TMA box of the activation scale atoms.
+//   warp 0      weight producer: per stage one bulk copy per interleaved packed weight block and
+//               one 3-D TMA box of the activation scale atoms, each from its own lane.
 //   warp 2      activation producer: tensor-map TMA boxes (128B swizzle, 64 or 32 rows) of only the
-//               token rows the tile holds.
+//               token rows the tile holds, each from its own lane.
 //   warps 7..10 scale/metadata loaders, one per TMEM lane quadrant: read the stage's metadata and
 //               scale atoms from shared memory and tcgen05.st them into one of three TMEM sets.
 //   warp 1      TMEM owner and MMA issuer: per stage only tcgen05.mma(.sp) kind::mxf4nvf4
@@ -145,6 +145,34 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       "@P cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];\n\t}" ::
           "r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+// Per-lane forms: every lane of the (converged) warp executes the instruction and the lanes with
+// `on` set each issue their own copy.  The TMA unit works through the copies of one issuing thread
+// one after another, so the copies of a stage are spread over lanes to be in flight together.
+__device__ __forceinline__ void bulk_g2s_lane(bool on, uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred P;\n\tsetp.ne.b32 P, %4, 0;\n\t"
+      "@P cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n\t}" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar), "r"((uint32_t)on)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_2d_lane(bool on, uint32_t dst, const CUtensorMap* map, int x, int y,
+                                                 uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred P;\n\tsetp.ne.b32 P, %5, 0;\n\t"
+      "@P cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n\t}" ::
+          "r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "r"((uint32_t)on)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_lane(bool on, uint32_t dst, const CUtensorMap* map, int x, int y, int z,
+                                                 uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred P;\n\tsetp.ne.b32 P, %6, 0;\n\t"
+      "@P cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];\n\t}" ::
+          "r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar), "r"((uint32_t)on)
       : "memory");
 }
 __device__ __forceinline__ void lds128(uint32_t saddr, uint32_t& a, uint32_t& b, uint32_t& c, uint32_t& d) {
@@ -376,6 +404,13 @@ __device__ __forceinline__ int tile_at_cost(long long target, const long long* c
   return pref[lo] + (int)(nt * mte + tt);
 }
 
+// 256-wide K chunks per ring stage: short token tiles take longer stages (fewer waits per weight
+// byte); 128-token tiles keep two-chunk stages, also on CTA pairs (three-chunk stages, three of
+// them in shared memory, measured slower than five two-chunk stages).
+__host__ __device__ constexpr int stage_chunks(bool sparse, int BN, bool glu, int cg) {
+  return glu ? 2 : sparse ? (BN <= 32 ? 3 : 2) : (BN <= 32 ? 2 : 1);
+}
+
 // Compile-time stage geometry of one (sparse/dense, token tile, SwiGLU, CTA group) instantiation.
 // With the SwiGLU epilogue a tile holds two weight n-tiles (gate rows nt*128.., up rows
 // N/2 + nt*128..) that share the activation tile: two MMAs per k-block into two accumulators side
@@ -390,7 +425,7 @@ struct Geo {
   static constexpr int kKbLogical = kSparse ? 128 : 64;            // logical K per MMA
   static constexpr int kKbPerChunk = kChunkK / kKbLogical;         // 2 sparse, 4 dense
   // 256-wide K chunks per stage: short token tiles take longer stages (fewer waits per weight byte)
-  static constexpr int kCPS = kGLU ? 2 : kSparse ? (kBN <= 32 ? 3 : 2) : (kBN <= 32 ? 2 : 1);
+  static constexpr int kCPS = stage_chunks(kSparse, kBN, kGLU, kCG);
   static constexpr int kKbps = kCPS * kKbPerChunk;                 // k-blocks per stage
   static constexpr int kCB = kSparse ? kSparseChunkBytes : kDenseChunkBytes;   // packed chunk block
   static constexpr int kCBMeta = 8192;                             // metadata offset in a chunk block
@@ -600,9 +635,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
   const uint32_t tmem = ctl->tmem_base;
 
   if (warp == 0 || warp == 2) {
-    // =============================== producers: warp 0 weights, warp 2 activations
+    // =============================== producers: warp 0 weights, warp 2 activations.  The copies of
+    // a stage are issued from separate lanes (see bulk_g2s_lane): the TMA unit works through one
+    // thread's copies one after another, so one lane issuing every copy would keep a single copy
+    // in flight per producer.
     const bool wprod = warp == 0;
-    int s = 0, issued = 0;
+    int s = 0, g = 0;   // ring slot and stage counter
     uint32_t ph = 0;
     for (int j = 0; j < n_my && !*abort_flag; ++j) {
       const TileDesc c = my_tile(j, ttab, p.tcap, pref, offs, E, kBN, p.sched, tb, unit, nunits);
@@ -625,35 +663,36 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
         const uint32_t st = sbase + (uint32_t)s * G::kStage;
         const uint32_t fb = full_bar(s);
         if (wprod) {
-          // weights (+ metadata + weight scales) and the activation scale atoms: the activation
-          // producer issues one TMA per box already.  The scale atoms cover the whole tile's
-          // tokens from its first row (in both CTAs of a pair: each CTA's MMA share needs the
-          // scales of all N token columns).
+          // weights (+ metadata + weight scales): lane t * nch + ch copies chunk block ch of weight
+          // n-tile t (t = 1: the SwiGLU up n-tile); lane 31 copies the activation scale atoms of the
+          // whole tile's tokens from its first row (in both CTAs of a pair: each CTA's MMA share
+          // needs the scales of all N token columns)
           mbar_arrive_expect_tx(fb, (uint32_t)(G::kNT * nch * G::kCB + G::kKbps * 512));
-          bulk_g2s(st + G::kOffW, wsrc + (size_t)kc * G::kCB, nch * G::kCB, fb);
-          if (kGLU) bulk_g2s(st + G::kOffW + G::kCPS * G::kCB, wsrc_up + (size_t)kc * G::kCB, nch * G::kCB, fb);
-          tma_load_3d(st + G::kOffSFB, &tmap_sfb, 0, c.r0, kc * G::kKbPerChunk, fb);
+          const int t = lane / nch, ch = lane - t * nch;
+          bulk_g2s_lane(lane < G::kNT * nch, st + G::kOffW + (t * G::kCPS + ch) * G::kCB,
+                        (t == 0 ? wsrc : wsrc_up) + (size_t)(kc + ch) * G::kCB, G::kCB, fb);
+          tma_load_3d_lane(lane == 31, st + G::kOffSFB, &tmap_sfb, 0, c.r0, kc * G::kKbPerChunk, fb);
         } else {
+          // activation codes: lane ch * nb + b copies box b (64-row boxes first) of chunk ch
           mbar_arrive_expect_tx(fb, (uint32_t)(nch * rows * 128));
-          for (int ch = 0; ch < nch; ++ch) {
-            for (int b = 0; b < n64; ++b)
-              tma_load_2d(st + ch * G::kBChunk + b * 64 * 128, &tmap_b64, (kc + ch) * 128, r0 + b * 64, fb);
-            for (int b = 0; b < n32; ++b)
-              tma_load_2d(st + ch * G::kBChunk + (64 * n64 + b * G::kBoxH) * 128, &tmap_b, (kc + ch) * 128,
-                          r0 + 64 * n64 + b * G::kBoxH, fb);
-          }
+          const int nb = n64 + n32;
+          const int ch = nb > 0 ? lane / nb : 0, b = lane - ch * nb;
+          const bool b64 = b < n64;
+          const int roff = b64 ? 64 * b : 64 * n64 + (b - n64) * G::kBoxH;
+          tma_load_2d_lane(lane < nch * nb, st + ch * G::kBChunk + roff * 128, b64 ? &tmap_b64 : &tmap_b,
+                           (kc + ch) * 128, r0 + roff, fb);
         }
-        ++issued;
+        ++g;
         if (++s == S) { s = 0; ph ^= 1u; }
       }
       if (!ok) break;
     }
     if (*abort_flag && lane == 0) {
-      // wait (2 s in all) for copies still landing in the stages this warp filled
+      // wait (2 s in all) for copies still landing in the stages this warp filled: the last S
+      // before stage g (the first one it did not issue)
       const uint64_t t0 = globaltimer_ns();
-      for (int i = 0; i < S && i < issued; ++i) {
-        if (--s < 0) { s = S - 1; ph ^= 1u; }
-        while (!mbar_try_wait(full_bar(s), ph) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
+      for (int g2 = g > S ? g - S : 0; g2 < g; ++g2) {
+        while (!mbar_try_wait(full_bar(g2 % S), (uint32_t)(g2 / S) & 1u) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
         }
       }
     }
@@ -1007,7 +1046,7 @@ static GemmPlan make_plan(bool sparse, int BN, int E, int tcap, bool glu = false
   g.BN = BN;
   g.tcap = tcap;
   const int nt = glu ? 2 : 1;   // weight n-tiles per tile (gate + up with the SwiGLU epilogue)
-  g.cps = glu ? 2 : sparse ? (BN <= 32 ? 3 : 2) : (BN <= 32 ? 2 : 1);
+  g.cps = stage_chunks(sparse, BN, glu, cg);
   const int kbps = g.cps * (sparse ? 2 : 4);
   const int body =
       g.cps * (BN / cg) * 128 + nt * g.cps * (sparse ? kSparseChunkBytes : kDenseChunkBytes) + kbps * 512;
