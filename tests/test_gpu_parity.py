@@ -297,6 +297,9 @@ GEMM_CASES = [
     # whose second CTA gets no rows (8, 1), one row (17), a partial half (100 -> N = 112), exactly
     # half (64, 128) and every ragged edge around them
     ([1, 8, 9, 16, 17, 56, 57, 63, 64, 65, 100, 127, 128, 129, 255, 256, 257, 0, 300], 512, 512),
+    # the same pair tiles are 256 tokens in two 128-token halves: second halves of 8 (no rows on the
+    # second CTA), 17, 32, 64, 72 and 112 rows, and tiles after a full first tile
+    ([136, 145, 160, 192, 200, 240, 512, 520, 3], 256, 768),
 ]
 
 
