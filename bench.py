@@ -272,6 +272,9 @@ class Workload:
     def dense_gemm(self):
         gsg.grouped_dense_gemm(self.qa16, self.pd, self.route.offsets, self.max_rows, out=self.Yd)
 
+    def dense_gemm_native(self):
+        gsg.grouped_dense_gemm_native(self.qa16, self.pd, self.route.offsets, self.max_rows, out=self.Yd)
+
     # algorithmic bytes of one grouped GEMM launch
     def gemm_bytes(self):
         c = self.cfg
@@ -695,10 +698,18 @@ def run_ours(args, world, rank, local):
             dense_ms, _ = timed_graph_ms(gt_dense, max(10, args.steps // 2), flush, world)
         else:
             dense_ms, _ = timed_ms(capture(wl.dense_gemm).replay, max(10, args.steps // 2), flush, world)
-        control = {"kernel": "dense-NVFP4 grouped GEMM (16-element UE4M3 blocks, 4.5 bit/weight), same skeleton",
+        gt_native = capture_timed(wl.dense_gemm_native) if in_graph else None
+        if gt_native is not None:
+            native_ms, _ = timed_graph_ms(gt_native, max(10, args.steps // 2), flush, world)
+        else:
+            native_ms, _ = timed_ms(capture(wl.dense_gemm_native).replay, max(10, args.steps // 2), flush, world)
+        control = {"kernel": "dense-NVFP4 grouped GEMM (16-element UE4M3 blocks, 4.5 bit/weight), same skeleton; "
+                             "weights as MMA operand A (transposed, as the sparse kernel) and tokens as operand A "
+                             "(native, activation-stationary)",
                    "gemm_ms": dense_ms, "tflops": flops / (dense_ms * 1e-3) / 1e12,
                    "hbm_gbs": wl.dense_gemm_bytes() / (dense_ms * 1e-3) / 1e9,
-                   "sparse_speedup": dense_ms / gemm_ms}
+                   "sparse_speedup": dense_ms / gemm_ms,
+                   "native_gemm_ms": native_ms, "sparse_speedup_vs_native": native_ms / gemm_ms}
 
     traffic = traffic_from_profiles(cfg.name, int(gemm_bytes))
     secondary = None
@@ -836,7 +847,8 @@ def run_all_configs(args, local):
         torch.cuda.synchronize()
         res = {"config": name, "E": cfg.E, "K": cfg.K, "N": cfg.N, "tokens": cfg.T, "top_k": cfg.top_k,
                "routed_rows": cfg.R, "touched_experts": wl.touched, "max_rows_per_expert": wl.max_rows}
-        for tag, fn in (("gemm", wl.gemm), ("step", wl.step), ("dense_gemm", wl.dense_gemm)):
+        for tag, fn in (("gemm", wl.gemm), ("step", wl.step), ("dense_gemm", wl.dense_gemm),
+                        ("dense_native_gemm", wl.dense_gemm_native)):
             gt = capture_timed(fn)
             for _ in range(3):
                 flush.fill_(1)
@@ -867,6 +879,7 @@ def run_all_configs(args, local):
                     "gemm_total_gbs": (w + a + y) / g_s / 1e9, "gemm_hbm_frac": (w + a + y) / g_s / 1e9 / hbm,
                     "dense_gemm_gbs": wl.dense_gemm_bytes() / (res["dense_gemm_us"] * 1e-6) / 1e9,
                     "sparse_speedup": res["dense_gemm_us"] / res["gemm_us"],
+                    "sparse_speedup_vs_native": res["dense_native_gemm_us"] / res["gemm_us"],
                     "gemm_frac_of_read": res["read_same_bytes_us"] / res["gemm_us"],
                     "hbm_peak_gbs": hbm, "peak_source": kind, "reps": reps,
                     "timing": "the larger of: in-graph CUDA events around each replay, L2 flushed (256 MB write + "
@@ -1051,8 +1064,10 @@ def run_sweep(args, local):
                 Yd = torch.empty(R, N, dtype=torch.bfloat16, device=dev)
                 run_s = lambda: gsg.grouped_sparse_gemm(qa32, pwG, off, nt, out=Ys)
                 run_d = lambda: gsg.grouped_dense_gemm(qa16, pdG, off, nt, out=Yd)
+                run_n = lambda: gsg.grouped_dense_gemm_native(qa16, pdG, off, nt, out=Yd)
                 line = {"sweep": shape, "K": K, "N": N, "G": G, "tokens_per_expert": nt, "R": R}
-                for tag, fn, wbytes in (("sparse", run_s, G * sp_per), ("dense", run_d, G * dn_per)):
+                for tag, fn, wbytes in (("sparse", run_s, G * sp_per), ("dense", run_d, G * dn_per),
+                                        ("dense_native", run_n, G * dn_per)):
                     gt = capture_timed(fn)
                     for _ in range(3):
                         flush.fill_(1)
@@ -1074,6 +1089,7 @@ def run_sweep(args, local):
                                  "mj_per_call": e_call}
                     del gt
                 line["sparse_speedup"] = line["dense"]["us"] / line["sparse"]["us"]
+                line["sparse_speedup_vs_native"] = line["dense_native"]["us"] / line["sparse"]["us"]
                 st = gsg.get_device_status()
                 if st != 0:
                     raise RuntimeError(f"device status {st} in the sweep")

@@ -28,7 +28,7 @@ __all__ = [
     "pack_sparse_nvfp4", "pack_dense_nvfp4", "moe_route_permute", "moe_route_permute_noalloc",
     "quantize_act_nvfp4", "moe_dispatch_nvfp4",
     "grouped_sparse_gemm", "grouped_sparse_gemm_swiglu", "grouped_sparse_gemm_combine", "combine_workspace",
-    "grouped_dense_gemm", "unpermute_scale", "OP_COMBINE", "OP_DISPATCH",
+    "grouped_dense_gemm", "grouped_dense_gemm_native", "unpermute_scale", "OP_COMBINE", "OP_DISPATCH",
     "get_device_status",
     "save_packed", "load_packed",
     "act_scales_bytes", "workspace_size", "OP_PACK_SPARSE", "OP_PACK_DENSE", "OP_ROUTE",
@@ -46,7 +46,7 @@ EXPORTED_SYMBOLS = [
     "gsg_quantize_act_nvfp4", "gsg_grouped_sparse_gemm", "gsg_grouped_dense_gemm",
     "gsg_unpermute_scale", "gsg_get_device_status", "gsg_status_string", "gsg_version",
     "gsg_moe_route_permute_noalloc", "gsg_grouped_sparse_gemm_swiglu", "gsg_grouped_sparse_gemm_combine",
-    "gsg_moe_dispatch_nvfp4", "gsg_test_set_gemm_stall_ns",
+    "gsg_moe_dispatch_nvfp4", "gsg_test_set_gemm_stall_ns", "gsg_grouped_dense_gemm_native",
 ]
 
 _STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported shape", -3: "CUDA error",
@@ -91,6 +91,7 @@ def load_library(build_if_missing: bool = False) -> ctypes.CDLL:
         "gsg_moe_dispatch_nvfp4": (i, [vp, vp, i, i, i, i, i, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
         "gsg_grouped_sparse_gemm": (i, [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, i, vp]),
         "gsg_grouped_dense_gemm": (i, [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, i, vp]),
+        "gsg_grouped_dense_gemm_native": (i, [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, i, vp]),
         "gsg_unpermute_scale": (i, [vp, vp, vp, i, i, i, vp, vp]),
         "gsg_get_device_status": (i, [vp]),
         "gsg_status_string": (ctypes.c_char_p, [i]),
@@ -447,6 +448,22 @@ def grouped_dense_gemm(act: QuantizedActivations, w: PackedDenseWeights, offsets
         out = torch.empty(max(act.R, 1), w.N, dtype=out_dtype, device=act.codes.device)
     ydt = OUT_F32 if out.dtype == torch.float32 else OUT_BF16
     _check("gsg_grouped_dense_gemm", lib().gsg_grouped_dense_gemm(
+        _ptr(act.codes), _ptr(act.scales), _ptr(act.x_scale), _ptr(w.packed), _ptr(w.w_scale),
+        _ptr(offsets), w.E, w.N, w.K, act.R, max_rows_per_expert, _ptr(out), ydt, _stream(stream)))
+    return out
+
+
+def grouped_dense_gemm_native(act: QuantizedActivations, w: PackedDenseWeights, offsets: torch.Tensor,
+                              max_rows_per_expert: int = -1, out: Optional[torch.Tensor] = None,
+                              out_dtype: torch.dtype = torch.bfloat16, stream=None) -> torch.Tensor:
+    """The dense-NVFP4 control with the token rows as MMA operand A (the activation-stationary
+    orientation, gsg_grouped_dense_gemm_native); the same result as grouped_dense_gemm."""
+    assert act.sf_block == 16 and act.K == w.K
+    _need_cuda(act.codes, act.scales, offsets)
+    if out is None:
+        out = torch.empty(max(act.R, 1), w.N, dtype=out_dtype, device=act.codes.device)
+    ydt = OUT_F32 if out.dtype == torch.float32 else OUT_BF16
+    _check("gsg_grouped_dense_gemm_native", lib().gsg_grouped_dense_gemm_native(
         _ptr(act.codes), _ptr(act.scales), _ptr(act.x_scale), _ptr(w.packed), _ptr(w.w_scale),
         _ptr(offsets), w.E, w.N, w.K, act.R, max_rows_per_expert, _ptr(out), ydt, _stream(stream)))
     return out

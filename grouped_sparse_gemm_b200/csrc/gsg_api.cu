@@ -219,7 +219,8 @@ gsg_status_t gsg_moe_dispatch_nvfp4(const int32_t* topk_ids, const uint16_t* X, 
 
 static gsg_status_t gemm_common(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, const float* x_scale,
                                 const uint8_t* w_packed, const float* w_scale, const int32_t* off, int E, int N,
-                                int K, int R, int max_rows, void* Y, int y_dtype, void* stream) {
+                                int K, int R, int max_rows, void* Y, int y_dtype, void* stream,
+                                bool native = false) {
   if (R < 0 || (y_dtype != GSG_OUT_BF16 && y_dtype != GSG_OUT_F32)) return GSG_ERR_INVALID_ARG;
   if (!weight_shape_ok(E, N, K) || !gsg::gemm_supported(E)) return GSG_ERR_UNSUPPORTED_SHAPE;
   if ((long long)R > (1ll << 30)) return GSG_ERR_UNSUPPORTED_SHAPE;
@@ -231,7 +232,8 @@ static gsg_status_t gemm_common(bool sparse, const uint8_t* a_codes, const uint8
   gsg_status_t st = device_state(&d);
   if (st != GSG_OK) return st;
   const int rc = gsg::launch_gemm(sparse, a_codes, a_scales, x_scale, w_packed, w_scale, off, E, N, K, R, max_rows,
-                                  Y, y_dtype == GSG_OUT_F32 ? 1 : 0, d->status, d->num_sms, as_stream(stream));
+                                  Y, y_dtype == GSG_OUT_F32 ? 1 : 0, d->status, d->num_sms, as_stream(stream),
+                                  nullptr, nullptr, nullptr, native);
   return rc == 0 ? GSG_OK : GSG_ERR_CUDA;
 }
 
@@ -249,6 +251,15 @@ gsg_status_t gsg_grouped_dense_gemm(const uint8_t* a_codes, const uint8_t* a_sca
                                     int max_rows_per_expert, void* Y, int y_dtype, void* stream) {
   return gemm_common(false, a_codes, a_scales, x_tensor_scale, w_packed, w_tensor_scale, expert_offsets, E, N, K, R,
                      max_rows_per_expert, Y, y_dtype, stream);
+}
+
+gsg_status_t gsg_grouped_dense_gemm_native(const uint8_t* a_codes, const uint8_t* a_scales,
+                                           const float* x_tensor_scale, const uint8_t* w_packed,
+                                           const float* w_tensor_scale, const int32_t* expert_offsets, int E, int N,
+                                           int K, int R, int max_rows_per_expert, void* Y, int y_dtype,
+                                           void* stream) {
+  return gemm_common(false, a_codes, a_scales, x_tensor_scale, w_packed, w_tensor_scale, expert_offsets, E, N, K, R,
+                     max_rows_per_expert, Y, y_dtype, stream, true);
 }
 
 gsg_status_t gsg_grouped_sparse_gemm_swiglu(const uint8_t* a_codes, const uint8_t* a_scales,

@@ -449,13 +449,17 @@ struct Geo {
 // together; see Geo.  CTA rank 0 of the pair (the leader) issues the pair's MMAs and owns the
 // barriers the MMAs wait on (tfull, acce: arrived on by both CTAs' loader and epilogue warps);
 // every MMA completion is signalled to the barriers of both CTAs (empty, accf).
-template <bool kSparse, int kBN, bool kGLU, int kCG>
+// kNative: the dense control in the activation-stationary orientation -- the tile's 128 token rows
+// are MMA operand A (M = 128, padded when fewer rows are routed) and the weight n-tile is operand
+// B (N = 128); the accumulator then holds a token per TMEM lane and a feature per column.
+template <bool kSparse, int kBN, bool kGLU, int kCG, bool kNative = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ CUtensorMap tmap_b64,
                     const __grid_constant__ CUtensorMap tmap_sfb,
                     const GemmParams p) {
   using G = Geo<kSparse, kBN, kGLU, kCG>;
   constexpr bool kPair = kCG == 2;
+  static_assert(!kNative || (!kSparse && kBN == 128 && !kGLU && kCG == 1), "native orientation: dense, 128 tokens");
   extern __shared__ uint8_t smem_raw[];
   // NT: weight n-tiles; tiles run over NT / (kNT * kCG) columns (the gate n-tiles with the SwiGLU
   // epilogue, n-tile pairs for CTA pairs)
@@ -766,7 +770,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
     const int n_mma = rank == 0u ? n_my : 0;
     for (int j = 0; j < n_mma && !*abort_flag; ++j) {
       const TileDesc c = my_tile(j, ttab, p.tcap, pref, offs, E, kBN, p.sched, tb, unit, nunits);
-      const uint32_t idesc = make_idesc(kSparse, (c.valid + 15) & ~15, kTileN * kCG);
+      const uint32_t idesc = kNative ? make_idesc(false, kTileN, kBN)   // M = 128 tokens, N = 128 weight rows
+                                     : make_idesc(kSparse, (c.valid + 15) & ~15, kTileN * kCG);
       if (p.stall_ns != 0ull && j == (n_mma > 1 ? 1 : 0) &&
           !wait_warp(never_bar, 0u, abort_flag, p.status, p.stall_ns))
         break;
@@ -799,7 +804,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
                 const uint32_t d = d_tmem + (uint32_t)(t * G::kAccStride);
                 const int kt = t * G::kKbps + kbi;
                 const uint32_t sfa = tset + G::kColSFA + 4 * kt, sfb = tset + G::kColSFB + 4 * kbi;
-                if constexpr (kSparse && kPair)
+                if constexpr (kNative)   // tokens as A, weights as B: the operands and their scales swap
+                  tc_mma_dense(d, bdesc, adesc, idesc, accum, sfb, sfa);
+                else if constexpr (kSparse && kPair)
                   tc_mma_sparse_pair(d, adesc, bdesc, idesc, accum, sfa, sfb, tset + 2 * kt);
                 else if constexpr (kSparse)
                   tc_mma_sparse(d, adesc, bdesc, idesc, accum, sfa, sfb, tset + 2 * kt);
@@ -845,7 +852,35 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
       tc_fence_after();
       const float scale = __fmul_rn(sx, wsc[c.e]);
       const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + kColAcc + (uint32_t)(acc * G::kNT * G::kAccStride);
-      if constexpr (kGLU) {
+      if constexpr (kNative) {
+        // lane = token 32q + lane of the tile, columns = the n-tile's 128 features: each lane scales
+        // and stores its own token's row segment (16-byte stores, 16 features at a time)
+        const int tok = 32 * q + lane;
+        const size_t col0 = (size_t)c.nt * kTileN;
+        for (int f0 = 0; f0 < kTileN; f0 += 16) {
+          float v[16];
+          tc_ld_16(taddr + f0, v);
+          if (tok < valid) {
+            if (p.y_f32) {
+              float* Yr = static_cast<float*>(p.Y) + (size_t)(r0 + tok) * p.N + col0 + f0;
+#pragma unroll
+              for (int w = 0; w < 4; ++w)
+                *reinterpret_cast<float4*>(Yr + 4 * w) =
+                    make_float4(__fmul_rn(v[4 * w], scale), __fmul_rn(v[4 * w + 1], scale),
+                                __fmul_rn(v[4 * w + 2], scale), __fmul_rn(v[4 * w + 3], scale));
+            } else {
+              uint32_t pk[8];
+#pragma unroll
+              for (int w = 0; w < 8; ++w)
+                pk[w] = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(v[2 * w], scale))) |
+                        ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(v[2 * w + 1], scale))) << 16);
+              uint4* Yr = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.Y) + (size_t)(r0 + tok) * p.N + col0 + f0);
+              Yr[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              Yr[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            }
+          }
+        }
+      } else if constexpr (kGLU) {
         // SwiGLU output preparation, 32 tokens at a time: lane = feature f of this warp's
         // 32-feature block (one NVFP4 block of the down-projection's K), h = silu(gate) * up in
         // fp32; the block is transposed through shared memory so that each lane then owns one
@@ -1103,9 +1138,9 @@ static EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-template <bool kSparse, int kBN, bool kGLU = false, int kCG = 1>
+template <bool kSparse, int kBN, bool kGLU = false, int kCG = 1, bool kNative = false>
 static cudaError_t set_attr_one(int bytes) {
-  return cudaFuncSetAttribute(grouped_gemm_kernel<kSparse, kBN, kGLU, kCG>,
+  return cudaFuncSetAttribute(grouped_gemm_kernel<kSparse, kBN, kGLU, kCG, kNative>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
@@ -1142,13 +1177,13 @@ cudaError_t gemm_set_smem_attrs() {
   if (e != cudaSuccess) return e;
   maxb -= 1024;   // room for the kernels' static shared memory
   g_smem_limit = maxb;
-  cudaError_t errs[13] = {set_attr_one<true, 16>(maxb),       set_attr_one<true, 32>(maxb),
+  cudaError_t errs[14] = {set_attr_one<true, 16>(maxb),       set_attr_one<true, 32>(maxb),
                           set_attr_one<true, 64>(maxb),       set_attr_one<true, 128>(maxb),
                           set_attr_one<false, 16>(maxb),      set_attr_one<false, 32>(maxb),
                           set_attr_one<false, 64>(maxb),      set_attr_one<false, 128>(maxb),
                           set_attr_one<true, 16, true>(maxb), set_attr_one<true, 32, true>(maxb),
                           set_attr_one<true, 64, true>(maxb), set_attr_one<true, 128, false, 2>(maxb),
-                          set_attr_one<false, 128, false, 2>(maxb)};
+                          set_attr_one<false, 128, false, 2>(maxb), set_attr_one<false, 128, false, 1, true>(maxb)};
   for (cudaError_t x : errs)
     if (x != cudaSuccess) return x;
   g_pair_units[1] = max_pairs<true>(maxb);
@@ -1169,8 +1204,11 @@ static cudaError_t launch_bn(int BN, int grid, size_t smem, cudaStream_t stream,
 template <bool kSparse>
 static cudaError_t launch_bn(int BN, int grid, size_t smem, cudaStream_t stream, const CUtensorMap& tb,
                              const CUtensorMap& tb64, const CUtensorMap& ts, const GemmParams& p, bool glu,
-                             bool pair) {
+                             bool pair, bool native = false) {
   if (glu) return launch_bn<true, true>(BN, grid, smem, stream, tb, tb64, ts, p);
+  if (!kSparse && native)
+    return launch_pdl(grouped_gemm_kernel<false, 128, false, 1, true>, grid, kGemmThreads, smem, stream, tb, tb64, ts,
+                      p);
   if (BN == 128 && pair)
     return launch_pdl_cluster(grouped_gemm_kernel<kSparse, 128, false, 2>, grid, kGemmThreads, smem, stream, 2u, tb,
                               tb64, ts, p);
@@ -1185,16 +1223,17 @@ static cudaError_t launch_bn(int BN, int grid, size_t smem, cudaStream_t stream,
 int launch_gemm(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, const float* x_scale,
                 const uint8_t* w_packed, const float* w_scale, const int32_t* off, int E, int N, int K, int R,
                 int max_rows, void* Y, int y_f32, int* status, int num_sms, cudaStream_t stream,
-                uint8_t* h_scales, const float* h_scale, const CombineArgs* comb) {
+                uint8_t* h_scales, const float* h_scale, const CombineArgs* comb, bool native) {
   EncodeTiledFn enc = get_encode_fn();
   if (enc == nullptr) return 2;
   const bool glu = h_scales != nullptr;
-  int BN = gemm_pick_bn(max_rows, R, E);
+  if (native && (sparse || glu || comb != nullptr)) return 1;
+  int BN = native ? 128 : gemm_pick_bn(max_rows, R, E);   // the native orientation: 128-token tiles (MMA M)
   if (glu && BN > 64) BN = 64;   // two accumulators per tile: 64-token tiles at most
   // 128-token tiles run as CTA pairs (256 weight rows per tile) when N holds whole n-tile pairs
   // and the device can co-schedule pairs
   const int pair_units = g_pair_units[sparse ? 1 : 0];
-  const bool pair = BN == 128 && !glu && (N / kTileN) % 2 == 0 && pair_units > 0;
+  const bool pair = BN == 128 && !glu && !native && (N / kTileN) % 2 == 0 && pair_units > 0;
   const int cg = pair ? 2 : 1;
   const int units = pair ? (pair_units < num_sms / 2 ? pair_units : num_sms / 2) : num_sms;   // pairs or CTAs
   const int grid = units * cg;
@@ -1259,7 +1298,7 @@ int launch_gemm(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, co
   p.k = comb ? comb->k : 1;
   p.stall_ns = g_test_stall_ns.load();
   const cudaError_t e = sparse ? launch_bn<true>(g.BN, grid, g.smem, stream, tb, tb64, ts, p, glu, pair)
-                               : launch_bn<false>(g.BN, grid, g.smem, stream, tb, tb64, ts, p, false, pair);
+                               : launch_bn<false>(g.BN, grid, g.smem, stream, tb, tb64, ts, p, false, pair, native);
   return e == cudaSuccess ? 0 : 1;
 }
 

@@ -66,6 +66,7 @@ cudaError_t gemm_set_smem_attrs();
 int launch_gemm(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, const float* x_scale,
                 const uint8_t* w_packed, const float* w_scale, const int32_t* off, int E, int N, int K, int R,
                 int max_rows, void* Y, int y_f32, int* status, int num_sms, cudaStream_t stream,
-                uint8_t* h_scales = nullptr, const float* h_scale = nullptr, const CombineArgs* comb = nullptr);
+                uint8_t* h_scales = nullptr, const float* h_scale = nullptr, const CombineArgs* comb = nullptr,
+                bool native = false);
 
 }  // namespace gsg

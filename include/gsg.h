@@ -190,6 +190,18 @@ gsg_status_t gsg_grouped_dense_gemm(const uint8_t* a_codes, const uint8_t* a_sca
                                     const int32_t* expert_offsets, int E, int N, int K, int R,
                                     int max_rows_per_expert, void* Y, int y_dtype, void* stream);
 
+/* gsg_grouped_dense_gemm_native -- the same dense control in the activation-stationary ("native")
+ * orientation of the paper's kernel benchmark (§D.2, p.19, Figure 5: CUTLASS dense NVFP4 "native"
+ * and "transposed").  Each tile's 128 token rows are MMA operand A and the weight n-tile is
+ * operand B; gsg_grouped_dense_gemm (and the sparse kernel) put the weights in A and the tokens in
+ * B ("transposed").  Same arguments, result and errors as gsg_grouped_dense_gemm; every token tile
+ * is 128 rows (MMA M), padded when an expert has fewer routed rows. */
+gsg_status_t gsg_grouped_dense_gemm_native(const uint8_t* a_codes, const uint8_t* a_scales,
+                                           const float* x_tensor_scale,
+                                           const uint8_t* w_packed, const float* w_tensor_scale,
+                                           const int32_t* expert_offsets, int E, int N, int K, int R,
+                                           int max_rows_per_expert, void* Y, int y_dtype, void* stream);
+
 /* gsg_grouped_sparse_gemm_swiglu -- the up-projection with SwiGLU output preparation fused into
  * the epilogue, producing the down-projection's NVFP4 input directly.
  * Paper: §D.1 (p.19): the serving integration fuses SwiGLU output preparation for the second

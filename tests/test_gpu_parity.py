@@ -273,7 +273,7 @@ def _gemm_case(counts, N, K, seed=0, sparse=True):
                 w=w, canon=canon, sws=sws, sf=sf)
 
 
-def _run_gemm(gsg, c, sparse, hint, out_dtype):
+def _run_gemm(gsg, c, sparse, hint, out_dtype, native=False):
     t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
     act = gsg.QuantizedActivations(codes=t(c["a_codes"]), scales=t(c["a_quad"]),
                                    x_scale=torch.tensor([c["s_x"]], dtype=torch.float32, device=DEV),
@@ -285,6 +285,8 @@ def _run_gemm(gsg, c, sparse, hint, out_dtype):
         return gsg.grouped_sparse_gemm(act, w, off, max_rows_per_expert=hint, out_dtype=out_dtype)
     w = gsg.PackedDenseWeights(packed=t(c["w"]["packed"]), w_scale=t(c["w"]["w_scale"]), E=c["E"], N=c["N"],
                                K=c["K"])
+    if native:
+        return gsg.grouped_dense_gemm_native(act, w, off, max_rows_per_expert=hint, out_dtype=out_dtype)
     return gsg.grouped_dense_gemm(act, w, off, max_rows_per_expert=hint, out_dtype=out_dtype)
 
 
@@ -329,6 +331,19 @@ def test_dense_gemm_oracle_inputs(gsg, counts, N, K):
     y_ref, bound = tl.reference_rows(np.arange(c["R"]), c["off"], c["q"], c["sc"], 16, c["canon"], c["s_x"],
                                      c["sws"], sparse=False, w_sf=16)
     tl.assert_gemm_close(y[:c["R"]], y_ref, bound, f"dense {counts}")
+
+
+@pytest.mark.parametrize("counts,N,K", GEMM_CASES)
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_dense_native_gemm_oracle_inputs(gsg, counts, N, K, out_dtype):
+    """The dense control in the activation-stationary orientation (tokens as MMA operand A)."""
+    c = _gemm_case(counts, N, K, sparse=False)
+    y = _run_gemm(gsg, c, False, -1, out_dtype, native=True)
+    torch.cuda.synchronize()
+    _status_ok(gsg)
+    y_ref, bound = tl.reference_rows(np.arange(c["R"]), c["off"], c["q"], c["sc"], 16, c["canon"], c["s_x"],
+                                     c["sws"], sparse=False, w_sf=16)
+    tl.assert_gemm_close(y[:c["R"]], y_ref, bound, f"dense native {counts}")
 
 
 def test_gemm_deterministic(gsg):
