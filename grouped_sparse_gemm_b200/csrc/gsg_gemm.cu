@@ -594,7 +594,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
   // bytes per tile: weights wc, plus ac per token row (codes, scales, output row segment)
   const long long wc = (long long)G::kNT * kCG * kTileN * p.K * (kSparse ? 11 : 18) / 32;
   const long long ac = p.K / 2 + p.K / (kSparse ? 32 : 16) + (long long)G::kNT * kCG * kTileN * (p.y_f32 ? 4 : 2);
-  {
+  if (p.sched == kSchedRuns) {   // (only the byte-balanced schedule reads the costs; uniform branch)
     // chunked exclusive scan of cost_e = NTt * (ceil(rows_e / BN) * wc + rows_e * ac)
     const int per = (E + kGemmThreads - 1) / kGemmThreads;
     const int e0 = threadIdx.x * per, e1 = min(e0 + per, E);
