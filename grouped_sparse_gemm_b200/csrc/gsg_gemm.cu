@@ -39,7 +39,6 @@ constexpr int kMaxAcc = 8;
 constexpr int kNSets = 3;                  // TMEM sets of metadata + scales
 constexpr uint32_t kSetCols = 64;
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;   // 2 s
-constexpr int kPrefetchRings = 1;                     // L2 prefetch distance, in ring lengths
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColAcc = kNSets * kSetCols;       // first accumulator (192)
 constexpr int kOutStageBytes = 16 * 32 * 4;           // epilogue transpose buffer per warp
@@ -174,21 +173,6 @@ __device__ __forceinline__ void tma_load_3d_lane(bool on, uint32_t dst, const CU
       "@P cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];\n\t}" ::
           "r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar), "r"((uint32_t)on)
-      : "memory");
-}
-// L2 prefetches (no shared memory, no barrier): a byte range, and one tensor-map box.
-__device__ __forceinline__ void prefetch_l2_lane(bool on, const void* src, uint32_t bytes) {
-  asm volatile(
-      "{\n\t.reg .pred P;\n\tsetp.ne.b32 P, %2, 0;\n\t"
-      "@P cp.async.bulk.prefetch.L2.global [%0], %1;\n\t}" ::"l"(src),
-      "r"(bytes), "r"((uint32_t)on)
-      : "memory");
-}
-__device__ __forceinline__ void prefetch_tile_2d_lane(bool on, const CUtensorMap* map, int x, int y) {
-  asm volatile(
-      "{\n\t.reg .pred P;\n\tsetp.ne.b32 P, %3, 0;\n\t"
-      "@P cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];\n\t}" ::"l"(reinterpret_cast<uint64_t>(map)),
-      "r"(x), "r"(y), "r"((uint32_t)on)
       : "memory");
 }
 __device__ __forceinline__ void lds128(uint32_t saddr, uint32_t& a, uint32_t& b, uint32_t& c, uint32_t& d) {
@@ -662,7 +646,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
     const bool wprod = warp == 0;
     int s = 0, g = 0;   // ring slot and stage counter
     uint32_t ph = 0;
-    const int stages_per_tile = (KC + G::kCPS - 1) / G::kCPS;
     for (int j = 0; j < n_my && !*abort_flag; ++j) {
       const TileDesc c = my_tile(j, ttab, p.tcap, pref, offs, E, kBN, p.sched, tb, unit, nunits);
       const uint8_t* wsrc = p.w_packed + ((size_t)c.e * NT + c.nt * kCG + rank) * KC * G::kCB;
@@ -702,32 +685,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
           const int roff = b64 ? 64 * b : 64 * n64 + (b - n64) * G::kBoxH;
           tma_load_2d_lane(lane < nch * nb, st + ch * G::kBChunk + roff * 128, b64 ? &tmap_b64 : &tmap_b,
                            (kc + ch) * 128, r0 + roff, fb);
-        }
-        // L2 prefetch of the same operand for the stage kPrefetchRings ring lengths ahead, so that its
-        // copy, when its ring slot comes free, finds the bytes in L2 instead of DRAM (every tile has
-        // the same number of stages, so that stage's tile is found in the tile table)
-        {
-          const int gf = g + kPrefetchRings * S;
-          const int jf = gf / stages_per_tile, kcf = (gf - jf * stages_per_tile) * G::kCPS;
-          if (jf < n_my) {
-            const TileDesc cf = my_tile(jf, ttab, p.tcap, pref, offs, E, kBN, p.sched, tb, unit, nunits);
-            const int nchf = KC - kcf >= G::kCPS ? G::kCPS : KC - kcf;
-            if (wprod) {
-              const uint8_t* wf = p.w_packed + ((size_t)cf.e * NT + (size_t)cf.nt * kCG + rank) * KC * G::kCB;
-              const int t = lane / nchf, ch = lane - t * nchf;
-              prefetch_l2_lane(lane < G::kNT * nchf,
-                               (t == 0 ? wf : wf + (size_t)(NT / 2) * KC * G::kCB) + (size_t)(kcf + ch) * G::kCB,
-                               G::kCB);
-            } else {
-              const int nhf = kPair ? ((cf.valid + 15) & ~15) / 2 : kBN;
-              const int cntf = min(max(cf.valid - (int)rank * nhf, 0), nhf);
-              const int rowsf = (cntf + G::kBoxH - 1) / G::kBoxH * G::kBoxH;
-              const int nbf = rowsf / G::kBoxH;   // 32-row boxes (or one box of BN rows)
-              const int ch = nbf > 0 ? lane / nbf : 0, b = lane - ch * nbf;
-              prefetch_tile_2d_lane(lane < nchf * nbf, &tmap_b, (kcf + ch) * 128,
-                                    cf.r0 + (int)rank * nhf + b * G::kBoxH);
-            }
-          }
         }
         ++g;
         if (++s == S) { s = 0; ph ^= 1u; }
