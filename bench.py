@@ -257,11 +257,13 @@ class Workload:
                                         out=self.out)
 
     def launches_per_step(self) -> int:
-        """Library kernels one step launches (the library's routing rule: one launch up to 2048
-        rows, histogram + scatter while ceil(R/1024)*E <= 16384, else histogram + scan + scatter)."""
-        R, E = self.cfg.R, self.cfg.E
+        """Library kernels one step launches (the library's rules: routing in one launch up to 2048
+        rows, histogram + scatter while ceil(R/1024)*E <= 16384, else histogram + scan + scatter;
+        the quantizer in one launch, two from R*K = 2^27 when the scale words are staged)."""
+        R, E, K = self.cfg.R, self.cfg.E, self.cfg.K
         route = 1 if R <= 2048 else (2 if -(-R // 1024) * E <= 16384 else 3)
-        return route + 1 + 1 + 1        # routing (the amax pass in its first launch), quantize, GEMM, scatter
+        quant = 2 if R * K >= (1 << 27) else 1
+        return route + quant + 1 + 1    # routing (the amax pass in its first launch), quantize, GEMM, scatter
 
     def gemm(self):
         gsg.grouped_sparse_gemm(self.qa, self.pw, self.route.offsets, self.max_rows, out=self.Y)
