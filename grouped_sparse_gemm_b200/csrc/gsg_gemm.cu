@@ -1094,13 +1094,21 @@ static GemmPlan make_plan(bool sparse, int BN, int E, int tcap, bool glu = false
   if (BN == 128 && cg == 1 && budget > kStageBudget128) budget = kStageBudget128;
   g.stages = (budget - tcap * 16) / g.stage;
   if (g.stages > kMaxStages) g.stages = kMaxStages;
+  // the ring comes before the tile table: where the table would cost a stage, it keeps only what
+  // fits beside the full ring (a CTA decodes its later tiles from the expert offsets instead)
+  int ring = budget / g.stage;
+  if (ring > kMaxStages) ring = kMaxStages;
+  if (g.stages < ring) {
+    g.stages = ring;
+    g.tcap = (budget - ring * g.stage) / 16;
+  }
   const int acc_stride = (BN < 32 ? 32 : BN) * nt;
   g.nacc = (int)((kTmemCols - kColAcc) / acc_stride);
   if (g.nacc > kMaxAcc) g.nacc = kMaxAcc;
   const int nbars = 2 * g.stages + kNSets + 2 * g.nacc + 2;
   g.smem = 1024 + (size_t)g.stages * g.stage + nbars * 8 + sizeof(Ctl) + (size_t)(3 * E + 2) * 4 + 16 +
            (size_t)(E + 1) * 8 + 16 +
-           (size_t)tcap * 16 + ostage;
+           (size_t)g.tcap * 16 + ostage;
   return g;
 }
 

@@ -71,6 +71,18 @@ for _b in (1, 32, 128, 256):
 CONFIGS["1t_up_prefill_e64"] = MoEConfig("1t_up_prefill_e64", E=64, K=7168, N=4096, T=1368, top_k=8,
                                          routing="zipf", zipf_s=1.1, w_sigma=0.015,
                                          outlier_frac=0.005, outlier_scale=30.0)
+# The 1T prefill up-projection at 65,536 tokens top-8 (R = 524,288): eight times the rows on the
+# same weights, 30.8 dense-equivalent TFLOP against 10.2 GB of algorithmic traffic (packed weights,
+# activation codes and scales, bf16 output), past the ridge point of the sparse NVFP4 tensor roof.
+# A measurement of the kernel where the tensor pipe, not HBM, is the binding roof; not one of the
+# expert-projection workloads.  The _e64 variant keeps its rows per expert on 64 experts (10,920
+# tokens) for profiler captures.
+CONFIGS["1t_up_prefill_65k"] = MoEConfig("1t_up_prefill_65k", E=384, K=7168, N=4096, T=65536, top_k=8,
+                                         routing="zipf", zipf_s=1.1, w_sigma=0.015,
+                                         outlier_frac=0.005, outlier_scale=30.0)
+CONFIGS["1t_up_prefill_65k_e64"] = MoEConfig("1t_up_prefill_65k_e64", E=64, K=7168, N=4096, T=10920, top_k=8,
+                                             routing="zipf", zipf_s=1.1, w_sigma=0.015,
+                                             outlier_frac=0.005, outlier_scale=30.0)
 
 
 @dataclasses.dataclass(frozen=True)

@@ -121,6 +121,49 @@ def test_gemm_full_size_sampled(gsg, name):
     assert torch.equal(Y[sel], Y32[sel].to(torch.bfloat16))
 
 
+def test_gemm_65k_tokens_sampled(gsg):
+    """The 1T up-projection at 65,536 tokens top-8 (R = 524,288 routed rows, past the tensor roof's
+    ridge point): routing bit for bit over the whole batch, the activation tensor scale, the
+    quantized codes and scales of the sampled rows bit for bit, and the GEMM on the sampled rows
+    of the sampled experts at the stated bound (bf16 and fp32 outputs).  Output offsets reach
+    2^32 bytes here, so 32-bit address arithmetic anywhere on the path would show."""
+    from oracle import gemm as ogemm
+    from oracle import quant as oquant
+    cfg = inputs.CONFIGS["1t_up_prefill_65k"]
+    R, K = cfg.R, cfg.K
+    ids = inputs.routing(cfg)
+    off, ps, ip = tl.route_np(ids, cfg.E)
+    counts = np.diff(off)
+    sample_e = _sample_experts(counts)
+    pw, canon, sws = _pack_all(gsg, cfg, lambda e: inputs.expert_weight(cfg, e, DEV), sample_e)
+    X = inputs.activations(cfg)
+    r, qa = gsg.moe_dispatch_nvfp4(ids.to(DEV), X.to(DEV), cfg.E, 32)
+    Y = gsg.grouped_sparse_gemm(qa, pw, r.offsets, int(counts.max()), out_dtype=torch.bfloat16)
+    Y32 = gsg.grouped_sparse_gemm(qa, pw, r.offsets, int(counts.max()), out_dtype=torch.float32)
+    assert gsg.get_device_status() == 0
+    np.testing.assert_array_equal(r.offsets.cpu().numpy(), off)
+    np.testing.assert_array_equal(r.perm_src.cpu().numpy()[:R], ps)
+    np.testing.assert_array_equal(r.inv_perm.cpu().numpy()[:R], ip)
+    s_x = oquant.act_tensor_scale(X.float().numpy())
+    assert qa.x_scale.item() == s_x
+    rows = _sample_rows(off, sample_e)
+    sel = torch.from_numpy(rows).to(DEV)
+    q, sc = oquant.quantize_rows(X[torch.from_numpy(ps[rows] // cfg.top_k)].float().numpy(), 32, s_x)
+    np.testing.assert_array_equal(olayout.unpack_act_codes(qa.codes[sel].cpu().numpy()), q)
+    q5 = qa.scales.view(K // 128, -1, 4, 4)
+    np.testing.assert_array_equal(q5[:, sel, 0, :].cpu().numpy().transpose(1, 0, 2).reshape(rows.size, K // 32), sc)
+    # reference rows, expert by expert
+    experts = ogemm.expert_of_rows(off, rows)
+    y_ref, bound = np.zeros((rows.size, cfg.N)), np.zeros((rows.size, cfg.N))
+    for e in np.unique(experts):
+        i = np.nonzero(experts == e)[0]
+        y_ref[i], bound[i] = ogemm.gemm_rows(oquant.decode_rows(q[i], sc[i], 32),
+                                             opack.decode_sparse_expert(*canon[e]), float(s_x) * float(sws[e]))
+    tl.assert_gemm_close(Y32[sel], y_ref, bound, "65k tokens sampled rows, fp32 output")
+    tl.assert_gemm_close(Y[sel], y_ref, bound, "65k tokens sampled rows, bf16 output")
+    assert torch.equal(Y[sel], Y32[sel].to(torch.bfloat16))
+
+
 @pytest.mark.parametrize("name", ["30b_layer", "1t_layer"])
 def test_moe_layer_full_size_sampled(gsg, name):
     """route + quantize -> up-projection with the SwiGLU epilogue -> down-projection -> unpermute
