@@ -6,8 +6,9 @@
 // §2 "Hardware opportunity" (p.3) -- paired 4:8 NVFP4 runs at twice the dense NVFP4 rate;
 // §D.2 (p.19) -- a dense control that differs from the sparse kernel only in sparsity.
 //
-// One CTA per SM, 352 threads (11 warps), warp-specialised around one shared-memory ring whose
-// stages hold 256 to 768 logical K of one tile (weights, activation codes and both scales):
+// One CTA per SM, 352 threads (11 warps; 480 = 15 warps for wide pair tiles), warp-specialised
+// around one shared-memory ring whose stages hold 256 to 768 logical K of one tile (weights,
+// activation codes and both scales):
 //   warp 0      weight producer: per stage one bulk copy per interleaved packed weight block and
 //               one 3-D TMA box of the activation scale atoms, each from its own lane.
 //   warp 2      activation producer: tensor-map TMA boxes (128B swizzle, 64 or 32 rows) of only the
@@ -18,7 +19,14 @@
 //               block_scale (M = 128 weight rows, N = the tile's token count rounded to 16, K = 128
 //               logical sparse / 64 dense) and one tcgen05.commit; up to eight TMEM accumulators.
 //   warps 3..6  epilogue: tcgen05.ld accumulator lanes, multiply by s_x * s_w[e], store rows of Y.
+//   warps 11..14 (wide pair tiles only) a second epilogue, for the tile's second n-tile pair.
 // Every TMA and tcgen05 instruction is issued by an elected lane of a converged warp.
+// 128-token tiles run on CTA pairs (cta_group::2, M = 256 weight rows).  Where N holds whole
+// groups of four n-tiles, a pair tile is wide: 512 weight rows (two MMAs per k-block into two
+// accumulators) against one 128-token activation tile, so the activations cross from L2 to the
+// SMs once for 512 weight rows instead of once per 256.  Its two accumulators fill TMEM beside the
+// metadata sets, so there is one accumulator buffer; the MMA warp waits for the epilogue between
+// tiles, and the two epilogue warp groups halve that wait.
 // Tiles are (expert e, 128 weight rows nt, token tile mt) in e -> nt -> mt order; CTAs take
 // tiles round-robin and decode their own tile list into shared memory once, at set-up.
 // Experts with no rows produce no tiles.  Every mbarrier wait is bounded:
@@ -34,6 +42,10 @@
 namespace gsg {
 
 constexpr int kGemmThreads = 352;
+// a wide pair tile adds four epilogue warps (11..14) that drain the tile's second n-tile while
+// warps 3..6 drain the first
+constexpr int kGemmThreadsWide = 480;
+__host__ __device__ constexpr int gemm_threads(bool wide) { return wide ? kGemmThreadsWide : kGemmThreads; }
 constexpr int kMaxE = 1024;
 constexpr int kMaxAcc = 8;
 constexpr int kNSets = 3;                  // TMEM sets of metadata + scales
@@ -407,8 +419,8 @@ __device__ __forceinline__ int tile_at_cost(long long target, const long long* c
 // 256-wide K chunks per ring stage: short token tiles take longer stages (fewer waits per weight
 // byte); 128-token tiles keep two-chunk stages, also on CTA pairs (three-chunk stages, three of
 // them in shared memory, measured slower than five two-chunk stages).
-__host__ __device__ constexpr int stage_chunks(bool sparse, int BN, bool glu, int cg) {
-  return glu ? 2 : sparse ? (BN <= 32 ? 3 : 2) : (BN <= 32 ? 2 : 1);
+__host__ __device__ constexpr int stage_chunks(bool sparse, int BN, bool glu, int cg, bool wide = false) {
+  return wide ? (sparse ? 2 : 1) : glu ? 2 : sparse ? (BN <= 32 ? 3 : 2) : (BN <= 32 ? 2 : 1);
 }
 
 // Compile-time stage geometry of one (sparse/dense, token tile, SwiGLU, CTA group) instantiation.
@@ -418,14 +430,15 @@ __host__ __device__ constexpr int stage_chunks(bool sparse, int BN, bool glu, in
 // by a pair of CTAs on two SMs: CTA r holds n-tile 2*np + r and half of the token rows, and the
 // pair's MMAs (M = 256) read both CTAs' shared memory, so each SM stages its own weights but only
 // half of the shared activation tile.
-template <bool kSparse, int kBN, bool kGLU = false, int kCG = 1>
+template <bool kSparse, int kBN, bool kGLU = false, int kCG = 1, bool kWide = false>
 struct Geo {
   static_assert(kCG == 1 || (kCG == 2 && !kGLU && kBN == 128), "CTA pairs: 128-token tiles, plain epilogue");
-  static constexpr int kNT = kGLU ? 2 : 1;                         // weight n-tiles per tile
+  static_assert(!kWide || kCG == 2, "wide tiles run on CTA pairs");
+  static constexpr int kNT = (kGLU || kWide) ? 2 : 1;              // weight n-tiles per tile (per CTA)
   static constexpr int kKbLogical = kSparse ? 128 : 64;            // logical K per MMA
   static constexpr int kKbPerChunk = kChunkK / kKbLogical;         // 2 sparse, 4 dense
   // 256-wide K chunks per stage: short token tiles take longer stages (fewer waits per weight byte)
-  static constexpr int kCPS = stage_chunks(kSparse, kBN, kGLU, kCG);
+  static constexpr int kCPS = stage_chunks(kSparse, kBN, kGLU, kCG, kWide);
   static constexpr int kKbps = kCPS * kKbPerChunk;                 // k-blocks per stage
   static constexpr int kCB = kSparse ? kSparseChunkBytes : kDenseChunkBytes;   // packed chunk block
   static constexpr int kCBMeta = 8192;                             // metadata offset in a chunk block
@@ -452,12 +465,13 @@ struct Geo {
 // kNative: the dense control in the activation-stationary orientation -- the tile's 128 token rows
 // are MMA operand A (M = 128, padded when fewer rows are routed) and the weight n-tile is operand
 // B (N = 128); the accumulator then holds a token per TMEM lane and a feature per column.
-template <bool kSparse, int kBN, bool kGLU, int kCG, bool kNative = false>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+template <bool kSparse, int kBN, bool kGLU, int kCG, bool kNative = false, bool kWide = false>
+__global__ void __launch_bounds__(gemm_threads(kWide), 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ CUtensorMap tmap_b64,
                     const __grid_constant__ CUtensorMap tmap_sfb,
                     const GemmParams p) {
-  using G = Geo<kSparse, kBN, kGLU, kCG>;
+  using G = Geo<kSparse, kBN, kGLU, kCG, kWide>;
+  constexpr int kThreads = gemm_threads(kWide);
   constexpr bool kPair = kCG == 2;
   static_assert(!kNative || (!kSparse && kBN == 128 && !kGLU && kCG == 1), "native orientation: dense, 128 tokens");
   extern __shared__ uint8_t smem_raw[];
@@ -504,7 +518,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) { mbar_init(full_bar(s), 2); mbar_init(empty_bar(s), 1); }
     for (int s = 0; s < kNSets; ++s) mbar_init(tfull_bar(s), 4 * kCG);
-    for (int a = 0; a < NACC; ++a) { mbar_init(accf_bar(a), 1); mbar_init(acce_bar(a), 4 * kCG); }
+    for (int a = 0; a < NACC; ++a) { mbar_init(accf_bar(a), 1); mbar_init(acce_bar(a), 4 * kCG * (kWide ? 2 : 1)); }
     mbar_init(drain_bar, 1);
     mbar_init(never_bar, 1);
     ctl->abort = 0;
@@ -547,7 +561,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
   __syncthreads();
   {
     // chunked exclusive scan of tiles_e = ceil(rows_e / BN) * NTt over E experts
-    const int per = (E + kGemmThreads - 1) / kGemmThreads;
+    const int per = (E + kThreads - 1) / kThreads;
     const int e0 = threadIdx.x * per, e1 = min(e0 + per, E);
     int local = 0;
     for (int e = e0; e < e1; ++e) {
@@ -561,7 +575,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
       int n = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += n;
     }
-    __shared__ int wsum[kGemmThreads / 32];
+    __shared__ int wsum[kThreads / 32];
     if (lane == 31) wsum[warp] = incl;
     __syncthreads();
     int before = 0;
@@ -573,14 +587,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
       if (rows < 0) rows = 0;
       run += ((rows + kBN - 1) / kBN) * NTt;
     }
-    if (threadIdx.x == kGemmThreads - 1) pref[E] = before + incl;
+    if (threadIdx.x == kThreads - 1) pref[E] = before + incl;
   }
   // bytes per tile: weights wc, plus ac per token row (codes, scales, output row segment)
   const long long wc = (long long)G::kNT * kCG * kTileN * p.K * (kSparse ? 11 : 18) / 32;
   const long long ac = p.K / 2 + p.K / (kSparse ? 32 : 16) + (long long)G::kNT * kCG * kTileN * (p.y_f32 ? 4 : 2);
   if (p.sched == kSchedRuns) {   // (only the byte-balanced schedule reads the costs; uniform branch)
     // chunked exclusive scan of cost_e = NTt * (ceil(rows_e / BN) * wc + rows_e * ac)
-    const int per = (E + kGemmThreads - 1) / kGemmThreads;
+    const int per = (E + kThreads - 1) / kThreads;
     const int e0 = threadIdx.x * per, e1 = min(e0 + per, E);
     long long local = 0;
     for (int e = e0; e < e1; ++e) {
@@ -593,7 +607,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
       const long long n = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += n;
     }
-    __shared__ long long csum[kGemmThreads / 32];
+    __shared__ long long csum[kThreads / 32];
     if (lane == 31) csum[warp] = incl;
     __syncthreads();
     long long run = incl - local;
@@ -603,7 +617,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
       const int rows = max(offs[e + 1] - offs[e], 0);
       run += (long long)NTt * (((rows + kBN - 1) / kBN) * wc + rows * ac);
     }
-    if (threadIdx.x == kGemmThreads - 1) costp[E] = run;
+    if (threadIdx.x == kThreads - 1) costp[E] = run;
   }
   if (bad) set_status(p.status, GSG_ERR_BAD_ROUTING);
   __syncthreads();
@@ -648,8 +662,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
     uint32_t ph = 0;
     for (int j = 0; j < n_my && !*abort_flag; ++j) {
       const TileDesc c = my_tile(j, ttab, p.tcap, pref, offs, E, kBN, p.sched, tb, unit, nunits);
-      const uint8_t* wsrc = p.w_packed + ((size_t)c.e * NT + c.nt * kCG + rank) * KC * G::kCB;
-      const uint8_t* wsrc_up = wsrc + (size_t)(NT / 2) * KC * G::kCB;   // SwiGLU: the matching up n-tile
+      // this CTA's first weight n-tile: tile c.nt spans n-tiles [c.nt * kCG * kNT, +kCG * kNT) of the
+      // expert (SwiGLU: the gate n-tiles only), CTA r of a pair takes every other one from r
+      const uint8_t* wsrc =
+          p.w_packed + ((size_t)c.e * NT + c.nt * kCG * (kWide ? 2 : 1) + rank) * KC * G::kCB;
+      // its second n-tile: SwiGLU, the matching up n-tile; a wide pair tile, the next pair's
+      const uint8_t* wsrc_up = wsrc + (size_t)(kWide ? kCG : NT / 2) * KC * G::kCB;
       // this CTA's token rows [r0, r0 + cnt): all of the tile's, or for a CTA pair the half of the
       // MMA's N = valid rounded up to 16 that this CTA supplies (rank 1: the upper half)
       const int nh = kPair ? ((c.valid + 15) & ~15) / 2 : kBN;
@@ -700,7 +718,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
         }
       }
     }
-  } else if (warp >= 7) {
+  } else if (warp >= 7 && warp <= 10) {
     // =============================== metadata / scale loaders (TMEM quadrant q = warp % 4)
     const int q = warp & 3;
     const int row = 32 * q + lane;
@@ -840,7 +858,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
       }
     }
   } else {
-    // =============================== epilogue (warps 3..6 -> TMEM lane quadrants 3,0,1,2)
+    // =============================== epilogue (warps 3..6, and 11..14 for wide tiles -> TMEM lane
+    // quadrants 3,0,1,2)
     const int q = warp & 3;
     const float sx = __ldg(p.x_scale);
     int acc = 0;
@@ -942,12 +961,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
       // Each 16-token chunk: TMEM lane (= output feature) -> registers, scale, transpose through
       // the warp's shared buffer into [token][32 features], then 16-byte stores of whole row
       // segments (64 B bf16 / 128 B fp32 per token).
-      uint8_t* obuf = ostage + (size_t)(warp - 3) * kOutStageBytes;
+      uint8_t* obuf = ostage + (size_t)(warp >= 11 ? warp - 7 : warp - 3) * kOutStageBytes;
       const uint32_t obuf_s = smem_u32(obuf);
-      const size_t col0 = ((size_t)c.nt * kCG + rank) * kTileN + 32 * q;   // first feature of this warp
+      // the tile's n-tiles: a wide pair tile's second one goes to warps 11..14
+      const int u_begin = kWide ? (warp >= 11 ? 1 : 0) : 0, u_end = kWide ? u_begin + 1 : G::kNT;
+      for (int u = u_begin; u < u_end; ++u) {
+      // first feature of this warp
+      const size_t col0 = ((size_t)c.nt * kCG * G::kNT + u * kCG + rank) * kTileN + 32 * q;
       for (int c0 = 0; c0 < valid; c0 += 16) {
         float v[16];
-        tc_ld_16(taddr + c0, v);
+        tc_ld_16(taddr + (uint32_t)(u * G::kAccStride) + c0, v);
         if (p.y_f32) {
 #pragma unroll
           for (int j = 0; j < 16; ++j)
@@ -1033,6 +1056,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
         __syncwarp();
       }
       }
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {   // the accumulator may be overwritten (for a pair: once both CTAs read it)
@@ -1076,18 +1100,20 @@ static int g_smem_limit = 232448 - 1024;
 // tcap: capacity of the per-CTA tile table (tiles beyond it are decoded on the fly); an upper
 // bound on a CTA's tiles is ceil((ceil(R/BN) + E) * NT / grid).  cg = 2: a CTA of a pair, which
 // stages half of the tile's token rows (the geometry of Geo<..., 2>).
-static GemmPlan make_plan(bool sparse, int BN, int E, int tcap, bool glu = false, int cg = 1) {
+static GemmPlan make_plan(bool sparse, int BN, int E, int tcap, bool glu = false, int cg = 1, bool wide = false) {
   GemmPlan g;
   g.BN = BN;
   g.tcap = tcap;
-  const int nt = glu ? 2 : 1;   // weight n-tiles per tile (gate + up with the SwiGLU epilogue)
-  g.cps = stage_chunks(sparse, BN, glu, cg);
+  // weight n-tiles per tile and CTA: gate + up with the SwiGLU epilogue, two n-tile pairs for a
+  // wide pair tile
+  const int nt = glu || wide ? 2 : 1;
+  g.cps = stage_chunks(sparse, BN, glu, cg, wide);
   const int kbps = g.cps * (sparse ? 2 : 4);
   const int body =
       g.cps * (BN / cg) * 128 + nt * g.cps * (sparse ? kSparseChunkBytes : kDenseChunkBytes) + kbps * 512;
   g.stage = (body + 1023) / 1024 * 1024;
   // everything but the stage ring and the tile table, at its largest
-  const int ostage = 4 * (glu ? kGluStageBytes : kOutStageBytes);
+  const int ostage = (wide ? 8 : 4) * (glu ? kGluStageBytes : kOutStageBytes);
   const int fixed = 1024 + (2 * kMaxStages + kNSets + 2 * kMaxAcc + 2) * 8 + (int)sizeof(Ctl) + (3 * E + 2) * 4 +
                     16 + (E + 1) * 8 + 16 + ostage;
   int budget = g_smem_limit - fixed;
@@ -1146,21 +1172,22 @@ static EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-template <bool kSparse, int kBN, bool kGLU = false, int kCG = 1, bool kNative = false>
+template <bool kSparse, int kBN, bool kGLU = false, int kCG = 1, bool kNative = false, bool kWide = false>
 static cudaError_t set_attr_one(int bytes) {
-  return cudaFuncSetAttribute(grouped_gemm_kernel<kSparse, kBN, kGLU, kCG, kNative>,
+  return cudaFuncSetAttribute(grouped_gemm_kernel<kSparse, kBN, kGLU, kCG, kNative, kWide>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
 // CTA pairs the device can hold at once at one CTA per SM (the pairs' SMs must share a GPC), per
 // sparse/dense; 0 when the device cannot run them (then 128-token tiles run one CTA per tile).
 static int g_pair_units[2] = {0, 0};
+static int g_wide_units[2] = {0, 0};   // the same for the wide pair tiles
 
-template <bool kSparse>
+template <bool kSparse, bool kWide = false>
 static int max_pairs(int smem) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2);
-  cfg.blockDim = dim3(kGemmThreads);
+  cfg.blockDim = dim3(gemm_threads(kWide));
   cfg.dynamicSmemBytes = (size_t)smem;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1170,7 +1197,8 @@ static int max_pairs(int smem) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_kernel<kSparse, 128, false, 2>, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_kernel<kSparse, 128, false, 2, false, kWide>, &cfg) !=
+      cudaSuccess) {
     cudaGetLastError();   // clear the error: pairs are then simply not used
     return 0;
   }
@@ -1185,17 +1213,21 @@ cudaError_t gemm_set_smem_attrs() {
   if (e != cudaSuccess) return e;
   maxb -= 1024;   // room for the kernels' static shared memory
   g_smem_limit = maxb;
-  cudaError_t errs[14] = {set_attr_one<true, 16>(maxb),       set_attr_one<true, 32>(maxb),
+  cudaError_t errs[16] = {set_attr_one<true, 16>(maxb),       set_attr_one<true, 32>(maxb),
                           set_attr_one<true, 64>(maxb),       set_attr_one<true, 128>(maxb),
                           set_attr_one<false, 16>(maxb),      set_attr_one<false, 32>(maxb),
                           set_attr_one<false, 64>(maxb),      set_attr_one<false, 128>(maxb),
                           set_attr_one<true, 16, true>(maxb), set_attr_one<true, 32, true>(maxb),
                           set_attr_one<true, 64, true>(maxb), set_attr_one<true, 128, false, 2>(maxb),
-                          set_attr_one<false, 128, false, 2>(maxb), set_attr_one<false, 128, false, 1, true>(maxb)};
+                          set_attr_one<false, 128, false, 2>(maxb), set_attr_one<false, 128, false, 1, true>(maxb),
+                          set_attr_one<true, 128, false, 2, false, true>(maxb),
+                          set_attr_one<false, 128, false, 2, false, true>(maxb)};
   for (cudaError_t x : errs)
     if (x != cudaSuccess) return x;
   g_pair_units[1] = max_pairs<true>(maxb);
   g_pair_units[0] = max_pairs<false>(maxb);
+  g_wide_units[1] = max_pairs<true, true>(maxb);
+  g_wide_units[0] = max_pairs<false, true>(maxb);
   return cudaSuccess;
 }
 
@@ -1212,11 +1244,14 @@ static cudaError_t launch_bn(int BN, int grid, size_t smem, cudaStream_t stream,
 template <bool kSparse>
 static cudaError_t launch_bn(int BN, int grid, size_t smem, cudaStream_t stream, const CUtensorMap& tb,
                              const CUtensorMap& tb64, const CUtensorMap& ts, const GemmParams& p, bool glu,
-                             bool pair, bool native = false) {
+                             bool pair, bool native = false, bool wide = false) {
   if (glu) return launch_bn<true, true>(BN, grid, smem, stream, tb, tb64, ts, p);
   if (!kSparse && native)
     return launch_pdl(grouped_gemm_kernel<false, 128, false, 1, true>, grid, kGemmThreads, smem, stream, tb, tb64, ts,
                       p);
+  if (BN == 128 && pair && wide)
+    return launch_pdl_cluster(grouped_gemm_kernel<kSparse, 128, false, 2, false, true>, grid, kGemmThreadsWide, smem,
+                              stream, 2u, tb, tb64, ts, p);
   if (BN == 128 && pair)
     return launch_pdl_cluster(grouped_gemm_kernel<kSparse, 128, false, 2>, grid, kGemmThreads, smem, stream, 2u, tb,
                               tb64, ts, p);
@@ -1240,16 +1275,21 @@ int launch_gemm(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, co
   if (glu && BN > 64) BN = 64;   // two accumulators per tile: 64-token tiles at most
   // 128-token tiles run as CTA pairs (256 weight rows per tile) when N holds whole n-tile pairs
   // and the device can co-schedule pairs
-  const int pair_units = g_pair_units[sparse ? 1 : 0];
+  // a wide pair tile (no combine epilogue, N a multiple of 512) holds two n-tile pairs, 512 weight
+  // rows, and reads its 128 tokens' activations once for both
+  const bool wide = BN == 128 && !glu && !native && comb == nullptr && (N / kTileN) % 4 == 0 &&
+                    g_wide_units[sparse ? 1 : 0] > 0;
+  const int pair_units = wide ? g_wide_units[sparse ? 1 : 0] : g_pair_units[sparse ? 1 : 0];
   const bool pair = BN == 128 && !glu && !native && (N / kTileN) % 2 == 0 && pair_units > 0;
   const int cg = pair ? 2 : 1;
   const int units = pair ? (pair_units < num_sms / 2 ? pair_units : num_sms / 2) : num_sms;   // pairs or CTAs
   const int grid = units * cg;
-  const long long bound = (((long long)R + BN - 1) / BN + E) * (N / kTileN / (glu ? 2 : 1) / cg);
+  const int ntt = glu || (pair && wide) ? 2 : 1;   // weight n-tiles per tile and CTA
+  const long long bound = (((long long)R + BN - 1) / BN + E) * (N / kTileN / ntt / cg);
   // schedule: contiguous byte-balanced runs when every expert fits one token tile (max_rows known)
   // and the CTAs can hold at least 32 tiles each (at most min(E, R) experts are touched), else
   // round-robin
-  const int NTt = N / kTileN / (glu ? 2 : 1) / cg;
+  const int NTt = N / kTileN / ntt / cg;
   const long long touched_max = R < E ? R : E;
   const int sched = (!pair && max_rows > 0 && max_rows <= BN && touched_max * NTt >= 32LL * units) ? kSchedRuns
                                                                                                   : kSchedRoundRobin;
@@ -1263,7 +1303,7 @@ int launch_gemm(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, co
     tcap = (bound + units - 1) / units;
   }
   if (tcap > kMaxTableTiles) tcap = kMaxTableTiles;
-  const GemmPlan g = make_plan(sparse, BN, E, (int)tcap, glu, cg);
+  const GemmPlan g = make_plan(sparse, BN, E, (int)tcap, glu, cg, pair && wide);
   if (g.stages < kNSets || g.smem > (size_t)g_smem_limit) return 1;   // ring too shallow: refuse, launch nothing
   const int box_h = g.BN / cg < 32 ? g.BN / cg : 32;
   const int kbps = g.cps * (sparse ? 2 : 4);
@@ -1305,8 +1345,8 @@ int launch_gemm(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, co
   p.out = comb ? comb->out : nullptr;
   p.k = comb ? comb->k : 1;
   p.stall_ns = g_test_stall_ns.load();
-  const cudaError_t e = sparse ? launch_bn<true>(g.BN, grid, g.smem, stream, tb, tb64, ts, p, glu, pair)
-                               : launch_bn<false>(g.BN, grid, g.smem, stream, tb, tb64, ts, p, false, pair, native);
+  const cudaError_t e = sparse ? launch_bn<true>(g.BN, grid, g.smem, stream, tb, tb64, ts, p, glu, pair, false, wide)
+                               : launch_bn<false>(g.BN, grid, g.smem, stream, tb, tb64, ts, p, false, pair, native, wide);
   return e == cudaSuccess ? 0 : 1;
 }
 
