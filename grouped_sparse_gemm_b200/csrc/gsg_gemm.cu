@@ -278,6 +278,27 @@ __device__ __forceinline__ void tc_mma_dense_pair(uint32_t d, uint64_t adesc, ui
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
       : "memory");
 }
+// 32 accumulator columns of this lane's TMEM row, times `scale`, rounded to bf16 and packed in
+// pairs: h[i] = column 2i (low half) and column 2i + 1 (high half).
+__device__ __forceinline__ void tc_ld_32_bf16(uint32_t taddr, float scale, uint32_t h[16]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(__uint_as_float(r[2 * i]), scale)));
+    const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(__uint_as_float(r[2 * i + 1]), scale)));
+    h[i] = lo | (hi << 16);
+  }
+}
+
 __device__ __forceinline__ void tc_ld_16(uint32_t taddr, float v[16]) {
   uint32_t r[16];
   asm volatile(
@@ -871,6 +892,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
       tc_fence_after();
       const float scale = __fmul_rn(sx, wsc[c.e]);
       const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + kColAcc + (uint32_t)(acc * G::kNT * G::kAccStride);
+      bool released = false;   // the accumulator already handed back to the MMA warp
       if constexpr (kNative) {
         // lane = token 32q + lane of the tile, columns = the n-tile's 128 features: each lane scales
         // and stores its own token's row segment (16-byte stores, 16 features at a time)
@@ -965,7 +987,53 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
       const uint32_t obuf_s = smem_u32(obuf);
       // the tile's n-tiles: a wide pair tile's second one goes to warps 11..14
       const int u_begin = kWide ? (warp >= 11 ? 1 : 0) : 0, u_end = kWide ? u_begin + 1 : G::kNT;
-      for (int u = u_begin; u < u_end; ++u) {
+      if constexpr (kBN == 128 && G::kNT == 1 + (kWide ? 1 : 0)) {
+        if (!p.y_f32 && p.perm_src == nullptr) {
+          // bf16 output of a 128-token tile (one n-tile per warp): the warp's whole accumulator
+          // block in 32-column TMEM loads, held as packed bf16, and the accumulator released
+          // before any store, so the MMA warp's next tile waits for the loads, not for the stores
+          const uint32_t tcol = taddr + (uint32_t)(u_begin * G::kAccStride);
+          const size_t col0 = ((size_t)c.nt * kCG * G::kNT + u_begin * kCG + rank) * kTileN + 32 * q;
+          uint32_t hb[64];
+#pragma unroll
+          for (int h = 0; h < 4; ++h)
+            if (32 * h < valid) tc_ld_32_bf16(tcol + 32u * h, scale, hb + 16 * h);   // warp-uniform
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            if constexpr (kPair) mbar_arrive_cluster(cluster_addr(acce_bar(acc), 0u));
+            else mbar_arrive(acce_bar(acc));
+          }
+          released = true;
+          __nv_bfloat16* Y = static_cast<__nv_bfloat16*>(p.Y);
+#pragma unroll
+          for (int g = 0; g < 8; ++g) {
+            if (16 * g < valid) {   // warp-uniform
+#pragma unroll
+              for (int j = 0; j < 16; j += 2) {
+                const uint32_t w = hb[8 * g + j / 2];
+                asm volatile("st.shared.u16 [%0], %1;" ::"r"(obuf_s + (uint32_t)(j * 64 + lane * 2)),
+                             "h"((unsigned short)(w & 0xffffu)) : "memory");
+                asm volatile("st.shared.u16 [%0], %1;" ::"r"(obuf_s + (uint32_t)((j + 1) * 64 + lane * 2)),
+                             "h"((unsigned short)(w >> 16)) : "memory");
+              }
+              __syncwarp();
+#pragma unroll
+              for (int k = 0; k < 2; ++k) {   // 16 tokens x 4 chunks of 16 B
+                const int ci = lane + 32 * k, tok = ci >> 2, part = ci & 3;
+                if (16 * g + tok < valid) {
+                  uint32_t a, b, cc, d;
+                  lds128(obuf_s + (uint32_t)(tok * 64 + part * 16), a, b, cc, d);
+                  *reinterpret_cast<uint4*>(Y + (size_t)(r0 + 16 * g + tok) * p.N + col0 + part * 8) =
+                      make_uint4(a, b, cc, d);
+                }
+              }
+              __syncwarp();
+            }
+          }
+        }
+      }
+      for (int u = u_begin; u < u_end && !released; ++u) {
       // first feature of this warp
       const size_t col0 = ((size_t)c.nt * kCG * G::kNT + u * kCG + rank) * kTileN + 32 * q;
       for (int c0 = 0; c0 < valid; c0 += 16) {
@@ -1057,11 +1125,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
       }
       }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {   // the accumulator may be overwritten (for a pair: once both CTAs read it)
-        if constexpr (kPair) mbar_arrive_cluster(cluster_addr(acce_bar(acc), 0u));
-        else mbar_arrive(acce_bar(acc));
+      if (!released) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {   // the accumulator may be overwritten (for a pair: once both CTAs read it)
+          if constexpr (kPair) mbar_arrive_cluster(cluster_addr(acce_bar(acc), 0u));
+          else mbar_arrive(acce_bar(acc));
+        }
       }
       if (++acc == NACC) { acc = 0; aph ^= 1u; }
     }
