@@ -473,6 +473,28 @@ class E2EPipeline:
             res.append(a.elapsed_time(b) / reps)
         return res
 
+    def copies_together_ms(self, reps: int = 20) -> float:
+        """Device time per step of the uploads and the download issued together on their two
+        streams (what the pipelined loop overlaps): the host link's two directions at once."""
+        torch.cuda.synchronize()
+        cur = torch.cuda.current_stream()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(cur)
+        self.up.wait_stream(cur)
+        self.down.wait_stream(cur)
+        for _ in range(reps):
+            with torch.cuda.stream(self.up):
+                self.X[0].copy_(self.X_p, non_blocking=True)
+                self.ids[0].copy_(self.ids_p, non_blocking=True)
+                self.gates[0].copy_(self.g_p, non_blocking=True)
+            with torch.cuda.stream(self.down):
+                self.out_p[1].copy_(self.out[1], non_blocking=True)
+        cur.wait_stream(self.up)
+        cur.wait_stream(self.down)
+        b.record(cur)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps
+
 
 # ------------------------------------------------------------------ CPU oracle (baseline / reference arm)
 class OracleSample:
@@ -675,6 +697,7 @@ def run_ours(args, world, rank, local):
         e2e_ms = max_over_ranks(pipe.run(max(10, args.steps // 10)), world, dev)
         host_ms = pipe.host_ms
         h2d_ms, d2h_ms = pipe.copy_ms()
+        both_ms = pipe.copies_together_ms()
 
         # the same calls one step at a time (copies, step, copy back), L2 flushed before each
         def e2e_step():
@@ -691,7 +714,7 @@ def run_ours(args, world, rank, local):
                        "uploads and downloads overlap neighbouring steps' compute; weights rotate over 3 "
                        "replicas, no L2 flush",
                "parts_us": {"host_issue_per_step": host_ms * 1e3, "h2d_alone": h2d_ms * 1e3,
-                            "d2h_alone": d2h_ms * 1e3},
+                            "d2h_alone": d2h_ms * 1e3, "h2d_and_d2h_together": both_ms * 1e3},
                "serial": {"value": job_value(flops, world, serial_ms), "ms_per_step": serial_ms,
                           "how": "one step at a time, every stream joined before the end event, L2 flushed "
                                  "before each step"}}
