@@ -316,12 +316,22 @@ def test_sparse_gemm_oracle_inputs(gsg, counts, N, K, hint):
     tl.assert_gemm_close(y[:c["R"]], y_ref, bound, f"sparse {counts} hint {hint}")
 
 
-@pytest.mark.parametrize("counts,N,K", GEMM_CASES[:3])
-def test_sparse_gemm_bf16_output(gsg, counts, N, K):
-    c = _gemm_case(counts, N, K, sparse=True)
-    y = _run_gemm(gsg, c, True, -1, torch.bfloat16)
-    y_ref, bound = tl.reference_rows(np.arange(c["R"]), c["off"], c["q"], c["sc"], 32, c["canon"], c["s_x"], c["sws"])
-    tl.assert_gemm_close(y[:c["R"]], y_ref, bound, "sparse bf16")
+@pytest.mark.parametrize("counts,N,K", GEMM_CASES)
+@pytest.mark.parametrize("sparse", [True, False])
+def test_gemm_bf16_output(gsg, counts, N, K, sparse):
+    """bf16 output of every tile shape (128-token tiles, CTA pairs and wide pair tiles included, whose
+    epilogue packs the accumulator into bf16 pairs in registers): within the bound, and exactly the
+    fp32 output rounded once to bf16."""
+    c = _gemm_case(counts, N, K, sparse=sparse)
+    y = _run_gemm(gsg, c, sparse, -1, torch.bfloat16)
+    y32 = _run_gemm(gsg, c, sparse, -1, torch.float32)
+    torch.cuda.synchronize()
+    _status_ok(gsg)
+    sf = 32 if sparse else 16
+    y_ref, bound = tl.reference_rows(np.arange(c["R"]), c["off"], c["q"], c["sc"], sf, c["canon"], c["s_x"], c["sws"],
+                                     sparse=sparse, w_sf=sf)
+    tl.assert_gemm_close(y[:c["R"]], y_ref, bound, f"{'sparse' if sparse else 'dense'} bf16 {counts}")
+    assert torch.equal(y[:c["R"]], y32[:c["R"]].to(torch.bfloat16))
 
 
 @pytest.mark.parametrize("counts,N,K", GEMM_CASES)
