@@ -47,6 +47,7 @@ EXPORTED_SYMBOLS = [
     "gsg_unpermute_scale", "gsg_get_device_status", "gsg_status_string", "gsg_version",
     "gsg_moe_route_permute_noalloc", "gsg_grouped_sparse_gemm_swiglu", "gsg_grouped_sparse_gemm_combine",
     "gsg_moe_dispatch_nvfp4", "gsg_test_set_gemm_stall_ns", "gsg_grouped_dense_gemm_native",
+    "gsg_test_set_gemm_table_cap",
 ]
 
 _STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported shape", -3: "CUDA error",
@@ -100,6 +101,7 @@ def load_library(build_if_missing: bool = False) -> ctypes.CDLL:
         "gsg_grouped_sparse_gemm_swiglu": (i, [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp, vp, vp, vp]),
         "gsg_grouped_sparse_gemm_combine": (i, [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, vp, vp, sz, vp, vp]),
         "gsg_test_set_gemm_stall_ns": (None, [ctypes.c_ulonglong]),
+        "gsg_test_set_gemm_table_cap": (None, [ctypes.c_int]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)

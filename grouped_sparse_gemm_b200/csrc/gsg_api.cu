@@ -368,5 +368,6 @@ const char* gsg_status_string(gsg_status_t s) {
 int gsg_version(void) { return 1; }
 
 void gsg_test_set_gemm_stall_ns(unsigned long long ns) { gsg::gemm_set_test_stall(ns); }
+void gsg_test_set_gemm_table_cap(int tiles) { gsg::gemm_set_test_table_cap(tiles); }
 
 }  // extern "C"

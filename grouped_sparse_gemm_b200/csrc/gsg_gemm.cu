@@ -1213,6 +1213,10 @@ constexpr int kMaxTableTiles = 1024;
 // test hook: the MMA warp's stall of GemmParams::stall_ns for the launches that follow (0 = off)
 static std::atomic<unsigned long long> g_test_stall_ns{0ull};
 void gemm_set_test_stall(unsigned long long ns) { g_test_stall_ns.store(ns); }
+// test hook: at most this many entries of the per-CTA tile table (-1 = no limit); the tiles past
+// it are decoded from the expert offsets as the roles reach them
+static std::atomic<int> g_test_table_cap{-1};
+void gemm_set_test_table_cap(int cap) { g_test_table_cap.store(cap); }
 
 // Token tile: the smallest of 16/32/64 that holds the largest expert; past 64 rows, 128 only when
 // experts average at least 64 rows (R / E), since a 128-row activation chunk takes shared memory
@@ -1373,6 +1377,8 @@ int launch_gemm(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, co
     tcap = (bound + units - 1) / units;
   }
   if (tcap > kMaxTableTiles) tcap = kMaxTableTiles;
+  const int tcap_test = g_test_table_cap.load();
+  if (tcap_test >= 0 && tcap > tcap_test) tcap = tcap_test;
   const GemmPlan g = make_plan(sparse, BN, E, (int)tcap, glu, cg, pair && wide);
   if (g.stages < kNSets || g.smem > (size_t)g_smem_limit) return 1;   // ring too shallow: refuse, launch nothing
   const int box_h = g.BN / cg < 32 ? g.BN / cg : 32;

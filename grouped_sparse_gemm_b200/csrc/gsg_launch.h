@@ -61,6 +61,8 @@ bool gemm_supported(int E);
 // test hook: GEMM launches after this call stall their MMA warp for `ns` on a barrier nothing
 // arrives on (0 = off); see GemmParams::stall_ns
 void gemm_set_test_stall(unsigned long long ns);
+// test hook: GEMM launches after this call keep at most `cap` tile-table entries per CTA (-1 = off)
+void gemm_set_test_table_cap(int cap);
 int gemm_pick_bn(int max_rows, int R, int E);
 cudaError_t gemm_set_smem_attrs();
 int launch_gemm(bool sparse, const uint8_t* a_codes, const uint8_t* a_scales, const float* x_scale,

@@ -301,6 +301,16 @@ gsg_status_t gsg_moe_route_permute_noalloc(const int32_t* topk_ids, int T, int k
 void gsg_test_set_gemm_stall_ns(unsigned long long ns);
 
 /* ----------------------------------------------------------------------------------------
+ * gsg_test_set_gemm_table_cap -- test hook for the grouped GEMM's tile bookkeeping.  Not a step of
+ * the method.  Every CTA of a grouped GEMM decodes the list of its tiles (expert, n-tile, token
+ * rows) from the expert offsets once, into a table in shared memory; a CTA with more tiles than
+ * the table holds decodes the rest as it reaches them.  tiles >= 0: launches afterwards keep at
+ * most `tiles` table entries, so that path runs at any size (results are bit-identical); -1 (the
+ * default) switches the hook off.  Process-wide: set it only while no other thread launches.
+ */
+void gsg_test_set_gemm_table_cap(int tiles);
+
+/* ----------------------------------------------------------------------------------------
  * Status.  gsg_get_device_status synchronizes `stream`, returns the device status word of the
  * current device and clears it.  gsg_status_string never returns NULL.
  */

@@ -407,6 +407,30 @@ def test_gemm_wait_timeout_aborts_cleanly(gsg, sparse, counts):
     tl.assert_gemm_close(y[:c["R"]], y_ref, bound, "after a timed-out launch")
 
 
+@pytest.mark.parametrize("sparse", [True, False])
+@pytest.mark.parametrize("counts,N,K", [GEMM_CASES[2], GEMM_CASES[4], GEMM_CASES[5]])
+def test_gemm_tiles_decoded_without_table(gsg, sparse, counts, N, K):
+    """Tiles past a CTA's tile table are decoded from the expert offsets as the roles reach them
+    (the path of launches with more tiles per CTA than the table holds): with the table capped at
+    0 and 1 entries the result is bit-identical to the normal launch and within the bound."""
+    c = _gemm_case(counts, N, K, sparse=sparse)
+    y0 = _run_gemm(gsg, c, sparse, -1, torch.float32)
+    L = gsg.lib()
+    try:
+        for cap in (0, 1):
+            L.gsg_test_set_gemm_table_cap(cap)
+            y = _run_gemm(gsg, c, sparse, -1, torch.float32)
+            torch.cuda.synchronize()
+            _status_ok(gsg)
+            assert torch.equal(y[:c["R"]], y0[:c["R"]]), f"table cap {cap}"
+    finally:
+        L.gsg_test_set_gemm_table_cap(-1)
+    sf = 32 if sparse else 16
+    y_ref, bound = tl.reference_rows(np.arange(c["R"]), c["off"], c["q"], c["sc"], sf, c["canon"], c["s_x"],
+                                     c["sws"], sparse=sparse, w_sf=sf)
+    tl.assert_gemm_close(y0[:c["R"]], y_ref, bound, "with the full tile table")
+
+
 def test_dense_and_sparse_agree_on_48_weights(gsg):
     """The control differs from the sparse kernel only in sparsity: a W that is already paired
     4:8 gives results within tolerance of one reference on both (32-blocks copied into 16-blocks)."""

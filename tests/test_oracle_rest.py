@@ -175,6 +175,26 @@ def test_layout_round_trips_and_handworked_positions():
     s1 = np.zeros((128, 8), np.uint8)
     s1[33, 6] = 77              # row 33, k-block 1, block 2 -> 512 + 16*1 + 4*1 + 2
     assert layout.tile_scales(s1).reshape(-1)[512 + 22] == 77
+    # metadata: n-tile 1, row 2, 8-group 37 = chunk 1, group 5 -> (1*2 + 1)*2048 + 2*16 + 5//2 = 6178,
+    # high nibble (odd group)
+    m1 = np.zeros((256, 64), np.uint8)
+    m1[130, 37] = 0x9
+    tm = layout.tile_meta(m1).reshape(-1)
+    assert tm[6178] == 0x90 and int(tm.astype(np.int64).sum()) == 0x90
+    # a whole sparse chunk block (N=128, K=512: two chunk blocks of 11264 bytes), worked by hand:
+    # value 200 of row 5 = chunk 1, k-block 1, stored value 8 -> byte 4096 + 5*16 + 4 = 4180 (low nibble);
+    # 8-group 40 of row 5 = chunk 1, group 8 -> 8192 + 5*16 + 4 = 8276 (low nibble);
+    # 32-block 9 of row 100 = chunk 1, k-block 0, block 1 -> 10240 + 16*(100%32) + 4*(100//32) + 1 = 10317
+    cv = np.zeros((128, 256), np.uint8)
+    cv[5, 200] = 0x3
+    pt = np.zeros((128, 64), np.uint8)
+    pt[5, 40] = 0x6
+    scs = np.zeros((128, 16), np.uint8)
+    scs[100, 9] = 0x55
+    blk = layout.packed_sparse(cv, pt, scs)
+    assert blk.shape == (1, 2, 11264)
+    assert blk[0, 1, 4180] == 0x03 and blk[0, 1, 8276] == 0x06 and blk[0, 1, 10317] == 0x55
+    assert int(blk.astype(np.int64).sum()) == 0x03 + 0x06 + 0x55
     # quad activation scales: entry (kb, r, c, j) = scale of row r + 32c
     R = 70
     asc = rng.integers(1, 127, size=(R, 8)).astype(np.uint8)
