@@ -439,7 +439,9 @@ __device__ __forceinline__ int tile_at_cost(long long target, const long long* c
 
 // 256-wide K chunks per ring stage: short token tiles take longer stages (fewer waits per weight
 // byte); 128-token tiles keep two-chunk stages, also on CTA pairs (three-chunk stages, three of
-// them in shared memory, measured slower than five two-chunk stages).
+// them in shared memory, measured slower than five two-chunk stages).  Wide pair tiles: two-chunk
+// stages for the sparse weights (three 62 KB stages; six one-chunk stages measured slower), one
+// chunk for the dense control's larger blocks.
 __host__ __device__ constexpr int stage_chunks(bool sparse, int BN, bool glu, int cg, bool wide = false) {
   return wide ? (sparse ? 2 : 1) : glu ? 2 : sparse ? (BN <= 32 ? 3 : 2) : (BN <= 32 ? 2 : 1);
 }
