@@ -488,6 +488,82 @@ struct Geo {
 // kNative: the dense control in the activation-stationary orientation -- the tile's 128 token rows
 // are MMA operand A (M = 128, padded when fewer rows are routed) and the weight n-tile is operand
 // B (N = 128); the accumulator then holds a token per TMEM lane and a feature per column.
+// Combine epilogue, second phase: once every CTA of the launch has written its routed rows to their
+// token slots (a bounded grid barrier on two counters of the workspace: every CTA is resident, one
+// per SM), the CTAs sum each token's k slots in j order -- the scatter's arithmetic: fp32 products
+// and running sum from 0, one bf16 rounding, eight outputs per thread (16-byte slot loads, the
+// token's slots all in flight).  The last CTA to leave sets both counters back to zero.
+__device__ void combine_tokens(const GemmParams& p, volatile int* abort_flag) {
+  __shared__ int go;
+  int* arrive = p.counters;
+  int* depart = p.counters + 1;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();   // this CTA's slot stores before its arrival
+    atomicAdd(arrive, 1);
+    const uint64_t t0 = globaltimer_ns();
+    int ok = 1;
+    while (*reinterpret_cast<volatile int*>(arrive) < (int)gridDim.x) {
+      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+        set_status(p.status, GSG_ERR_DEVICE_TIMEOUT);
+        ok = 0;
+        break;
+      }
+    }
+    __threadfence();   // the other CTAs' slot stores before this CTA's loads
+    go = ok && !*abort_flag;
+  }
+  __syncthreads();
+  if (go) {
+    const int T = p.R / p.k;
+    const unsigned n8 = (unsigned)p.N / 8u;
+    const unsigned total = (unsigned)T * n8;   // T * N / 8 < 2^31 (checked on the host)
+    const uint16_t* slots = static_cast<const uint16_t*>(p.Y);
+    for (unsigned u = blockIdx.x * blockDim.x + threadIdx.x; u < total; u += gridDim.x * blockDim.x) {
+      const int t = int(u / n8), c = int(u % n8);
+      float acc[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[q] = 0.0f;
+      for (int j0 = 0; j0 < p.k; j0 += 8) {
+        float g[8];
+        uint4 v[8];
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const bool in = j0 + jj < p.k;
+          g[jj] = in ? __ldg(p.gates + (size_t)t * p.k + j0 + jj) : 0.0f;
+          v[jj] = in ? __ldcg(reinterpret_cast<const uint4*>(slots + ((size_t)t * p.k + j0 + jj) * p.N) + c)
+                     : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          if (j0 + jj >= p.k) break;
+          const uint32_t w[4] = {v[jj].x, v[jj].y, v[jj].z, v[jj].w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            acc[2 * q] = __fadd_rn(acc[2 * q], __fmul_rn(g[jj], __uint_as_float(w[q] << 16)));
+            acc[2 * q + 1] = __fadd_rn(acc[2 * q + 1], __fmul_rn(g[jj], __uint_as_float(w[q] & 0xFFFF0000u)));
+          }
+        }
+      }
+      uint32_t o[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * q]));
+        const uint32_t hi = __bfloat16_as_ushort(__float2bfloat16_rn(acc[2 * q + 1]));
+        o[q] = lo | (hi << 16);
+      }
+      reinterpret_cast<uint4*>(p.out + (size_t)t * p.N)[c] = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (atomicAdd(depart, 1) == (int)gridDim.x - 1) {   // every CTA has passed the barrier
+      *reinterpret_cast<volatile int*>(arrive) = 0;
+      *reinterpret_cast<volatile int*>(depart) = 0;
+    }
+  }
+}
+
 template <bool kSparse, int kBN, bool kGLU, int kCG, bool kNative = false, bool kWide = false>
 __global__ void __launch_bounds__(gemm_threads(kWide), 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_constant__ CUtensorMap tmap_b64,
@@ -1068,7 +1144,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
           // slot f instead of row r
           const bool comb = p.perm_src != nullptr;
           int myf = (comb && lane < 16 && c0 + lane < valid) ? __ldg(p.perm_src + r0 + c0 + lane) : 0;
-          // a slot index outside [0, T*k) (corrupt routing) gets nothing stored or counted
+          // a slot index outside [0, T*k) (corrupt routing) gets nothing stored
           const unsigned badf = __ballot_sync(0xffffffffu, comb && lane < 16 && c0 + lane < valid &&
                                                                (myf < 0 || myf >= p.R));
           if (badf != 0u && lane == 0) set_status(p.status, GSG_ERR_BAD_ROUTING);
@@ -1082,44 +1158,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
               lds128(obuf_s + (uint32_t)(tok * 64 + part * 16), a, b, cc, d);
               const size_t dst = comb ? (size_t)f : (size_t)(r0 + c0 + tok);
               *reinterpret_cast<uint4*>(Y + dst * p.N + col0 + part * 8) = make_uint4(a, b, cc, d);
-            }
-          }
-          if (comb) {
-            // count this warp's 32 features of each chunk row towards its token; the warp that
-            // brings a token's count to k reduces the token's k slots in j order (the scatter's
-            // arithmetic: fp32 products and sum, j ascending, one bf16 rounding)
-            asm volatile("fence.acq_rel.gpu;" ::: "memory");   // this lane's slot stores before the count
-            __syncwarp();
-            const int g32 = (int)(col0 >> 5), ng32 = p.N >> 5;
-            bool last = false;
-            if (lane < 16 && c0 + lane < valid && !((badf >> lane) & 1u)) {
-              const int t = myf / p.k;
-              last = atomicAdd(p.counters + (size_t)t * ng32 + g32, 1) == p.k - 1;
-            }
-            unsigned todo = __ballot_sync(0xffffffffu, last);
-            if (todo) asm volatile("fence.acq_rel.gpu;" ::: "memory");   // the other slots' stores
-            while (todo) {
-              const int j = __ffs(todo) - 1;
-              todo &= todo - 1;
-              const int t = __shfl_sync(0xffffffffu, myf, j) / p.k;
-              float accum = 0.0f;
-              for (int j0 = 0; j0 < p.k; j0 += 8) {   // eight slots' loads in flight, then the sum in order
-                float gt[8];
-                unsigned short yb[8];
-#pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {
-                  const bool in = j0 + jj < p.k;
-                  gt[jj] = in ? __ldg(p.gates + (size_t)t * p.k + j0 + jj) : 0.0f;
-                  yb[jj] = in ? __ldcg(reinterpret_cast<const unsigned short*>(Y) + ((size_t)t * p.k + j0 + jj) * p.N +
-                                       col0 + lane)
-                              : (unsigned short)0;
-                }
-#pragma unroll
-                for (int jj = 0; jj < 8; ++jj)
-                  if (j0 + jj < p.k) accum = __fadd_rn(accum, __fmul_rn(gt[jj], __uint_as_float((uint32_t)yb[jj] << 16)));
-              }
-              p.out[(size_t)t * p.N + col0 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(accum));
-              if (lane == 0) p.counters[(size_t)t * ng32 + g32] = 0;
             }
           }
         }
@@ -1156,6 +1194,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, const __grid_con
     else
       asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
   }
+  if (p.perm_src != nullptr) combine_tokens(p, abort_flag);
 }
 
 // ------------------------------------------------------------------ host side

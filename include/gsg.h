@@ -234,11 +234,10 @@ gsg_status_t gsg_grouped_sparse_gemm_swiglu(const uint8_t* a_codes, const uint8_
  * launch, with the same result bit for bit.
  * Paper: §D.1 (p.19): the serving integration fuses dispatch and scatter into the expert GEMMs.
  * Every routed row is written (bf16, as Y would hold it) to its token slot f = t*k + j of the
- * workspace instead of row r; each epilogue warp then counts its 32 features of the row towards
- * token t, and the warp that completes a token's k contributions computes
+ * workspace instead of row r; once every CTA of the launch has written its rows (a bounded grid
+ * barrier on two of the workspace's counters), the CTAs compute
  *     out[t][n] = bf16_rne( sum_{j<k} fp32(gates[t][j] * slot[t*k + j][n]) )   (j ascending, from 0)
- * -- the scatter's arithmetic and order, so the result does not depend on which warp finishes
- * last.  R = T*k routed rows; perm_src int32 [R] and expert_offsets from gsg_moe_route_permute;
+ * -- the scatter's arithmetic and order.  R = T*k routed rows; perm_src int32 [R] and expert_offsets from gsg_moe_route_permute;
  * gates fp32 [T][k]; out bf16 [T][N].  A routed row whose perm_src entry lies outside [0, T*k)
  * is skipped (nothing stored for it) and sets GSG_ERR_BAD_ROUTING.
  * workspace: gsg_workspace_size(GSG_OP_COMBINE, E, N, K, T, k) bytes, 16-byte aligned: the slots

@@ -639,7 +639,7 @@ def test_combine_gemm_equals_gemm_then_unpermute(gsg, name):
 
 
 def test_combine_skips_corrupt_slot_indices(gsg):
-    """perm_src entries outside [0, T*k) are skipped by the combine epilogue (no store, no count)
+    """perm_src entries outside [0, T*k) are skipped by the combine epilogue (nothing stored)
     and reported as GSG_ERR_BAD_ROUTING; every token none of whose rows was corrupted still gets
     the scatter's result bit for bit."""
     cfg = inputs.custom_config("cc", E=6, K=512, N=256, T=48, top_k=4, routing="zipf", zipf_s=1.2)
