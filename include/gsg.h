@@ -70,7 +70,7 @@ enum {
   GSG_OP_ROUTE = 3,
   GSG_OP_QUANTIZE = 4,
   GSG_OP_GEMM = 5,
-  GSG_OP_COMBINE = 6,   /* gsg_grouped_sparse_gemm_combine: token slots + completion counters */
+  GSG_OP_COMBINE = 6,   /* gsg_grouped_sparse_gemm_combine: token slots + barrier counters    */
   GSG_OP_DISPATCH = 7   /* gsg_moe_dispatch_nvfp4: routing workspace + quantizer workspace    */
 };
 
@@ -241,9 +241,9 @@ gsg_status_t gsg_grouped_sparse_gemm_swiglu(const uint8_t* a_codes, const uint8_
  * gates fp32 [T][k]; out bf16 [T][N].  A routed row whose perm_src entry lies outside [0, T*k)
  * is skipped (nothing stored for it) and sets GSG_ERR_BAD_ROUTING.
  * workspace: gsg_workspace_size(GSG_OP_COMBINE, E, N, K, T, k) bytes, 16-byte aligned: the slots
- * bf16 [T*k][N] and then int32 completion counters [T][N/32].  The counters must be zero before
- * the first call (e.g. allocate the workspace zeroed); every call that completes leaves them zero
- * again, so a workspace can be reused call after call.  After a device error the outputs and the
+ * bf16 [T*k][N] and then int32 counters [T][N/32] (the first two count the CTAs through the grid
+ * barrier).  The counters must be zero before the first call (e.g. allocate the workspace zeroed);
+ * every call that completes leaves them zero again, so a workspace can be reused call after call.  After a device error the outputs and the
  * counters are unspecified: zero the workspace again.  Calls that share a workspace must not run
  * concurrently.
  */

@@ -606,7 +606,7 @@ def test_moe_layer_pipeline(gsg, name):
 @pytest.mark.parametrize("name", ["tiny", "30b_down_decode", "1t_down_decode_b1", "dup"])
 def test_combine_gemm_equals_gemm_then_unpermute(gsg, name):
     """The fused combine is the unfused GEMM (bf16 Y) + scatter bit for bit, on every token, and
-    it leaves its completion counters at zero so the workspace can be reused."""
+    it leaves its counters at zero so the workspace can be reused."""
     if name == "dup":     # a token that picks the same expert twice, and uneven expert loads
         cfg = inputs.custom_config("dup", E=5, K=512, N=256, T=40, top_k=3, routing="zipf", zipf_s=1.5)
         ids = inputs.routing(cfg)
