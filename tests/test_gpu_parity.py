@@ -638,6 +638,33 @@ def test_combine_gemm_equals_gemm_then_unpermute(gsg, name):
     np.testing.assert_array_equal(out.cpu().view(torch.uint16).numpy(), oref)
 
 
+def test_combine_wait_timeout_then_clean_call(gsg):
+    """The combine's abort path: with the timeout hook the launch returns GSG_ERR_DEVICE_TIMEOUT (its
+    CTAs still pass the grid barrier and reset its counters); the next normal call on the same
+    workspace is the scatter's result bit for bit and leaves the counters at zero."""
+    cfg = inputs.custom_config("ct", E=6, K=512, N=256, T=48, top_k=4, routing="zipf", zipf_s=1.2)
+    ids = inputs.routing(cfg)
+    X, g = inputs.activations(cfg).to(DEV), inputs.gates(cfg).to(DEV)
+    w = gsg.pack_sparse_nvfp4(inputs.all_weights(cfg).to(DEV))
+    r = gsg.moe_route_permute(ids.to(DEV), cfg.E)
+    qa = gsg.quantize_act_nvfp4(X, 32, r.inv_perm, cfg.top_k)
+    ref = gsg.unpermute_scale(gsg.grouped_sparse_gemm(qa, w, r.offsets), r.inv_perm, g, cfg.top_k)
+    ws = gsg.combine_workspace(cfg.E, cfg.N, cfg.K, cfg.T, cfg.top_k, DEV)
+    L = gsg.lib()
+    try:
+        L.gsg_test_set_gemm_stall_ns(1_000_000)
+        gsg.grouped_sparse_gemm_combine(qa, w, r, g, ws)
+        assert gsg.get_device_status() == -6
+    finally:
+        L.gsg_test_set_gemm_stall_ns(0)
+    slots = cfg.T * cfg.top_k * cfg.N * 2
+    assert not ws[(slots + 255) // 256 * 256:].any()          # the barrier's counters back at zero
+    out = gsg.grouped_sparse_gemm_combine(qa, w, r, g, ws)
+    _status_ok(gsg)
+    assert torch.equal(out, ref)
+    assert not ws[(slots + 255) // 256 * 256:].any()
+
+
 def test_combine_skips_corrupt_slot_indices(gsg):
     """perm_src entries outside [0, T*k) are skipped by the combine epilogue (nothing stored)
     and reported as GSG_ERR_BAD_ROUTING; every token none of whose rows was corrupted still gets
