@@ -592,6 +592,12 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def tensor_roof_binds(flops: float, nbytes: float, tensor_tflops: float, hbm_gbs: float) -> bool:
+    """The binding roof of a launch: the tensor pipe when its flops at the tensor peak take longer
+    than its bytes at the HBM peak (past the ridge point), else HBM."""
+    return flops / (tensor_tflops * 1e12) > nbytes / (hbm_gbs * 1e9)
+
+
 def traffic_from_profiles(config_name: str, algorithmic_bytes: int):
     """DRAM bytes per GEMM launch from the committed ncu summary, if the kernel is unchanged.
     An entry captured on a smaller case of the same instantiation ("scaled_from") is scaled to
@@ -675,7 +681,7 @@ def run_ours(args, world, rank, local):
     gemm_tflops = flops / (gemm_ms * 1e-3) / 1e12
     # the binding roof: the larger of the two lower bounds on the launch's time (the tensor roof
     # binds only past the ridge point, e.g. the 65,536-token 1T prefill)
-    tensor_bound = flops / (tensor_peak * 1e12) > gemm_bytes / (hbm_peak * 1e9)
+    tensor_bound = tensor_roof_binds(flops, gemm_bytes, tensor_peak, hbm_peak)
 
     # the same number of bytes read by a plain library reduction (torch int64 sum) on the same
     # harness (flush, in-graph events): what a bare read of the GEMM's traffic achieves at this size
@@ -919,7 +925,7 @@ def run_all_configs(args, local):
         res.update({"gemm_tflops": flops / g_s / 1e12, "gemm_weight_gbs": w / g_s / 1e9,
                     "gemm_total_gbs": (w + a + y) / g_s / 1e9, "gemm_hbm_frac": (w + a + y) / g_s / 1e9 / hbm,
                     "gemm_tensor_frac": flops / g_s / 1e12 / tensor,
-                    "binding_roof": "tensor" if flops / (tensor * 1e12) > (w + a + y) / (hbm * 1e9) else "hbm",
+                    "binding_roof": "tensor" if tensor_roof_binds(flops, w + a + y, tensor, hbm) else "hbm",
                     "dense_gemm_gbs": wl.dense_gemm_bytes() / (res["dense_gemm_us"] * 1e-6) / 1e9,
                     "sparse_speedup": res["dense_gemm_us"] / res["gemm_us"],
                     "sparse_speedup_vs_native": res["dense_native_gemm_us"] / res["gemm_us"],

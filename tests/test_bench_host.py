@@ -54,3 +54,20 @@ def test_cpu_sample_size():
     assert bench.cpu_sample_experts(inputs.CONFIGS["30b_up_prefill"], None) == 24
     assert bench.cpu_sample_experts(inputs.CONFIGS["1t_up_prefill"], None) == 4
     assert bench.cpu_sample_experts(inputs.CONFIGS["1t_up_prefill"], 7) == 7
+
+
+def test_binding_roof_of_the_workloads():
+    """HBM binds every expert-projection workload; the tensor pipe binds the 65,536-token extra
+    (the roofs: measured bf16 burst x 8 and the measured HBM copy, or the fallback figures)."""
+    peaks, _ = bench.measured_peaks()
+    tensor, hbm = float(peaks["bf16_tflops"]) * 8.0, float(peaks["hbm_gbs"])
+    for name, cfg in inputs.CONFIGS.items():
+        touched = min(cfg.E, cfg.R)
+        nbytes = touched * cfg.N * cfg.K * 11 // 32 + cfg.R * cfg.K // 2 + cfg.R * cfg.K // 32 + cfg.R * cfg.N * 2
+        flops = 2.0 * cfg.R * cfg.N * cfg.K
+        assert bench.tensor_roof_binds(flops, nbytes, tensor, hbm) == name.startswith("1t_up_prefill_65k"), name
+    # the ridge point: flop/B = tensor / hbm
+    ridge = tensor * 1e12 / (hbm * 1e9)
+    assert bench.tensor_roof_binds(1.01 * ridge, 1.0, tensor, hbm)
+    assert not bench.tensor_roof_binds(0.99 * ridge, 1.0, tensor, hbm)
+
