@@ -298,6 +298,7 @@ gsg_status_t gsg_grouped_sparse_gemm_combine(const uint8_t* a_codes, const uint8
   if (T < 0 || k < 1) return GSG_ERR_INVALID_ARG;
   if (!weight_shape_ok(E, N, K) || !gsg::gemm_supported(E)) return GSG_ERR_UNSUPPORTED_SHAPE;
   if ((long long)T * k > (1ll << 30)) return GSG_ERR_UNSUPPORTED_SHAPE;
+  if ((long long)T * (N / 8) >= (1ll << 31)) return GSG_ERR_UNSUPPORTED_SHAPE;   // token sums: 32-bit unit index
   if (T == 0) return GSG_OK;
   const int R = T * k;
   if (!a_codes || !a_scales || !x_tensor_scale || !w_packed || !w_tensor_scale || !expert_offsets || !perm_src ||

@@ -237,9 +237,10 @@ gsg_status_t gsg_grouped_sparse_gemm_swiglu(const uint8_t* a_codes, const uint8_
  * workspace instead of row r; once every CTA of the launch has written its rows (a bounded grid
  * barrier on two of the workspace's counters), the CTAs compute
  *     out[t][n] = bf16_rne( sum_{j<k} fp32(gates[t][j] * slot[t*k + j][n]) )   (j ascending, from 0)
- * -- the scatter's arithmetic and order.  R = T*k routed rows; perm_src int32 [R] and expert_offsets from gsg_moe_route_permute;
- * gates fp32 [T][k]; out bf16 [T][N].  A routed row whose perm_src entry lies outside [0, T*k)
- * is skipped (nothing stored for it) and sets GSG_ERR_BAD_ROUTING.
+ * -- the scatter's arithmetic and order.  R = T*k routed rows; perm_src int32 [R] and
+ * expert_offsets from gsg_moe_route_permute; gates fp32 [T][k]; out bf16 [T][N] (T*N/8 < 2^31,
+ * else GSG_ERR_UNSUPPORTED_SHAPE).  A routed row whose perm_src entry lies outside [0, T*k) is
+ * skipped (nothing stored for it) and sets GSG_ERR_BAD_ROUTING.
  * workspace: gsg_workspace_size(GSG_OP_COMBINE, E, N, K, T, k) bytes, 16-byte aligned: the slots
  * bf16 [T*k][N] and then int32 counters [T][N/32] (the first two count the CTAs through the grid
  * barrier).  The counters must be zero before the first call (e.g. allocate the workspace zeroed);

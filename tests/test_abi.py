@@ -83,6 +83,12 @@ def test_host_argument_checks(L):
     assert L.gsg_quantize_act_nvfp4(P, 4, 256, 32, P, 2, None, P, P, P, None, 0, None) == -7
     assert L.gsg_unpermute_scale(P, P, P, 4, 2, 12, P, None) == -1
     assert L.gsg_unpermute_scale(P, P, P, 0, 2, 128, P, None) == 0
+    # the GEMM with the combine: bad k, bad N, too many token sums for a 32-bit index, NULL gates
+    assert L.gsg_grouped_sparse_gemm_combine(P, P, P, P, P, P, 4, 256, 256, 8, 0, -1, P, P, P, 1 << 20, P, None) == -1
+    assert L.gsg_grouped_sparse_gemm_combine(P, P, P, P, P, P, 4, 200, 256, 8, 2, -1, P, P, P, 1 << 20, P, None) == -2
+    assert L.gsg_grouped_sparse_gemm_combine(P, P, P, P, P, P, 4, 32768, 256, 1 << 20, 1, -1, P, P, P, 1 << 20, P,
+                                             None) == -2
+    assert L.gsg_grouped_sparse_gemm_combine(P, P, P, P, P, P, 4, 256, 256, 8, 2, -1, P, None, P, 1 << 20, P, None) == -1
     # two-phase scale path (R*K >= 2^27): its workspace is needed even with a caller-supplied s_x
     assert L.gsg_quantize_act_nvfp4(P, 2048, 8192, 32, P, 8, P, P, P, P, None, 0, None) == -7
     # the combined routing + quantize call: the checks of both calls, and its own workspace
