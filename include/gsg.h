@@ -244,9 +244,9 @@ gsg_status_t gsg_grouped_sparse_gemm_swiglu(const uint8_t* a_codes, const uint8_
  * workspace: gsg_workspace_size(GSG_OP_COMBINE, E, N, K, T, k) bytes, 16-byte aligned: the slots
  * bf16 [T*k][N] and then int32 counters [T][N/32] (the first two count the CTAs through the grid
  * barrier).  The counters must be zero before the first call (e.g. allocate the workspace zeroed);
- * every call that completes leaves them zero again, so a workspace can be reused call after call.  After a device error the outputs and the
- * counters are unspecified: zero the workspace again.  Calls that share a workspace must not run
- * concurrently.  The launch's CTAs (one per SM) wait for one another at the barrier: while another
+ * every call that completes leaves them zero again, so a workspace can be reused call after call.
+ * After a device error the outputs and the counters are unspecified: zero the workspace again.
+ * Calls that share a workspace must not run concurrently.  The launch's CTAs (one per SM) wait for one another at the barrier: while another
  * kernel keeps SMs busy on a concurrent stream, the CTAs already running wait for the rest, and a
  * wait longer than 2 s ends with GSG_ERR_DEVICE_TIMEOUT (outputs unspecified) instead of hanging.
  */
