@@ -246,9 +246,10 @@ gsg_status_t gsg_grouped_sparse_gemm_swiglu(const uint8_t* a_codes, const uint8_
  * barrier).  The counters must be zero before the first call (e.g. allocate the workspace zeroed);
  * every call that completes leaves them zero again, so a workspace can be reused call after call.
  * After a device error the outputs and the counters are unspecified: zero the workspace again.
- * Calls that share a workspace must not run concurrently.  The launch's CTAs (one per SM) wait for one another at the barrier: while another
- * kernel keeps SMs busy on a concurrent stream, the CTAs already running wait for the rest, and a
- * wait longer than 2 s ends with GSG_ERR_DEVICE_TIMEOUT (outputs unspecified) instead of hanging.
+ * Calls that share a workspace must not run concurrently.  The launch's CTAs (one per SM) wait
+ * for one another at the barrier: while another kernel keeps SMs busy on a concurrent stream, the
+ * CTAs already running wait for the rest, and a wait longer than 2 s ends with
+ * GSG_ERR_DEVICE_TIMEOUT (outputs unspecified) instead of hanging.
  */
 gsg_status_t gsg_grouped_sparse_gemm_combine(const uint8_t* a_codes, const uint8_t* a_scales,
                                              const float* x_tensor_scale,
